@@ -1,0 +1,359 @@
+"""CPU oracle for the MuScriptor KV-cached INT4 decoder step.
+
+TEST INFRASTRUCTURE ONLY.  This is the slow, plain reference that the CUDA
+library is checked against.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import it; the library never does, and the two share no
+code (the seeded input draws in ``synth`` are the only common module, and they
+hold none of the arithmetic below).
+
+Floating point: every activation, normalisation, softmax and dot product is
+computed in float64 (numpy; BLAS matmul as the one library primitive).  Two
+things are integer or fp32 decisions and are taken in fp32 on purpose, because
+the method fixes them there: the RTN INT4 quantiser (scale = absmax/7 and
+q = rint(w/scale), both IEEE fp32) and the dequantised weight value q*scale
+(one fp32 product).  The argmax is taken on the float64 logits, lowest index on
+ties.
+
+Sources (page title, section):
+  [W4A32]  "MuScriptor Medium — optimized W4A32 ONNX Runtime", sections
+           "Model variant" (INT4 g32 symmetric RTN backbone, fp32 activations,
+           cache, embeddings and LM head; 96 MatMulNBits, 24 GroupQueryAttention,
+           48 SkipLayerNormalization for 24 layers; fixed-capacity shared cache),
+           "Quick smoke test" (default cache length 2504, 469.5 MiB).
+  [ONNX-S] "MuScriptor small — ONNX conversion", section "muscriptor-small-lm.onnx"
+           (tokens i64 [1,S], prefix f32 [1,P,d] with P = 0 after the first
+           step, past_k/past_v [L,1,T,Hk,64], logits f32 [1,1393] last position
+           only, positions implicit from the cache length, one branch-free graph
+           for prefill and decode; greedy decoding).
+  [CARD]   "MuScriptor — small (≈100M)" model card, sections "Model description"
+           (decoder-only Transformer, spectrogram projected to d_model and used as
+           a prefix condition, greedy argmax decoding) and "Model variants".
+
+Readings where the pages are silent (each one is listed with its reason in the
+design notes of the repository):
+  * four backbone MatMuls per layer (96 / 24): fused QKV, O, FC1, FC2;
+  * pre-LayerNorm blocks, a final LayerNorm, eps 1e-5, biased variance;
+  * non-gated FFN of width d_ff with exact (erf) GELU;
+  * no biases on any MatMul or on the LM head;
+  * RoPE, base 1e4, on q and k at every position, pairs (i, i + 32) of each
+    64-wide head, angle pos * base^(-2i/64), rotation
+    (a, b) -> (a cos - b sin, a sin + b cos); the cache holds post-RoPE keys;
+  * fully causal attention over [prefix ; tokens], scale 1/sqrt(64), query head
+    h reads kv head h // (H / Hk);
+  * INT4 storage: u = q + 8 in a nibble, element 2i in the low nibble of byte i,
+    row-major [N][K/2] with row n = output feature n; scales fp32 [N][K/32].
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional, Sequence
+
+import numpy as np
+from scipy.special import erf as _erf
+
+GROUP = 32
+QMAX = 7
+
+
+# ---------------------------------------------------------------------------
+# INT4 weight format  [W4A32, "Model variant": symmetric RTN INT4, group size 32]
+# ---------------------------------------------------------------------------
+
+def quantize_int4_g32(w: np.ndarray):
+    """Symmetric round-to-nearest INT4 with one scale per 32 consecutive K elements.
+
+    ``w`` is fp32 [N, K] (row n = output feature n, K = input features).  For each
+    group: scale = absmax / 7 (fp32 division), q = clamp(rint(w / scale), -7, 7)
+    (fp32 division, round half to even).  An all-zero group has scale 0 and q 0.
+    Returns (q int8 [N, K], scale fp32 [N, K/32]).
+    """
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 32")
+    g = w.reshape(n, k // GROUP, GROUP)
+    absmax = np.max(np.abs(g), axis=2)                                    # fp32
+    scale = (absmax / np.float32(QMAX)).astype(np.float32)                # fp32 IEEE division
+    safe = np.where(scale == 0, np.float32(1), scale).astype(np.float32)
+    ratio = (g / safe[:, :, None]).astype(np.float32)                     # fp32 IEEE division
+    q = np.clip(np.rint(ratio), -QMAX, QMAX)
+    q = np.where(scale[:, :, None] == 0, 0, q).astype(np.int8)
+    return q.reshape(n, k), scale
+
+
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """Pack int8 q in [-8, 7] into bytes: u = q + 8, element 2i low nibble, 2i+1 high nibble."""
+    q = np.asarray(q)
+    n, k = q.shape
+    u = (q.astype(np.int16) + 8).astype(np.uint8)
+    lo = u[:, 0::2]
+    hi = u[:, 1::2]
+    return (lo | (hi << 4)).astype(np.uint8).reshape(n, k // 2)
+
+
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack_int4`: bytes [N, K/2] -> int8 q [N, K]."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    n, kh = packed.shape
+    q = np.empty((n, kh * 2), dtype=np.int8)
+    q[:, 0::2] = (packed & 0x0F).astype(np.int8) - 8
+    q[:, 1::2] = (packed >> 4).astype(np.int8) - 8
+    return q
+
+
+def dequantize(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """W[n, k] = q[n, k] * scale[n, k // 32], one fp32 product per element."""
+    n, k = q.shape
+    s = np.repeat(scale.astype(np.float32), GROUP, axis=1)
+    return (q.astype(np.float32) * s).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# Layer primitives (float64)
+# ---------------------------------------------------------------------------
+
+def layer_norm(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray, eps: float) -> np.ndarray:
+    """LayerNorm over the last axis: (x - mean) / sqrt(var + eps) * gamma + beta, biased var.
+
+    [W4A32, "Model variant"]: the SkipLayerNormalization nodes (residual add
+    followed by this normalisation).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(gamma, np.float64) + np.asarray(beta, np.float64)
+
+
+def gelu_erf(u: np.ndarray) -> np.ndarray:
+    """Exact GELU: 0.5 u (1 + erf(u / sqrt 2))."""
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1.0 + _erf(u / np.sqrt(2.0)))
+
+
+def rope(x: np.ndarray, positions: np.ndarray, base: float) -> np.ndarray:
+    """Rotary position embedding on [T, heads, 64], pairs (i, i + 32), angle pos * base^(-2i/64)."""
+    x = np.asarray(x, dtype=np.float64)
+    hd = x.shape[-1]
+    half = hd // 2
+    i = np.arange(half, dtype=np.float64)
+    theta = base ** (-2.0 * i / hd)                                       # [32]
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * theta[None, :]   # [T, 32]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a = x[..., :half]
+    b = x[..., half:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+              q_pos: np.ndarray, k_pos: np.ndarray) -> np.ndarray:
+    """Causal grouped-query attention.
+
+    q [Tq, H, 64], k and v [Tk, Hk, 64]; query i sees key j iff k_pos[j] <= q_pos[i].
+    Query head h reads kv head h // (H / Hk).  Scores scaled by 1/sqrt(64); softmax
+    with the row maximum subtracted.  Returns [Tq, H, 64].
+    [W4A32, "Model variant"]: GroupQueryAttention; [ONNX-S]: past_k/past_v heads.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    tq, h, hd = q.shape
+    hk = k.shape[1]
+    if h % hk:
+        raise ValueError("heads must be a multiple of kv heads")
+    rep = h // hk
+    visible = np.asarray(k_pos)[None, :] <= np.asarray(q_pos)[:, None]   # [Tq, Tk]
+    out = np.empty_like(q)
+    scale = 1.0 / np.sqrt(hd)
+    for hh in range(h):
+        g = hh // rep
+        s = (q[:, hh, :] @ k[:, g, :].T) * scale
+        s = np.where(visible, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        p /= p.sum(axis=1, keepdims=True)
+        out[:, hh, :] = p @ v[:, g, :]
+    return out
+
+
+def argmax_lowest(logits: np.ndarray) -> np.ndarray:
+    """Greedy choice: index of the maximum, lowest index on ties (over the last axis)."""
+    return np.argmax(np.asarray(logits), axis=-1)
+
+
+def top2_margin(logits: np.ndarray) -> np.ndarray:
+    """Largest minus second-largest logit (over the last axis)."""
+    part = np.sort(np.asarray(logits, np.float64), axis=-1)
+    return part[..., -1] - part[..., -2]
+
+
+# ---------------------------------------------------------------------------
+# Model
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class OracleLayer:
+    ln1_g: np.ndarray
+    ln1_b: np.ndarray
+    ln2_g: np.ndarray
+    ln2_b: np.ndarray
+    w: List[np.ndarray]                 # dequantised weights [N, K]: QKV, O, FC1, FC2
+    q: Optional[List[np.ndarray]] = None       # int8 codes (INT4 format only)
+    s: Optional[List[np.ndarray]] = None       # fp32 scales (INT4 format only)
+    packed: Optional[List[np.ndarray]] = None  # bytes (INT4 format only)
+
+
+class OracleModel:
+    """Decoder-only transformer of the pages, weights held dequantised.
+
+    ``weight_format`` "int4": every backbone matrix goes through
+    :func:`quantize_int4_g32` and :func:`dequantize` ([W4A32, "Model variant"]).
+    "fp16": every backbone matrix is rounded to IEEE half (the half-precision
+    weight variant of "MuScriptor for Core AI (.aimodel)", file table).  "fp32":
+    the matrices as drawn.  Embeddings, LayerNorms and the LM head stay fp32.
+    """
+
+    def __init__(self, draw, weight_format: str = "int4", store=np.float64):
+        sh = draw.shape
+        self.shape = sh
+        self.weight_format = weight_format
+        self.L, self.d, self.H, self.Hk = sh.n_layers, sh.d_model, sh.n_heads, sh.n_kv_heads
+        self.hd, self.F, self.V = sh.head_dim, sh.d_ff, sh.vocab
+        self.base, self.eps = sh.rope_base, sh.ln_eps
+        self.tok_emb = np.asarray(draw.tok_emb, np.float32)
+        self.lm_head = np.asarray(draw.lm_head, np.float64)
+        self.ln_f_g, self.ln_f_b = draw.ln_f_g, draw.ln_f_b
+        self.layers: List[OracleLayer] = []
+        for ld in draw.layers:
+            ws, qs, ss, ps = [], [], [], []
+            for w in ld.w:
+                if weight_format == "int4":
+                    q, s = quantize_int4_g32(w)
+                    qs.append(q)
+                    ss.append(s)
+                    ps.append(pack_int4(q))
+                    ws.append(dequantize(q, s).astype(store))
+                elif weight_format == "fp16":
+                    ws.append(np.asarray(w, np.float32).astype(np.float16).astype(store))
+                elif weight_format == "fp32":
+                    ws.append(np.asarray(w, np.float32).astype(store))
+                else:
+                    raise ValueError(weight_format)
+            self.layers.append(OracleLayer(ld.ln1_g, ld.ln1_b, ld.ln2_g, ld.ln2_b, ws,
+                                           qs or None, ss or None, ps or None))
+
+    # -- one pass over new rows, attending to the cache plus themselves --------
+    def _run(self, x: np.ndarray, cache: "OracleCache", all_logits: bool) -> np.ndarray:
+        """Append the rows ``x`` [n, d] (in sequence order) to ``cache`` and return logits.
+
+        Positions are implicit: the new rows take positions T..T+n-1 where T is the
+        cache length ([ONNX-S]).  Returns logits of every new row if ``all_logits``
+        else of the last row only.
+        """
+        n = x.shape[0]
+        t0 = cache.length
+        if t0 + n > cache.capacity:
+            raise ValueError("cache capacity exceeded")
+        pos = np.arange(t0, t0 + n)
+        kpos = np.arange(t0 + n)
+        H, Hk, hd = self.H, self.Hk, self.hd
+        x = np.asarray(x, np.float64)
+        for l, ly in enumerate(self.layers):
+            h = layer_norm(x, ly.ln1_g, ly.ln1_b, self.eps)
+            qkv = h @ ly.w[0].T
+            q = qkv[:, : H * hd].reshape(n, H, hd)
+            k = qkv[:, H * hd: (H + Hk) * hd].reshape(n, Hk, hd)
+            v = qkv[:, (H + Hk) * hd:].reshape(n, Hk, hd)
+            q = rope(q, pos, self.base)
+            k = rope(k, pos, self.base)
+            cache.k[l][t0: t0 + n] = k
+            cache.v[l][t0: t0 + n] = v
+            a = attention(q, cache.k[l][: t0 + n], cache.v[l][: t0 + n], pos, kpos)
+            x = x + a.reshape(n, H * hd) @ ly.w[1].T
+            h = layer_norm(x, ly.ln2_g, ly.ln2_b, self.eps)
+            x = x + gelu_erf(h @ ly.w[2].T) @ ly.w[3].T
+        cache.length = t0 + n
+        rows = x if all_logits else x[-1:]
+        y = layer_norm(rows, self.ln_f_g, self.ln_f_b, self.eps)
+        logits = y @ self.lm_head.T
+        return logits if all_logits else logits[0]
+
+    def embed(self, tokens: Sequence[int]) -> np.ndarray:
+        tokens = np.asarray(tokens, dtype=np.int64).reshape(-1)
+        if tokens.size and (tokens.min() < 0 or tokens.max() >= self.V):
+            raise ValueError("token id out of range")
+        return self.tok_emb[tokens].astype(np.float64)
+
+    def sequence(self, prefix: Optional[np.ndarray], tokens: Sequence[int]) -> np.ndarray:
+        """[prefix ; E[tokens]]: the prefix rows come first ([ONNX-S]; [CARD] prefix condition)."""
+        e = self.embed(tokens)
+        if prefix is None or len(prefix) == 0:
+            return e
+        return np.concatenate([np.asarray(prefix, np.float64), e], axis=0)
+
+    def new_cache(self, capacity: int) -> "OracleCache":
+        return OracleCache(self.L, self.Hk, self.hd, capacity)
+
+    # -- mode (i): full recompute ------------------------------------------------
+    def forward_full(self, prefix: Optional[np.ndarray], tokens: Sequence[int]):
+        """Logits at every position of [prefix ; tokens] with no prior cache: [P+S, V]."""
+        x = self.sequence(prefix, tokens)
+        cache = self.new_cache(x.shape[0])
+        return self._run(x, cache, all_logits=True), cache
+
+    # -- mode (ii): incremental with a cache --------------------------------------
+    def prefill(self, cache: "OracleCache", prefix: Optional[np.ndarray], tokens: Sequence[int]) -> np.ndarray:
+        """Append [prefix ; tokens] to the cache; return last-position logits [V]."""
+        return self._run(self.sequence(prefix, tokens), cache, all_logits=False)
+
+    def decode_step(self, cache: "OracleCache", token: int) -> np.ndarray:
+        """Append one token; return its logits [V]."""
+        return self._run(self.embed([token]), cache, all_logits=False)
+
+    def greedy(self, prefix, start_token: int, n_steps: int, capacity: int):
+        """Prefill [prefix ; start], then ``n_steps`` greedy steps feeding the argmax back.
+
+        Returns (tokens int64 [n_steps + 1], logits float64 [n_steps + 1, V]): row 0
+        is the prefill's last-position output, row i the output of decode step i.
+        """
+        cache = self.new_cache(capacity)
+        logits = [self.prefill(cache, prefix, [start_token])]
+        toks = [int(argmax_lowest(logits[-1]))]
+        for _ in range(n_steps):
+            logits.append(self.decode_step(cache, toks[-1]))
+            toks.append(int(argmax_lowest(logits[-1])))
+        return np.array(toks, np.int64), np.stack(logits)
+
+    def teacher_forced(self, prefix, tokens: Sequence[int]) -> np.ndarray:
+        """Logits after the prefill and after every forced token: [len(tokens), V].
+
+        Row 0 is the output at the first token's position, row i the output at
+        token i's position; the same rows a prefill of (prefix, tokens[0]) followed
+        by decode steps over tokens[1:] returns.
+        """
+        logits, _ = self.forward_full(prefix, tokens)
+        p = 0 if prefix is None else len(prefix)
+        return logits[p:]
+
+    def param_count(self) -> int:
+        n = 2 * self.V * self.d + self.d * 2
+        for ly in self.layers:
+            n += sum(w.size for w in ly.w) + 4 * self.d
+        return n
+
+
+class OracleCache:
+    """Post-RoPE keys and values, [L][capacity, Hk, 64] each, plus the current length."""
+
+    def __init__(self, n_layers: int, n_kv_heads: int, head_dim: int, capacity: int):
+        self.capacity = capacity
+        self.length = 0
+        self.k = [np.zeros((capacity, n_kv_heads, head_dim)) for _ in range(n_layers)]
+        self.v = [np.zeros((capacity, n_kv_heads, head_dim)) for _ in range(n_layers)]
+
+    def export(self):
+        """The pages' cache layout [L, 1, T, Hk, 64] ([ONNX-S] past_k / past_v)."""
+        t = self.length
+        k = np.stack([kk[:t] for kk in self.k])[:, None]
+        v = np.stack([vv[:t] for vv in self.v])[:, None]
+        return k, v

@@ -1,0 +1,452 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself.  Each test ties one part of it to
+a hand-worked example, a figure the pages print, a closed form, an invariant,
+brute force on tiny inputs, or a special case that reduces to a library routine
+(torch's layer_norm, gelu and scaled_dot_product_attention).  The last test
+plants mistakes in the oracle (on the CPU) and checks that the pins catch them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import synth
+from oracle import ms_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# INT4 g32
+# ----------------------------------------------------------------------------
+
+def test_int4_hand_example():
+    g = _gold("int4_g32_hand.json")
+    w = np.zeros((1, 32 * len(g["groups"])), np.float32)
+    for i, grp in enumerate(g["groups"]):
+        w[0, 32 * i: 32 * i + len(grp["w_head"])] = grp["w_head"]
+    q, s = O.quantize_int4_g32(w)
+    packed = O.pack_int4(q)
+    for i, grp in enumerate(g["groups"]):
+        assert s[0, i] == np.float32(grp["scale"])
+        assert list(q[0, 32 * i: 32 * i + 8]) == grp["q_head"]
+        assert np.all(q[0, 32 * i + 8: 32 * i + 32] == 0)
+        assert list(packed[0, 16 * i: 16 * i + 16]) == grp["bytes"]
+
+
+def test_pack_unpack_roundtrip_all_bytes():
+    b = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    q = O.unpack_int4(b)
+    assert q.min() == -8 and q.max() == 7
+    assert np.array_equal(O.pack_int4(q), b)
+    allq = np.array([[a, c] for a in range(-8, 8) for c in range(-8, 8)], np.int8).reshape(1, -1)
+    assert np.array_equal(O.unpack_int4(O.pack_int4(allq)), allq)
+
+
+def test_pack_nibble_order_bruteforce():
+    rng = np.random.default_rng(5)
+    q = rng.integers(-7, 8, size=(3, 64)).astype(np.int8)
+    p = O.pack_int4(q)
+    for n in range(3):
+        for i in range(32):
+            byte = int(p[n, i])
+            assert (byte & 15) - 8 == q[n, 2 * i]
+            assert (byte >> 4) - 8 == q[n, 2 * i + 1]
+
+
+def test_quantize_error_bound_and_extremes():
+    w = synth.make_matrix(48, 256, seed=11)
+    q, s = O.quantize_int4_g32(w)
+    assert q.min() >= -7 and q.max() <= 7
+    deq = O.dequantize(q, s).astype(np.float64)
+    sfull = np.repeat(s, 32, axis=1).astype(np.float64)
+    # |w - q s| <= s / 2 up to the fp32 rounding of the division and of the product
+    assert np.all(np.abs(w - deq) <= sfull * (0.5 + 1e-5) + 1e-12)
+    # the largest magnitude of every group maps to +-7
+    g = np.abs(w.reshape(48, 8, 32))
+    idx = g.argmax(axis=2)
+    qg = q.reshape(48, 8, 32)
+    picked = np.take_along_axis(qg, idx[..., None], axis=2)[..., 0]
+    assert np.all(np.abs(picked) == 7)
+    # no exact ties in continuous random draws (tie rule is then immaterial)
+    r = (w.reshape(48, 8, 32) / s[..., None]).astype(np.float32)
+    assert not np.any(np.abs(r - np.floor(r)) == 0.5)
+
+
+def test_quantize_sign_flip_invariance():
+    w = synth.make_matrix(8, 128, seed=12)
+    q1, s1 = O.quantize_int4_g32(w)
+    q2, s2 = O.quantize_int4_g32(-w)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(q1, -q2)
+    # scaling a group by a power of two scales its scale and keeps its codes
+    q3, s3 = O.quantize_int4_g32(w * np.float32(4.0))
+    assert np.array_equal(q1, q3) and np.array_equal(s1 * 4, s3)
+
+
+def test_dequant_matmul_bruteforce():
+    w = synth.make_matrix(3, 64, seed=13)
+    x = synth.make_activations(2, 64, seed=14)
+    q, s = O.quantize_int4_g32(w)
+    packed = O.pack_int4(q)
+    got = x.astype(np.float64) @ O.dequantize(q, s).astype(np.float64).T
+    for m in range(2):
+        for n in range(3):
+            acc = 0.0
+            for k in range(64):
+                byte = int(packed[n, k // 2])
+                u = (byte >> 4) if (k & 1) else (byte & 15)
+                wk = float(np.float32(np.float32(u - 8) * s[n, k // 32]))
+                acc += float(x[m, k]) * wk
+            assert abs(acc - got[m, n]) <= 1e-12 * (1 + abs(acc))
+
+
+# ----------------------------------------------------------------------------
+# Layer primitives
+# ----------------------------------------------------------------------------
+
+def test_layer_norm_closed_form_and_library():
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    eps = 1e-5
+    want = (x - 2.5) / math.sqrt(1.25 + eps)
+    assert np.allclose(O.layer_norm(x, np.ones(4), np.zeros(4), eps), want, rtol=0, atol=1e-15)
+    c = np.full((1, 16), 3.25)
+    beta = np.linspace(-1, 1, 16)
+    assert np.allclose(O.layer_norm(c, np.ones(16) * 2.0, beta, eps), beta, atol=1e-15)
+    xr = synth.make_activations(5, 96, seed=15).astype(np.float64) * 3 + 1
+    gm = 1 + 0.1 * synth.make_activations(1, 96, seed=16)[0].astype(np.float64)
+    bt = 0.1 * synth.make_activations(1, 96, seed=17)[0].astype(np.float64)
+    lib = F.layer_norm(torch.from_numpy(xr), (96,), torch.from_numpy(gm), torch.from_numpy(bt), eps).numpy()
+    assert np.allclose(O.layer_norm(xr, gm, bt, eps), lib, rtol=0, atol=1e-13)
+    h = O.layer_norm(xr, np.ones(96), np.zeros(96), eps)
+    assert np.allclose(h.mean(axis=1), 0, atol=1e-14)
+    assert np.allclose(h.var(axis=1), 1.0, atol=1e-4)
+
+
+def test_gelu_closed_forms_and_library():
+    assert O.gelu_erf(np.array([0.0]))[0] == 0.0
+    # Phi(1) = 0.841344746068542948585232545632...
+    assert abs(O.gelu_erf(np.array([1.0]))[0] - 0.8413447460685429) < 1e-15
+    u = np.linspace(-6, 6, 97)
+    assert np.allclose(O.gelu_erf(u) - O.gelu_erf(-u), u, atol=1e-14)
+    lib = F.gelu(torch.from_numpy(u), approximate="none").numpy()
+    assert np.allclose(O.gelu_erf(u), lib, atol=1e-14)
+
+
+def test_rope_identity_norm_and_unit_vectors():
+    x = synth.make_activations(4, 3 * 64, seed=18).astype(np.float64).reshape(4, 3, 64)
+    assert np.array_equal(O.rope(x, np.zeros(4), 1e4), x)
+    pos = np.array([1, 7, 100, 2503])
+    y = O.rope(x, pos, 1e4)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+    # unit vector e_i at position p lands on (cos p*theta_i, sin p*theta_i) at (i, i+32)
+    for i in (0, 1, 13, 31):
+        e = np.zeros((1, 1, 64))
+        e[0, 0, i] = 1.0
+        p = 37
+        th = 1e4 ** (-2.0 * i / 64)
+        r = O.rope(e, np.array([p]), 1e4)[0, 0]
+        assert abs(r[i] - math.cos(p * th)) < 1e-14 and abs(r[i + 32] - math.sin(p * th)) < 1e-14
+        assert np.count_nonzero(np.abs(r) > 1e-15) <= 2
+        e2 = np.zeros((1, 1, 64))
+        e2[0, 0, i + 32] = 1.0
+        r2 = O.rope(e2, np.array([p]), 1e4)[0, 0]
+        assert abs(r2[i] + math.sin(p * th)) < 1e-14 and abs(r2[i + 32] - math.cos(p * th)) < 1e-14
+
+
+def test_rope_relative_position():
+    q = synth.make_activations(1, 64, seed=19).astype(np.float64).reshape(1, 1, 64)
+    k = synth.make_activations(1, 64, seed=20).astype(np.float64).reshape(1, 1, 64)
+    dots = []
+    for p0 in (0, 5, 123, 1999):
+        rq = O.rope(q, np.array([p0 + 9]), 1e4)
+        rk = O.rope(k, np.array([p0]), 1e4)
+        dots.append(float((rq * rk).sum()))
+    assert np.allclose(dots, dots[0], rtol=1e-10)
+
+
+def _attention_bruteforce(q, k, v, qpos, kpos):
+    tq, h, hd = q.shape
+    hk = k.shape[1]
+    out = np.zeros_like(q)
+    for i in range(tq):
+        for hh in range(h):
+            g = hh // (h // hk)
+            sc = []
+            for j in range(k.shape[0]):
+                if kpos[j] <= qpos[i]:
+                    sc.append((j, sum(q[i, hh, c] * k[j, g, c] for c in range(hd)) / 8.0))
+            m = max(s for _, s in sc)
+            w = [(j, math.exp(s - m)) for j, s in sc]
+            z = sum(e for _, e in w)
+            for j, e in w:
+                out[i, hh] += (e / z) * v[j, g]
+    return out
+
+
+@pytest.mark.parametrize("h,hk", [(1, 1), (2, 1), (4, 2), (4, 1), (2, 2)])
+def test_attention_bruteforce(h, hk):
+    tq, tk = 3, 6
+    q = synth.make_activations(tq, h * 64, seed=21).astype(np.float64).reshape(tq, h, 64)
+    k = synth.make_activations(tk, hk * 64, seed=22).astype(np.float64).reshape(tk, hk, 64)
+    v = synth.make_activations(tk, hk * 64, seed=23).astype(np.float64).reshape(tk, hk, 64)
+    qpos = np.array([3, 4, 5])
+    kpos = np.arange(tk)
+    got = O.attention(q, k, v, qpos, kpos)
+    want = _attention_bruteforce(q, k, v, qpos, kpos)
+    assert np.allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_attention_special_cases():
+    # one visible key: the output is that value exactly
+    q = synth.make_activations(1, 128, seed=24).astype(np.float64).reshape(1, 2, 64)
+    k = synth.make_activations(4, 64, seed=25).astype(np.float64).reshape(4, 1, 64)
+    v = synth.make_activations(4, 64, seed=26).astype(np.float64).reshape(4, 1, 64)
+    out = O.attention(q, k, v, np.array([0]), np.arange(4))
+    assert np.array_equal(out[0, 0], v[0, 0]) and np.array_equal(out[0, 1], v[0, 0])
+    # kv heads = heads, and GQA: torch's scaled_dot_product_attention (causal)
+    for h, hk in ((3, 3), (4, 2), (6, 1)):
+        t = 9
+        q = synth.make_activations(t, h * 64, seed=27).astype(np.float64).reshape(t, h, 64)
+        k = synth.make_activations(t, hk * 64, seed=28).astype(np.float64).reshape(t, hk, 64)
+        v = synth.make_activations(t, hk * 64, seed=29).astype(np.float64).reshape(t, hk, 64)
+        lib = F.scaled_dot_product_attention(
+            torch.from_numpy(q).permute(1, 0, 2)[None], torch.from_numpy(k).permute(1, 0, 2)[None],
+            torch.from_numpy(v).permute(1, 0, 2)[None], is_causal=True, enable_gqa=(h != hk))
+        lib = lib[0].permute(1, 0, 2).numpy()
+        assert np.allclose(O.attention(q, k, v, np.arange(t), np.arange(t)), lib, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# Whole model
+# ----------------------------------------------------------------------------
+
+def _tiny_model(L=2, h=2, hk=1, ln_random=True, fmt="int4", vocab=37):
+    sh = synth.tiny_shape(n_layers=L, n_heads=h, n_kv_heads=hk, vocab=vocab)
+    draw = synth.make_weights(sh, seed=31, std=0.08, ln_random=ln_random)
+    return O.OracleModel(draw, fmt)
+
+
+def _torch_library_forward(m, prefix, tokens):
+    """The same decoder assembled from torch library routines in float64.
+
+    RoPE is written as a complex rotation (a + ib) * exp(i p theta) of each
+    (i, i + 32) pair, attention is torch's causal scaled_dot_product_attention
+    with grouped KV heads, LayerNorm and GELU are torch's.
+    """
+    x = torch.from_numpy(m.sequence(prefix, tokens))
+    n = x.shape[0]
+    H, Hk, hd = m.H, m.Hk, m.hd
+    pos = torch.arange(n, dtype=torch.float64)
+    theta = m.base ** (-torch.arange(0, hd, 2, dtype=torch.float64) / hd)
+    rot = torch.polar(torch.ones(n, hd // 2, dtype=torch.float64), pos[:, None] * theta[None])
+
+    def rope_c(t):  # t [n, heads, 64]
+        z = torch.complex(t[..., : hd // 2], t[..., hd // 2:]) * rot[:, None, :]
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    def ln(t, g, b):
+        return F.layer_norm(t, (m.d,), torch.from_numpy(np.asarray(g, np.float64)),
+                            torch.from_numpy(np.asarray(b, np.float64)), m.eps)
+
+    for ly in m.layers:
+        W = [torch.from_numpy(w.astype(np.float64)) for w in ly.w]
+        h = ln(x, ly.ln1_g, ly.ln1_b)
+        qkv = F.linear(h, W[0])
+        q = rope_c(qkv[:, : H * hd].reshape(n, H, hd))
+        k = rope_c(qkv[:, H * hd: (H + Hk) * hd].reshape(n, Hk, hd))
+        v = qkv[:, (H + Hk) * hd:].reshape(n, Hk, hd)
+        a = F.scaled_dot_product_attention(q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None],
+                                           v.permute(1, 0, 2)[None], is_causal=True,
+                                           enable_gqa=(H != Hk))[0].permute(1, 0, 2)
+        x = x + F.linear(a.reshape(n, H * hd), W[1])
+        h = ln(x, ly.ln2_g, ly.ln2_b)
+        x = x + F.linear(F.gelu(F.linear(h, W[2]), approximate="none"), W[3])
+    y = ln(x, m.ln_f_g, m.ln_f_b)
+    return F.linear(y, torch.from_numpy(m.lm_head)).numpy()
+
+
+@pytest.mark.parametrize("h,hk,fmt", [(2, 1, "int4"), (2, 2, "int4"), (4, 2, "fp16")])
+def test_model_matches_torch_library_assembly(h, hk, fmt):
+    m = _tiny_model(L=2, h=h, hk=hk, fmt=fmt)
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=5, seed=32)[0]
+    toks = synth.make_token_sequence(4, 1, vocab=m.V, seed=33)[0]
+    got, _ = m.forward_full(prefix, toks)
+    want = _torch_library_forward(m, prefix, toks)
+    assert got.shape == (9, m.V)
+    assert np.allclose(got, want, rtol=0, atol=1e-11)
+
+
+def test_incremental_equals_full_recompute():
+    m = _tiny_model(L=2, h=4, hk=2)
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=6, seed=34)[0]
+    toks = synth.make_token_sequence(7, 1, vocab=m.V, seed=35)[0]
+    full, full_cache = m.forward_full(prefix, toks)
+    cache = m.new_cache(32)
+    rows = [m.prefill(cache, prefix, toks[:1])]
+    for t in toks[1:]:
+        rows.append(m.decode_step(cache, int(t)))
+    inc = np.stack(rows)
+    assert np.allclose(inc, full[6:], rtol=0, atol=1e-12)
+    ki, vi = cache.export()
+    kf, vf = full_cache.export()
+    assert np.allclose(ki, kf, atol=1e-12) and np.allclose(vi, vf, atol=1e-12)
+    # prefill in two calls (prefix first, then tokens with no prefix) is the same sequence
+    c2 = m.new_cache(32)
+    m.prefill(c2, prefix, [])
+    last = m.prefill(c2, None, toks)
+    assert np.allclose(last, full[-1], atol=1e-12)
+
+
+def test_causality():
+    m = _tiny_model(L=2, h=2, hk=1)
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=4, seed=36)[0]
+    toks = synth.make_token_sequence(6, 1, vocab=m.V, seed=37)[0]
+    a, _ = m.forward_full(prefix, toks)
+    toks2 = toks.copy()
+    toks2[4] = (toks2[4] + 5) % m.V
+    b, _ = m.forward_full(prefix, toks2)
+    assert np.array_equal(a[: 4 + 4], b[: 4 + 4])
+    assert not np.allclose(a[8], b[8])
+
+
+def test_shapes_per_step_follow_the_pages():
+    figs = _gold("pages_figures.json")
+    m = _tiny_model(L=3, h=2, hk=1, vocab=figs["vocab"]["value"])
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=7, seed=38)[0]
+    cache = m.new_cache(16)
+    logits = m.prefill(cache, prefix, [5])
+    assert logits.shape == (figs["vocab"]["value"],)
+    k, v = cache.export()
+    assert k.shape == (3, 1, 8, 1, 64) and v.shape == k.shape          # [L, 1, T, Hk, 64]
+    m.decode_step(cache, int(O.argmax_lowest(logits)))
+    assert cache.export()[0].shape == (3, 1, 9, 1, 64)
+    with pytest.raises(ValueError):
+        m.prefill(cache, prefix, [1])                                   # 9 + 8 > 16: no room
+
+
+def test_zero_layers_is_embedding_then_head():
+    sh = synth.tiny_shape(n_layers=0, vocab=29)
+    draw = synth.make_weights(sh, seed=39, std=0.1, ln_random=True)
+    m = O.OracleModel(draw, "int4")
+    logits = m.prefill(m.new_cache(4), None, [17])
+    e = [float(t) for t in draw.tok_emb[17]]
+    mu = sum(e) / len(e)
+    var = sum((t - mu) ** 2 for t in e) / len(e)
+    y = [(t - mu) / math.sqrt(var + 1e-5) * float(g) + float(b) for t, g, b in zip(e, draw.ln_f_g, draw.ln_f_b)]
+    want = [sum(yy * float(w) for yy, w in zip(y, row)) for row in draw.lm_head]
+    assert np.allclose(logits, want, atol=1e-12)
+
+
+def test_residual_passthrough_when_block_outputs_vanish():
+    sh = synth.tiny_shape(n_layers=2, vocab=23)
+    draw = synth.make_weights(sh, seed=40, std=0.1, ln_random=True)
+    for ly in draw.layers:
+        ly.w[1][:] = 0.0      # W_o
+        ly.w[3][:] = 0.0      # W_2
+    m = O.OracleModel(draw, "int4")
+    prefix = synth.make_prefix(sh, 1, prefix_len=3, seed=41)[0]
+    logits = m.prefill(m.new_cache(8), prefix, [4, 9])
+    y = O.layer_norm(draw.tok_emb[9].astype(np.float64), draw.ln_f_g, draw.ln_f_b, 1e-5)
+    assert np.allclose(logits, y @ draw.lm_head.astype(np.float64).T, atol=1e-12)
+
+
+def test_param_counts_and_cache_size_match_the_pages():
+    figs = _gold("pages_figures.json")
+    for name, (d, h, L) in figs["variants"]["value"].items():
+        # page-faithful attention: kv heads = heads (small page: past_k has 12 heads)
+        sh = synth.Shape(name, L, d, h, h, 4 * d)
+        n = 2 * sh.vocab * d + sum(nn * kk for nn, kk in sh.matmul_shapes()) * L + (4 * L + 2) * d
+        lo, hi = figs["params"]["value"][name]
+        assert 0.97 * lo <= n <= 1.03 * hi, (name, n)
+    assert figs["medium_ops"]["value"]["MatMulNBits"] == 4 * figs["medium_ops"]["value"]["layers"]
+    # the medium cache at 2504 positions with 16 kv heads of 64, K and V, fp32
+    nbytes = 2 * 24 * 2504 * 16 * 64 * 4
+    assert round(nbytes / 2 ** 20, 1) == figs["medium_cache_mib_at_2504"]["value"]
+    c = O.OracleCache(24, 16, 64, 2504)
+    assert 2 * sum(k.size for k in c.k) * 4 == nbytes
+    assert list(figs["small_past_k"]["value"][:2]) == [synth.SMALL.n_layers, 1]
+    assert figs["small_past_k"]["value"][3:] == [synth.SMALL.n_kv_heads, synth.HEAD_DIM]
+    assert figs["prefix_rows"]["value"] == synth.PREFIX_LEN
+
+
+def test_greedy_feeds_argmax_back():
+    m = _tiny_model(L=1, h=2, hk=1)
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=3, seed=42)[0]
+    toks, logits = m.greedy(prefix, 3, 5, capacity=16)
+    assert toks.shape == (6,) and logits.shape == (6, m.V)
+    forced = m.teacher_forced(prefix, [3] + list(toks[:-1]))
+    assert np.allclose(forced, logits, atol=1e-12)
+    assert np.array_equal(O.argmax_lowest(forced), toks)
+    tie = np.array([0.5, 2.0, 2.0, -1.0])
+    assert O.argmax_lowest(tie) == 1
+
+
+# ----------------------------------------------------------------------------
+# Planted mistakes: each must be caught by at least one pin above
+# ----------------------------------------------------------------------------
+
+_ORIG_ROPE = O.rope
+
+
+def _rope_wrong_sign(x, positions, base):
+    return _ORIG_ROPE(x, -np.asarray(positions), base)
+
+
+def _rope_interleaved(x, positions, base):
+    y = np.asarray(x, np.float64).copy()
+    a, b = y[..., 0::2].copy(), y[..., 1::2].copy()
+    ang = np.asarray(positions, np.float64)[:, None] * base ** (-2.0 * np.arange(32) / 64)
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    y[..., 0::2], y[..., 1::2] = a * c - b * s, a * s + b * c
+    return y
+
+
+def _ln_unbiased(x, g, b, eps):
+    x = np.asarray(x, np.float64)
+    mu = x.mean(-1, keepdims=True)
+    return (x - mu) / np.sqrt(x.var(-1, ddof=1, keepdims=True) + eps) * g + b
+
+
+def _gelu_tanh(u):
+    u = np.asarray(u, np.float64)
+    return 0.5 * u * (1 + np.tanh(np.sqrt(2 / np.pi) * (u + 0.044715 * u ** 3)))
+
+
+def _attention_interleaved_groups(q, k, v, qp, kp):
+    h, hk = q.shape[1], k.shape[1]
+    perm = np.array([hh % hk for hh in range(h)])     # h -> h mod Hk instead of h // (H/Hk)
+    kk = k[:, perm, :]
+    vv = v[:, perm, :]
+    return _ORIG_ATT(q, kk, vv, qp, kp)
+
+
+_ORIG_ATT = O.attention
+
+
+@pytest.mark.parametrize("name,patch", [
+    ("rope sign", ("rope", _rope_wrong_sign)),
+    ("rope pairing", ("rope", _rope_interleaved)),
+    ("layernorm variance", ("layer_norm", _ln_unbiased)),
+    ("gelu variant", ("gelu_erf", _gelu_tanh)),
+    ("kv head mapping", ("attention", _attention_interleaved_groups)),
+])
+def test_planted_mistakes_are_caught(monkeypatch, name, patch):
+    attr, fn = patch
+    m = _tiny_model(L=2, h=4, hk=2, fmt="int4")
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=5, seed=43)[0]
+    toks = synth.make_token_sequence(4, 1, vocab=m.V, seed=44)[0]
+    want = _torch_library_forward(m, prefix, toks)
+    monkeypatch.setattr(O, attr, fn)
+    got, _ = m.forward_full(prefix, toks)
+    assert not np.allclose(got, want, rtol=0, atol=1e-6), name
