@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of the MuScriptor KV-cached INT4 decoder step on B200.
+
+One step = one pass of the whole decoder path over one synthetic input: reset the cache,
+prefill [prefix (503 rows) ; start token] (504 positions), then greedy decode
+(argmax fed back) for the workload's number of steps, through the library's C ABI
+(ms_prefill + ms_generate).  Default workload: the medium shape (24 layers, d 1024, 16
+heads with 4 kv heads, d_ff 4096, INT4 g32 backbone), batch 1, 2000 decode steps in a
+2504-position cache.  Weights and inputs are seeded synthetic draws (synth module).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent replica on
+its own GPU (the decoder does not shard); `value` sums all ranks' tokens over the slowest
+rank's time.  `--impl reference` times the CPU oracle on this host's cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "decode ms/token & tokens/s (b=1, batched), prefill ms; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="c3", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-decode-steps", type=int, default=16,
+                    help="decode steps in the oracle's timed sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _config_json(wl: synth.Workload, world: int):
+    sh = wl.shape
+    return {
+        "workload": (f"{wl.name}: L{sh.n_layers} d{sh.d_model} H{sh.n_heads}/Hk{sh.n_kv_heads} F{sh.d_ff} "
+                     f"V{sh.vocab} {wl.weight_format} backbone, batch {wl.batch}, prefill {wl.prefix_len}+1, "
+                     f"{wl.decode_steps} greedy decode steps, cache {wl.capacity}"),
+        "batch_per_gpu": wl.batch,
+        "prefill_rows": wl.prefix_len + 1,
+        "decode_steps": wl.decode_steps,
+        "cache_capacity": wl.capacity,
+        "l2": "weights+cache larger than L2; L2 flushed (256 MiB write) before every timed step",
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
+
+
+def _decode_bytes_per_token(wl: synth.Workload):
+    """Algorithmic bytes of one decode step per stream set: backbone weights (+ scales for
+    INT4), LM head, one embedding row per stream, and K and V over every cached position.
+    Returns (weight bytes per step, list of KV bytes per step over the run)."""
+    sh = wl.shape
+    w = 0
+    for (n, k) in sh.matmul_shapes():
+        w += n * k // 2 + n * (k // 32) * 4 if wl.weight_format == "int4" else n * k * 2
+    w *= sh.n_layers
+    w += sh.vocab * sh.d_model * 4 + wl.batch * sh.d_model * 4
+    p0 = wl.prefix_len + 1
+    kv = [2 * sh.n_layers * wl.batch * sh.n_kv_heads * (p0 + i + 1) * 64 * 4 for i in range(wl.decode_steps)]
+    return w, kv
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _gpu_id(torch, dev: int) -> str:
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+def _oracle_sample(wl: synth.Workload, n_decode: int):
+    """Time the CPU oracle on a bounded sample of the workload: prefill of stream 0 and
+    n_decode greedy steps.  Returns (tokens/s, seconds, threads, sample description)."""
+    from oracle import ms_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    draw = synth.make_weights(wl.shape, seed=0)
+    om = O.OracleModel(draw, wl.weight_format)
+    prefix = synth.make_prefix(wl.shape, 1, wl.prefix_len, seed=1)[0]
+    start = int(synth.make_start_tokens(1, seed=2)[0])
+    t0 = time.perf_counter()
+    om.greedy(prefix, start, n_decode, capacity=wl.prefix_len + 1 + n_decode)
+    dt = time.perf_counter() - t0
+    sample = (f"oracle (numpy fp64) on stream 0: prefill {wl.prefix_len}+1 rows then {n_decode} greedy "
+              f"decode steps; tokens/s = {n_decode + 1} tokens / time")
+    return (n_decode + 1) / dt, dt, threads, sample, om, draw
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[a.workload]
+    from oracle import ms_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    draw = synth.make_weights(wl.shape, seed=0)
+    om = O.OracleModel(draw, wl.weight_format)
+    prefix = synth.make_prefix(wl.shape, 1, wl.prefix_len, seed=1)[0]
+    start = int(synth.make_start_tokens(1, seed=2)[0])
+    n_dec = a.cpu_decode_steps
+    times = []
+    for i in range(a.warmup + a.steps):
+        t0 = time.perf_counter()
+        om.greedy(prefix, start, n_dec, capacity=wl.prefix_len + 1 + n_dec)
+        if i >= a.warmup:
+            times.append(time.perf_counter() - t0)
+    step = statistics.mean(times)
+    value = (n_dec + 1) * wl.batch / step if wl.batch == 1 else (n_dec + 1) / step
+    sample = (f"each step: oracle prefill {wl.prefix_len}+1 rows and {n_dec} greedy decode steps of stream 0 "
+              f"(a bounded sample of the workload)")
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config_json(wl, 1),
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_transformer_int4_b200 as ms
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = synth.WORKLOADS[a.workload]
+    sh, B = wl.shape, wl.batch
+
+    draw = synth.make_weights(sh, seed=0)
+    model = ms.Model.from_draw(draw, wl.weight_format, device=local)
+    del draw
+    prefix_h = torch.from_numpy(synth.make_prefix(sh, B, wl.prefix_len, seed=1)).pin_memory()
+    start_h = torch.from_numpy(synth.make_start_tokens(B, seed=2).reshape(B, 1)).pin_memory()
+    prefix = prefix_h.to(dev)
+    start = start_h.to(dev)
+    cache = ms.Cache(model, B, wl.capacity)
+    out_tok = torch.empty((wl.decode_steps, B), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(e0=None, e1=None, e2=None):
+        cache.reset()
+        flush.zero_()
+        if e0 is not None:
+            e0.record(stream)
+        cache.prefill(start, prefix)
+        if e1 is not None:
+            e1.record(stream)
+        cache.generate(wl.decode_steps, out_tokens=out_tok, logits=False)
+        if e2 is not None:
+            e2.record(stream)
+
+    for _ in range(a.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    assert cache.device_status() == ms.MS_OK
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
+    sampler = ClockSampler(_gpu_id(torch, local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    launches0 = cache.kernel_launches
+    t_wall = time.perf_counter()
+    for i in range(a.steps):
+        one_step(*ev[i])
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    launches = cache.kernel_launches - launches0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    assert cache.device_status() == ms.MS_OK
+
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens_per_step = B * (wl.decode_steps + 1)
+    value = world * tokens_per_step * a.steps / (total_ms / 1e3)
+    per_tok = [d / wl.decode_steps for d in dec_ms]
+
+    wbytes, kv = _decode_bytes_per_token(wl)
+    dec_bytes = wbytes * wl.decode_steps + sum(kv)
+    peak, peak_kind = _peaks()
+    achieved = dec_bytes / (statistics.mean(dec_ms) / 1e3) / 1e9
+
+    # end to end through host buffers: prefix and start token copied in from pinned host
+    # memory, generated tokens copied back, every step.
+    out_h = torch.empty((wl.decode_steps, B), dtype=torch.int32).pin_memory()
+    am_h = torch.empty((B,), dtype=torch.int32).pin_memory()
+    e2e_ms = []
+    for i in range(max(1, min(a.steps, 3))):
+        cache.reset()
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        prefix.copy_(prefix_h, non_blocking=True)
+        start.copy_(start_h, non_blocking=True)
+        _, am = cache.prefill(start, prefix)
+        cache.generate(wl.decode_steps, out_tokens=out_tok, logits=False)
+        am_h.copy_(am, non_blocking=True)
+        out_h.copy_(out_tok, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    h2d = prefix_h.numel() * 4 + start_h.numel() * 8
+    d2h = out_h.numel() * 4 + am_h.numel() * 4
+    e2e_val = world * tokens_per_step / (statistics.mean(e2e_ms) / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, dt, threads, sample, _, _ = _oracle_sample(wl, a.cpu_decode_steps)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample,
+               "seconds": dt}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": total_ms / a.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config_json(wl, world),
+            "prefill_ms": {"mean": statistics.mean(pre_ms), "median": statistics.median(pre_ms)},
+            "decode_ms_per_token": {"mean": statistics.mean(per_tok), "median": statistics.median(per_tok),
+                                    "p90": float(np.percentile(per_tok, 90))},
+            "decode_tokens_per_s": B * wl.decode_steps / (statistics.mean(dec_ms) / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "decode step (all kernels of one token, one CUDA graph)",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes_per_token": dec_bytes / wl.decode_steps},
+            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "wall_s": t_wall,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    cache.close()
+    model.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,375 @@
+// Attention over the shared in-place KV cache ("MuScriptor Medium — optimized W4A32
+// ONNX Runtime", Model variant: GroupQueryAttention nodes, fixed-capacity cache shared by
+// past and present).  Causal, scale 1/sqrt(64), query head h reads kv head h / (H / Hk).
+//
+// Cache layout: K and V each [B][Hk][cap][64] per layer, so the keys of one (stream,
+// kv head) are one contiguous run of 256-byte rows.
+#include <math.h>
+#include "ms_device.cuh"
+#include "ms_launch.cuh"
+
+namespace ms {
+
+// ---------------------------------------------------------------------------------
+// Decode: split-K flash-decoding.  Grid (splits, Hk, B).  Each CTA takes a contiguous
+// run of positions of one (stream, kv head), computes the scores of all H/Hk query heads
+// of the group against it (each key is read once for the whole group), keeps a running
+// max / sum / weighted V sum, and writes its partial (m, l, o).  The last CTA of the
+// (stream, kv head) to finish — an atomic ticket, nothing waits — merges the partials.
+// The split count adapts to the current length read from the device, so one launch
+// configuration (and one captured graph) serves every step.
+// ---------------------------------------------------------------------------------
+namespace {
+constexpr int kDecThreads = 128;
+constexpr int kDecSub = 64;        // positions staged in shared memory at a time
+constexpr int kMinPerSplit = 16;   // smallest run of positions worth a CTA
+constexpr int kDecTargetCtas = 2 * 148;
+
+struct AttnDecArgs {
+  const float* q;
+  const float* kc;
+  const float* vc;
+  int B, H, Hk, cap;
+  const int* dlen;
+  int add;
+  int splits;
+  float* part;
+  unsigned* counters;
+  float* o;
+};
+}  // namespace
+
+int attn_decode_splits(int B, int Hk, int cap) {
+  int s = (kDecTargetCtas + B * Hk - 1) / (B * Hk);
+  const int most = (cap + kMinPerSplit - 1) / kMinPerSplit;
+  if (s > most) s = most;
+  if (s < 1) s = 1;
+  return s;
+}
+
+template <int HPG>
+__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a) {
+  __shared__ float qs[HPG][64];
+  __shared__ float Ks[kDecSub][65];
+  __shared__ __align__(16) float Vs[kDecSub][64];
+  __shared__ float sc[HPG][kDecSub];
+  __shared__ float mh[HPG], lh[HPG], corr[HPG];
+  __shared__ unsigned last;
+  constexpr int kSlots = (HPG * 64 + kDecThreads - 1) / kDecThreads;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  pdl_wait();
+  pdl_trigger();
+  const int T = *a.dlen + a.add;
+  int s_act = (T + kMinPerSplit - 1) / kMinPerSplit;
+  if (s_act > (int)gridDim.x) s_act = gridDim.x;
+  if (s_act < 1) s_act = 1;
+  if (split >= s_act) return;
+  const int chunk = (T + s_act - 1) / s_act;
+  const int t0 = split * chunk;
+  const int t1 = min(T, t0 + chunk);
+
+  for (int i = tid; i < HPG * 64; i += kDecThreads)
+    qs[i >> 6][i & 63] = a.q[((size_t)b * a.H + g * HPG + (i >> 6)) * 64 + (i & 63)] * 0.125f;
+  if (tid < HPG) {
+    mh[tid] = -INFINITY;
+    lh[tid] = 0.f;
+  }
+  float oacc[kSlots];
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) oacc[k] = 0.f;
+
+  const size_t head = ((size_t)b * a.Hk + g) * a.cap;
+  const float* kb = a.kc + head * 64;
+  const float* vb = a.vc + head * 64;
+
+  for (int c0 = t0; c0 < t1; c0 += kDecSub) {
+    const int cn = min(kDecSub, t1 - c0);
+    __syncthreads();
+    for (int i = tid; i < cn * 16; i += kDecThreads) {
+      const int p = i >> 4, f = i & 15;
+      const float4 kv = reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64)[f];
+      Ks[p][4 * f + 0] = kv.x;
+      Ks[p][4 * f + 1] = kv.y;
+      Ks[p][4 * f + 2] = kv.z;
+      Ks[p][4 * f + 3] = kv.w;
+      reinterpret_cast<float4*>(&Vs[p][0])[f] = reinterpret_cast<const float4*>(vb + (size_t)(c0 + p) * 64)[f];
+    }
+    __syncthreads();
+    for (int i = tid; i < HPG * kDecSub; i += kDecThreads) {
+      const int h = i / kDecSub, p = i - h * kDecSub;
+      float s = -INFINITY;
+      if (p < cn) {
+        s = 0.f;
+#pragma unroll 16
+        for (int dd = 0; dd < 64; ++dd) s = fmaf(qs[h][dd], Ks[p][dd], s);
+      }
+      sc[h][p] = s;
+    }
+    __syncthreads();
+    for (int h = warp; h < HPG; h += kDecThreads / 32) {
+      const float v0 = sc[h][lane], v1 = sc[h][lane + 32];
+      const float mx = warp_max(fmaxf(v0, v1));
+      const float mold = mh[h];
+      const float mnew = fmaxf(mold, mx);
+      const float e0 = lane < cn ? expf(v0 - mnew) : 0.f;
+      const float e1 = lane + 32 < cn ? expf(v1 - mnew) : 0.f;
+      sc[h][lane] = e0;
+      sc[h][lane + 32] = e1;
+      const float sum = warp_sum(e0 + e1);
+      __syncwarp();
+      if (lane == 0) {
+        const float cf = expf(mold - mnew);
+        corr[h] = cf;
+        lh[h] = lh[h] * cf + sum;
+        mh[h] = mnew;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      const int idx = tid + k * kDecThreads;
+      if (idx < HPG * 64) {
+        const int h = idx >> 6, dd = idx & 63;
+        float acc = oacc[k] * corr[h];
+        for (int p = 0; p < cn; ++p) acc = fmaf(sc[h][p], Vs[p][dd], acc);
+        oacc[k] = acc;
+      }
+    }
+  }
+  __syncthreads();
+
+  float* pb = a.part + (((size_t)b * a.Hk + g) * a.splits + split) * HPG * 66;
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) {
+    const int idx = tid + k * kDecThreads;
+    if (idx < HPG * 64) pb[(idx >> 6) * 66 + 2 + (idx & 63)] = oacc[k];
+  }
+  if (tid < HPG) {
+    pb[tid * 66 + 0] = mh[tid];
+    pb[tid * 66 + 1] = lh[tid];
+  }
+  __threadfence();
+  __syncthreads();
+  unsigned* ctr = a.counters + (size_t)b * a.Hk + g;
+  if (tid == 0) last = (atomicAdd(ctr, 1u) == (unsigned)(s_act - 1)) ? 1u : 0u;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* p0 = a.part + ((size_t)b * a.Hk + g) * a.splits * HPG * 66;
+  for (int idx = tid; idx < HPG * 64; idx += kDecThreads) {
+    const int h = idx >> 6, dd = idx & 63;
+    float M = -INFINITY;
+    for (int s = 0; s < s_act; ++s) M = fmaxf(M, __ldcg(p0 + ((size_t)s * HPG + h) * 66));
+    float Lsum = 0.f, O = 0.f;
+    for (int s = 0; s < s_act; ++s) {
+      const float* ps = p0 + ((size_t)s * HPG + h) * 66;
+      const float w = expf(__ldcg(ps) - M);
+      Lsum = fmaf(w, __ldcg(ps + 1), Lsum);
+      O = fmaf(w, __ldcg(ps + 2 + dd), O);
+    }
+    a.o[((size_t)b * a.H + g * HPG + h) * 64 + dd] = O / Lsum;
+  }
+  if (tid == 0) *ctr = 0u;
+}
+
+template <int HPG>
+static cudaError_t attn_dec_go(const Launch& L, const AttnDecArgs& a) {
+  return launch_k(L, attn_decode_kernel<HPG>, dim3(a.splits, a.Hk, a.B), dim3(kDecThreads), 0, a);
+}
+
+cudaError_t launch_attn_decode(const Launch& L, const float* q, const float* kc, const float* vc, int B, int H,
+                               int Hk, int cap, const int* dlen, int add, const AttnDecodeWork& w, float* o) {
+  AttnDecArgs a;
+  a.q = q;
+  a.kc = kc;
+  a.vc = vc;
+  a.B = B;
+  a.H = H;
+  a.Hk = Hk;
+  a.cap = cap;
+  a.dlen = dlen;
+  a.add = add;
+  a.splits = w.splits;
+  a.part = w.part;
+  a.counters = w.counters;
+  a.o = o;
+  switch (H / Hk) {
+    case 1: return attn_dec_go<1>(L, a);
+    case 2: return attn_dec_go<2>(L, a);
+    case 3: return attn_dec_go<3>(L, a);
+    case 4: return attn_dec_go<4>(L, a);
+    case 6: return attn_dec_go<6>(L, a);
+    case 8: return attn_dec_go<8>(L, a);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Prefill: causal flash attention on CUDA cores.  Grid (ceil(n / 64), H, B): one CTA per
+// 64 new query rows of one head.  Key tiles of 64 from position 0 up to the tile's last
+// query; running max and sum per row; scores never leave shared memory.  Query rows are
+// at positions len + i, the keys are the cache rows rope_append has just written.
+// ---------------------------------------------------------------------------------
+namespace {
+constexpr int kPreT = 64;
+constexpr int kPrePad = kPreT + 4;
+
+struct AttnPreArgs {
+  const float* q;
+  const float* kc;
+  const float* vc;
+  int B, n, H, Hk, cap;
+  const int* dlen;
+  float* o;
+};
+
+constexpr size_t kPreSmem = sizeof(float) * (3 * 64 * kPrePad + 64 * 64);
+}  // namespace
+
+__global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
+  extern __shared__ __align__(16) float sm[];
+  float(*Qs)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm);                   // [d][row]
+  float(*Ks)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm + 64 * kPrePad);    // [d][key]
+  float(*Ps)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm + 2 * 64 * kPrePad);  // [key][row]
+  float(*Vs)[64] = reinterpret_cast<float(*)[64]>(sm + 3 * 64 * kPrePad);          // [key][d]
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int g = h / (a.H / a.Hk);
+  pdl_wait();
+  pdl_trigger();
+  const int pos0 = *a.dlen;
+  const int i0 = qt * kPreT;
+  const int ivalid = min(kPreT, a.n - i0);
+  const int kend = pos0 + i0 + ivalid;  // keys [0, kend) are needed
+
+  for (int idx = tid; idx < kPreT * 16; idx += 256) {
+    const int r = idx >> 4, f = idx & 15;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < ivalid) v = reinterpret_cast<const float4*>(a.q + ((size_t)b * a.n + i0 + r) * a.H * 64 + h * 64)[f];
+    Qs[4 * f + 0][r] = v.x * 0.125f;
+    Qs[4 * f + 1][r] = v.y * 0.125f;
+    Qs[4 * f + 2][r] = v.z * 0.125f;
+    Qs[4 * f + 3][r] = v.w * 0.125f;
+  }
+  float m_i[4], l_i[4], O[4][4];
+  int qpos[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m_i[i] = -INFINITY;
+    l_i[i] = 0.f;
+    qpos[i] = pos0 + i0 + ty * 4 + i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) O[i][j] = 0.f;
+  }
+  const size_t head = ((size_t)b * a.Hk + g) * a.cap;
+  const float* kb = a.kc + head * 64;
+  const float* vb = a.vc + head * 64;
+
+  for (int c0 = 0; c0 < kend; c0 += kPreT) {
+    __syncthreads();
+    for (int idx = tid; idx < kPreT * 16; idx += 256) {
+      const int r = idx >> 4, f = idx & 15;
+      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
+      if (c0 + r < kend) {
+        kv = reinterpret_cast<const float4*>(kb + (size_t)(c0 + r) * 64)[f];
+        vv = reinterpret_cast<const float4*>(vb + (size_t)(c0 + r) * 64)[f];
+      }
+      Ks[4 * f + 0][r] = kv.x;
+      Ks[4 * f + 1][r] = kv.y;
+      Ks[4 * f + 2][r] = kv.z;
+      Ks[4 * f + 3][r] = kv.w;
+      reinterpret_cast<float4*>(&Vs[r][0])[f] = vv;
+    }
+    __syncthreads();
+    float s[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
+#pragma unroll 8
+    for (int dd = 0; dd < 64; ++dd) {
+      const float4 qa = *reinterpret_cast<const float4*>(&Qs[dd][ty * 4]);
+      const float4 kk = *reinterpret_cast<const float4*>(&Ks[dd][tx * 4]);
+      const float qr[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float kr[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[i][j] = fmaf(qr[i], kr[j], s[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int key = c0 + tx * 4 + j;
+        if (key > qpos[i] || key >= kend) s[i][j] = -INFINITY;
+        mx = fmaxf(mx, s[i][j]);
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mnew = fmaxf(m_i[i], mx);
+      const float cf = mnew == -INFINITY ? 1.f : expf(m_i[i] - mnew);
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float p = s[i][j] == -INFINITY ? 0.f : expf(s[i][j] - mnew);
+        s[i][j] = p;
+        rs += p;
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
+      l_i[i] = l_i[i] * cf + rs;
+      m_i[i] = mnew;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) O[i][j] *= cf;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Ps[tx * 4 + j][ty * 4 + i] = s[i][j];
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kPreT; ++c) {
+      const float4 pa = *reinterpret_cast<const float4*>(&Ps[c][ty * 4]);
+      const float4 vv = *reinterpret_cast<const float4*>(&Vs[c][tx * 4]);
+      const float pr[4] = {pa.x, pa.y, pa.z, pa.w};
+      const float vr[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) O[i][j] = fmaf(pr[i], vr[j], O[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty * 4 + i;
+    if (r >= ivalid) continue;
+    const float inv = 1.0f / l_i[i];
+    float4 v = make_float4(O[i][0] * inv, O[i][1] * inv, O[i][2] * inv, O[i][3] * inv);
+    reinterpret_cast<float4*>(a.o + ((size_t)b * a.n + i0 + r) * a.H * 64 + h * 64)[tx] = v;
+  }
+}
+
+cudaError_t init_attrs_attn() { return allow_smem(attn_prefill_kernel, kMaxDynSmem); }
+
+cudaError_t launch_attn_prefill(const Launch& L, const float* q, const float* kc, const float* vc, int B, int n,
+                                int H, int Hk, int cap, const int* dlen, float* o) {
+  if (n <= 0) return cudaSuccess;
+  AttnPreArgs a;
+  a.q = q;
+  a.kc = kc;
+  a.vc = vc;
+  a.B = B;
+  a.n = n;
+  a.H = H;
+  a.Hk = Hk;
+  a.cap = cap;
+  a.dlen = dlen;
+  a.o = o;
+  return launch_k(L, attn_prefill_kernel, dim3((n + kPreT - 1) / kPreT, H, B), dim3(256), kPreSmem, a);
+}
+
+}  // namespace ms

@@ -1,0 +1,96 @@
+// Host-side launchers of the decoder kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ms {
+
+// Bits of the per-cache device status word.
+constexpr unsigned kErrTokenBit = 1u;    // a token id was outside [0, vocab) and was clamped
+constexpr unsigned kErrTimeoutBit = 2u;  // a bounded wait ran out
+constexpr unsigned kErrShapeBit = 4u;    // a device-side size check failed
+
+enum WFmt { kInt4 = 0, kFp16 = 1 };
+enum Epi { kStore = 0, kAdd = 1, kGelu = 2 };
+
+// Where a kernel runs and what it reports into.
+struct Launch {
+  cudaStream_t stream;
+  bool pdl;           // launch with programmatic stream serialisation
+  unsigned* status;   // device status word (may be null)
+};
+
+// A backbone matrix [N][K] (row n = output feature n) in the library's device layout.
+struct WView {
+  const uint8_t* q;   // INT4 nibbles [N][K/2]
+  const float* s;     // INT4 scales [N][K/32]
+  const uint16_t* h;  // fp16 [N][K]
+  int N, K;
+  int fmt;            // WFmt
+};
+
+// Opt every kernel that needs it into large dynamic shared memory on the current device.
+cudaError_t init_attrs_gemv();
+cudaError_t init_attrs_attn();
+
+cudaError_t launch_quantize_int4(const float* w, int N, int K, uint8_t* packed, float* scales,
+                                 cudaStream_t s);
+
+// x[b][i] rows of a prefill: prefix rows then embedded tokens; tokens int64 [B][S].
+cudaError_t launch_embed_prefill(const Launch& L, const int64_t* tokens, int S, const float* prefix,
+                                 int P, const float* tok_emb, int V, int d, int B, float* x);
+// x[b] = tok_emb[token[b]]; token from `tokens` (int32 [B]) or, if null, from
+// hist[(len - 1) * B + b] with len read from `dlen`.
+cudaError_t launch_embed_decode(const Launch& L, const int32_t* tokens, const int32_t* hist,
+                                const int* dlen, const float* tok_emb, int V, int d, int B, float* x);
+
+// x <- x + y (y may be null), h = LN(x) * g + b, per row.
+cudaError_t launch_skipln(const Launch& L, float* x, const float* y, const float* g, const float* b,
+                          float eps, int R, int d, float* h);
+
+// RoPE on the q and k parts of qkv rows (row r = b * n + i at position len + i, len read
+// from dlen) and append post-RoPE k and v to the layer's cache slices.
+cudaError_t launch_rope_append(const Launch& L, const float* qkv, int B, int n, int H, int Hk,
+                               const float* cosv, const float* sinv, const int* dlen, float* q_out,
+                               float* kc, float* vc, int cap);
+
+// Smallest-M path (decode): M <= 8.  Optional LayerNorm of x in the prologue (ln_g != null).
+cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx, int M,
+                        const float* ln_g, const float* ln_b, float eps, float* y, int ldy, int epi);
+bool gemv_fits(const WView& w, int M);
+
+// General-M path (prefill, batched decode).
+cudaError_t launch_gemm(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y,
+                        int ldy, int epi);
+
+// Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
+// the combine done by the last CTA of each (stream, kv head).
+struct AttnDecodeWork {
+  float* part;        // [B][Hk][splits][hpg][66]
+  unsigned* counters; // [B][Hk], zero between launches
+  int splits;         // grid splits (max)
+};
+cudaError_t launch_attn_decode(const Launch& L, const float* q, const float* kc, const float* vc,
+                               int B, int H, int Hk, int cap, const int* dlen, int add,
+                               const AttnDecodeWork& w, float* o);
+int attn_decode_splits(int B, int Hk, int cap);
+
+// Causal prefill attention for n new rows per stream at positions len .. len + n - 1.
+cudaError_t launch_attn_prefill(const Launch& L, const float* q, const float* kc, const float* vc,
+                                int B, int n, int H, int Hk, int cap, const int* dlen, float* o);
+
+// LM head + argmax over rows x[m * ldx], m < M.  Writes logits (may be null), argmax
+// (may be null), hist[(len + hist_off) * B + m] (may be null) and, in its last CTA,
+// *dlen += len_add.
+struct LmHeadWork {
+  float* part_val;    // [grid][64]
+  int* part_idx;      // [grid][64]
+  unsigned* counter;  // one word, zero between launches
+};
+cudaError_t launch_lm_head(const Launch& L, const float* x, int ldx, int M, int d, const float* ln_g,
+                           const float* ln_b, float eps, const float* W, int V, float* logits,
+                           int32_t* argmax, int32_t* hist, int hist_B, int hist_off, int* dlen,
+                           int len_add, const LmHeadWork& w);
+int lm_head_grid(int V);
+
+}  // namespace ms

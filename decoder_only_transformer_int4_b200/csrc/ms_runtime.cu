@@ -1,0 +1,742 @@
+// Host runtime of the C ABI in include/ms.h: owns the device copy of the weights, the
+// fixed-capacity KV cache and its work buffers, and sequences the kernels of one
+// decoder call (prefill, decode step, greedy loop from a captured CUDA graph).
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <cmath>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/ms.h"
+#include "ms_kernels.h"
+#include "ms_launch.cuh"
+
+namespace ms {
+std::atomic<unsigned long long>& launch_counter() {
+  static std::atomic<unsigned long long> n{0};
+  return n;
+}
+}  // namespace ms
+
+namespace {
+
+thread_local std::string g_err;
+
+ms_status fail(ms_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define CUDA_TRY(call)                                                              \
+  do {                                                                              \
+    cudaError_t e_ = (call);                                                        \
+    if (e_ != cudaSuccess) {                                                        \
+      if (e_ == cudaErrorMemoryAllocation) {                                        \
+        cudaGetLastError();                                                         \
+        return fail(MS_ERR_OOM, "%s: %s", #call, cudaGetErrorString(e_));           \
+      }                                                                             \
+      return fail(MS_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));            \
+    }                                                                               \
+  } while (0)
+
+// Makes `dev` current for the duration of a call and restores the caller's device.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over one cudaMalloc'd arena (256-byte aligned pieces).
+struct Arena {
+  char* base = nullptr;
+  size_t size = 0, used = 0;
+  template <typename T>
+  T* take(size_t count) {
+    size_t off = round_up(used, 256);
+    used = off + count * sizeof(T);
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+struct DevLayer {
+  float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+  ms::WView w[4];
+};
+
+bool shape_ok(const ms_config* c, std::string* why) {
+  char b[256];
+  auto bad = [&](const char* m) {
+    snprintf(b, sizeof(b), "%s", m);
+    *why = b;
+    return false;
+  };
+  if (c->n_layers < 0) return bad("n_layers < 0");
+  if (c->head_dim != 64) return bad("head_dim must be 64");
+  if (c->d_model <= 0 || c->d_model % 256 != 0) return bad("d_model must be a positive multiple of 256");
+  if (c->d_model > 2048) return bad("d_model above 2048 is not supported");
+  if (c->d_ff <= 0 || c->d_ff % 256 != 0) return bad("d_ff must be a positive multiple of 256");
+  if (c->n_heads <= 0 || c->n_kv_heads <= 0 || c->n_heads % c->n_kv_heads != 0)
+    return bad("n_heads must be a positive multiple of n_kv_heads");
+  const int hpg = c->n_heads / c->n_kv_heads;
+  if (hpg != 1 && hpg != 2 && hpg != 3 && hpg != 4 && hpg != 6 && hpg != 8)
+    return bad("n_heads / n_kv_heads must be 1, 2, 3, 4, 6 or 8");
+  if ((c->n_heads * 64) % 256 != 0) return bad("n_heads * 64 must be a multiple of 256");
+  if (c->vocab < 1) return bad("vocab < 1");
+  if (c->weight_format != MS_W_INT4_G32 && c->weight_format != MS_W_FP16) return bad("unknown weight_format");
+  if (!(c->ln_eps > 0.f) || !(c->rope_base > 0.f)) return bad("ln_eps and rope_base must be positive");
+  return true;
+}
+
+void mat_nk(const ms_config& c, int i, int* N, int* K) {
+  const int d = c.d_model, H = c.n_heads, Hk = c.n_kv_heads, F = c.d_ff;
+  switch (i) {
+    case 0: *N = (H + 2 * Hk) * 64; *K = d; break;
+    case 1: *N = d; *K = H * 64; break;
+    case 2: *N = F; *K = d; break;
+    default: *N = d; *K = F; break;
+  }
+}
+
+// Library-owned scratch for the single-operation entry points (per device).
+struct OpScratch {
+  float* part_val = nullptr;
+  int* part_idx = nullptr;
+  unsigned* counter = nullptr;
+};
+std::mutex g_scratch_mu;
+std::vector<OpScratch> g_scratch;
+
+// Kernel attributes are set once per device, outside any stream capture.
+std::mutex g_attr_mu;
+std::vector<char> g_attr_done;
+
+cudaError_t ensure_kernel_attributes() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if ((int)g_attr_done.size() <= dev) g_attr_done.resize(dev + 1, 0);
+  if (g_attr_done[dev]) return cudaSuccess;
+  e = ms::init_attrs_gemv();
+  if (e == cudaSuccess) e = ms::init_attrs_attn();
+  if (e == cudaSuccess) g_attr_done[dev] = 1;
+  return e;
+}
+
+}  // namespace
+
+struct ms_model {
+  ms_config cfg;
+  int device = 0;
+  Arena arena;
+  float *tok_emb = nullptr, *lm_head = nullptr, *ln_f_g = nullptr, *ln_f_b = nullptr;
+  std::vector<DevLayer> layers;
+};
+
+struct ms_cache {
+  ms_model* m = nullptr;
+  int B = 0, cap = 0, len = 0;
+  bool has_next = false;  // hist holds the argmax of position len - 1
+  Arena arena;
+  float *k = nullptr, *v = nullptr;        // [L][B][Hk][cap][64]
+  float *cosv = nullptr, *sinv = nullptr;  // [cap][32]
+  int* dlen = nullptr;
+  int32_t* hist = nullptr;                 // [cap][B]
+  unsigned* status = nullptr;
+  unsigned* att_counters = nullptr;        // [B][Hk]
+  float* att_part = nullptr;
+  int splits = 1;
+  float* lm_val = nullptr;
+  int* lm_idx = nullptr;
+  unsigned* lm_counter = nullptr;
+  float *x = nullptr, *h = nullptr, *y = nullptr, *qkv = nullptr, *q = nullptr, *o = nullptr, *u = nullptr;
+  float* logits = nullptr;                 // [B][V] internal
+  size_t rows_cap = 0;
+  cudaGraphExec_t gen_exec = nullptr;
+  size_t gen_nodes = 0;
+  cudaStream_t gen_stream = nullptr;     // used when the caller passes the legacy stream
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+  unsigned long long launches = 0;  // kernels launched for this cache
+};
+
+namespace {
+
+size_t layer_stride(const ms_cache* c) {
+  return (size_t)c->B * c->m->cfg.n_kv_heads * c->cap * 64;
+}
+
+ms::Launch launch_of(ms_cache* c, cudaStream_t s, bool pdl) { return ms::Launch{s, pdl, c->status}; }
+
+// ---- one decoder call, kernel by kernel ----------------------------------------------
+// Prefill of n = P + S rows per stream.  Rows of stream b are b * n + i.
+cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, const float* prefix, int P,
+                        float* logits, int32_t* argmax, cudaStream_t st) {
+  const ms_config& g = m->cfg;
+  const int n = P + S, B = c->B, R = B * n, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads;
+  const int nq = (H + 2 * Hk) * 64;
+  ms::Launch L0 = launch_of(c, st, false), L = launch_of(c, st, true);
+  cudaError_t e = ms::launch_embed_prefill(L0, tokens, S, prefix, P, m->tok_emb, g.vocab, d, B, c->x);
+  for (int l = 0; l < g.n_layers && e == cudaSuccess; ++l) {
+    const DevLayer& ly = m->layers[l];
+    float* kc = c->k + l * layer_stride(c);
+    float* vc = c->v + l * layer_stride(c);
+    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
+    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
+    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o);
+    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
+    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu);
+    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore);
+  }
+  if (e == cudaSuccess)
+    e = ms::launch_skipln(L, c->x, g.n_layers > 0 ? c->y : nullptr, m->ln_f_g, m->ln_f_b, g.ln_eps, R, d, c->h);
+  ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
+  if (e == cudaSuccess)
+    e = ms::launch_lm_head(L, c->h + (size_t)(n - 1) * d, n * d, B, d, nullptr, nullptr, g.ln_eps, m->lm_head, g.vocab,
+                           logits, argmax, c->hist, B, n - 1, c->dlen, n, w);
+  return e;
+}
+
+// One decode step: one row per stream.  tokens == nullptr reads the previous argmax from
+// the cache's token history (the greedy loop).
+cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* logits, int32_t* argmax,
+                       cudaStream_t st, bool first_pdl) {
+  const ms_config& g = m->cfg;
+  const int B = c->B, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads, F = g.d_ff;
+  const int nq = (H + 2 * Hk) * 64;
+  ms::Launch L0 = launch_of(c, st, first_pdl), L = launch_of(c, st, true);
+  const bool small = (B == 1 || B == 2 || B == 4 || B == 8);
+  ms::AttnDecodeWork aw{c->att_part, c->att_counters, c->splits};
+  cudaError_t e = ms::launch_embed_decode(L0, tokens, c->hist, c->dlen, m->tok_emb, g.vocab, d, B, c->x);
+  for (int l = 0; l < g.n_layers && e == cudaSuccess; ++l) {
+    const DevLayer& ly = m->layers[l];
+    float* kc = c->k + l * layer_stride(c);
+    float* vc = c->v + l * layer_stride(c);
+    const bool gv = small && ms::gemv_fits(ly.w[0], B) && ms::gemv_fits(ly.w[1], B) && ms::gemv_fits(ly.w[2], B) &&
+                    ms::gemv_fits(ly.w[3], B);
+    if (gv) {
+      e = ms::launch_gemv(L, ly.w[0], c->x, d, B, ly.ln1_g, ly.ln1_b, g.ln_eps, c->qkv, nq, ms::kStore);
+    } else {
+      e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
+      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
+    }
+    if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
+    if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o);
+    if (gv) {
+      if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[1], c->o, H * 64, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
+      if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[3], c->u, F, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
+    } else {
+      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
+      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
+      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
+    }
+  }
+  ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
+  if (e == cudaSuccess)
+    e = ms::launch_lm_head(L, c->x, d, B, d, m->ln_f_g, m->ln_f_b, g.ln_eps, m->lm_head, g.vocab, logits, argmax,
+                           c->hist, B, 0, c->dlen, 1, w);
+  return e;
+}
+
+ms_status check_launch(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return MS_OK;
+  return fail(MS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+// =====================================================================================
+// C ABI
+// =====================================================================================
+extern "C" {
+
+const char* ms_last_error(void) { return g_err.c_str(); }
+
+ms_status ms_quantize_int4_g32(const float* w, int N, int K, uint8_t* packed, float* scales, void* stream) {
+  if (!w || !packed || !scales) return fail(MS_ERR_INVALID_ARG, "ms_quantize_int4_g32: null pointer");
+  if (N < 1 || K < 32 || K % 32 != 0) return fail(MS_ERR_SHAPE, "ms_quantize_int4_g32: need N >= 1 and K a multiple of 32");
+  if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(packed) & 15))
+    return fail(MS_ERR_INVALID_ARG, "ms_quantize_int4_g32: w and packed must be 16-byte aligned");
+  return check_launch(ms::launch_quantize_int4(w, N, K, packed, scales, (cudaStream_t)stream), "quantize kernel");
+}
+
+size_t ms_cache_kv_bytes(const ms_config* cfg, int batch, int capacity) {
+  if (!cfg || batch < 1 || capacity < 1 || cfg->n_layers < 0 || cfg->n_kv_heads < 1) return 0;
+  return (size_t)2 * cfg->n_layers * batch * cfg->n_kv_heads * (size_t)capacity * 64 * sizeof(float);
+}
+
+ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device, ms_model** out) {
+  if (!cfg || !wt || !out) return fail(MS_ERR_INVALID_ARG, "ms_model_create: null argument");
+  *out = nullptr;
+  std::string why;
+  if (!shape_ok(cfg, &why)) return fail(MS_ERR_SHAPE, "ms_model_create: %s", why.c_str());
+  const ms_config& c = *cfg;
+  if (!wt->tok_emb || !wt->lm_head || !wt->ln_f_g || !wt->ln_f_b || (c.n_layers > 0 && !wt->layers))
+    return fail(MS_ERR_INVALID_ARG, "ms_model_create: null weight pointer");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const ms_layer_weights& lw = wt->layers[l];
+    if (!lw.ln1_g || !lw.ln1_b || !lw.ln2_g || !lw.ln2_b)
+      return fail(MS_ERR_INVALID_ARG, "ms_model_create: layer %d: null LayerNorm pointer", l);
+    for (int i = 0; i < 4; ++i) {
+      if (c.weight_format == MS_W_INT4_G32 && (!lw.w[i] || !lw.s[i]))
+        return fail(MS_ERR_INVALID_ARG, "ms_model_create: layer %d matrix %d: null INT4 pointer", l, i);
+      if (c.weight_format == MS_W_FP16 && !lw.w16[i])
+        return fail(MS_ERR_INVALID_ARG, "ms_model_create: layer %d matrix %d: null fp16 pointer", l, i);
+    }
+  }
+  int ndev = 0;
+  CUDA_TRY(cudaGetDeviceCount(&ndev));
+  if (device < 0 || device >= ndev) return fail(MS_ERR_INVALID_ARG, "ms_model_create: no device %d", device);
+  DeviceGuard dg(device);
+  if (!dg.ok) return fail(MS_ERR_CUDA, "ms_model_create: cudaSetDevice(%d) failed", device);
+
+  {
+    cudaError_t ea = ensure_kernel_attributes();
+    if (ea != cudaSuccess) return fail(MS_ERR_CUDA, "ms_model_create: kernel attributes: %s", cudaGetErrorString(ea));
+  }
+  ms_model* m = new (std::nothrow) ms_model;
+  if (!m) return fail(MS_ERR_OOM, "ms_model_create: host allocation failed");
+  m->cfg = c;
+  m->device = device;
+  const int d = c.d_model, V = c.vocab;
+  // pass 1: sizes; pass 2: pointers
+  for (int pass = 0; pass < 2; ++pass) {
+    Arena& a = m->arena;
+    a.used = 0;
+    m->tok_emb = a.take<float>((size_t)V * d);
+    m->lm_head = a.take<float>((size_t)V * d);
+    m->ln_f_g = a.take<float>(d);
+    m->ln_f_b = a.take<float>(d);
+    m->layers.assign(c.n_layers, DevLayer{});
+    for (int l = 0; l < c.n_layers; ++l) {
+      DevLayer& L = m->layers[l];
+      L.ln1_g = a.take<float>(d);
+      L.ln1_b = a.take<float>(d);
+      L.ln2_g = a.take<float>(d);
+      L.ln2_b = a.take<float>(d);
+      for (int i = 0; i < 4; ++i) {
+        int N, K;
+        mat_nk(c, i, &N, &K);
+        ms::WView& w = L.w[i];
+        w.N = N;
+        w.K = K;
+        w.fmt = c.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
+        w.q = nullptr;
+        w.s = nullptr;
+        w.h = nullptr;
+        if (w.fmt == ms::kInt4) {
+          w.q = a.take<uint8_t>((size_t)N * K / 2);
+          w.s = a.take<float>((size_t)N * K / 32);
+        } else {
+          w.h = a.take<uint16_t>((size_t)N * K);
+        }
+      }
+    }
+    if (pass == 0) {
+      a.size = round_up(a.used, 256);
+      cudaError_t e = cudaMalloc(&a.base, a.size);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete m;
+        return fail(e == cudaErrorMemoryAllocation ? MS_ERR_OOM : MS_ERR_CUDA, "ms_model_create: cudaMalloc(%zu): %s",
+                    a.size, cudaGetErrorString(e));
+      }
+    }
+  }
+  auto cp = [&](void* dst, const void* src, size_t bytes) -> cudaError_t {
+    return cudaMemcpy(dst, src, bytes, cudaMemcpyDefault);
+  };
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = cp(m->tok_emb, wt->tok_emb, (size_t)V * d * 4);
+  if (e == cudaSuccess) e = cp(m->lm_head, wt->lm_head, (size_t)V * d * 4);
+  if (e == cudaSuccess) e = cp(m->ln_f_g, wt->ln_f_g, (size_t)d * 4);
+  if (e == cudaSuccess) e = cp(m->ln_f_b, wt->ln_f_b, (size_t)d * 4);
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    const ms_layer_weights& lw = wt->layers[l];
+    DevLayer& L = m->layers[l];
+    if (e == cudaSuccess) e = cp(L.ln1_g, lw.ln1_g, (size_t)d * 4);
+    if (e == cudaSuccess) e = cp(L.ln1_b, lw.ln1_b, (size_t)d * 4);
+    if (e == cudaSuccess) e = cp(L.ln2_g, lw.ln2_g, (size_t)d * 4);
+    if (e == cudaSuccess) e = cp(L.ln2_b, lw.ln2_b, (size_t)d * 4);
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
+      const ms::WView& w = L.w[i];
+      if (w.fmt == ms::kInt4) {
+        e = cp(const_cast<uint8_t*>(w.q), lw.w[i], (size_t)w.N * w.K / 2);
+        if (e == cudaSuccess) e = cp(const_cast<float*>(w.s), lw.s[i], (size_t)w.N * w.K / 32 * 4);
+      } else {
+        e = cp(const_cast<uint16_t*>(w.h), lw.w16[i], (size_t)w.N * w.K * 2);
+      }
+    }
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(m->arena.base);
+    delete m;
+    return fail(MS_ERR_CUDA, "ms_model_create: weight copy: %s", cudaGetErrorString(e));
+  }
+  *out = m;
+  return MS_OK;
+}
+
+ms_status ms_model_destroy(ms_model* m) {
+  if (!m) return fail(MS_ERR_INVALID_ARG, "ms_model_destroy: null model");
+  DeviceGuard dg(m->device);
+  cudaFree(m->arena.base);
+  delete m;
+  return MS_OK;
+}
+
+size_t ms_model_weight_bytes(const ms_model* m) { return m ? m->arena.used : 0; }
+
+ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) {
+  if (!m || !out) return fail(MS_ERR_INVALID_ARG, "ms_cache_create: null argument");
+  *out = nullptr;
+  if (batch < 1 || batch > 64) return fail(MS_ERR_SHAPE, "ms_cache_create: batch must be in [1, 64]");
+  if (capacity < 1) return fail(MS_ERR_SHAPE, "ms_cache_create: capacity must be >= 1");
+  DeviceGuard dg(m->device);
+  const ms_config& g = m->cfg;
+  ms_cache* c = new (std::nothrow) ms_cache;
+  if (!c) return fail(MS_ERR_OOM, "ms_cache_create: host allocation failed");
+  c->m = m;
+  c->B = batch;
+  c->cap = capacity;
+  c->splits = ms::attn_decode_splits(batch, g.n_kv_heads, capacity);
+  c->rows_cap = (size_t)batch * capacity;
+  const int hpg = g.n_heads / g.n_kv_heads;
+  const size_t R = c->rows_cap;
+  const int lmg = ms::lm_head_grid(g.vocab);
+  for (int pass = 0; pass < 2; ++pass) {
+    Arena& a = c->arena;
+    a.used = 0;
+    c->k = a.take<float>((size_t)g.n_layers * layer_stride(c) + 64);
+    c->v = a.take<float>((size_t)g.n_layers * layer_stride(c) + 64);
+    c->cosv = a.take<float>((size_t)capacity * 32);
+    c->sinv = a.take<float>((size_t)capacity * 32);
+    c->dlen = a.take<int>(4);
+    c->status = a.take<unsigned>(4);
+    c->lm_counter = a.take<unsigned>(4);
+    c->att_counters = a.take<unsigned>((size_t)batch * g.n_kv_heads);
+    c->hist = a.take<int32_t>((size_t)capacity * batch);
+    c->att_part = a.take<float>((size_t)batch * g.n_kv_heads * c->splits * hpg * 66);
+    c->lm_val = a.take<float>((size_t)lmg * 64);
+    c->lm_idx = a.take<int>((size_t)lmg * 64);
+    c->x = a.take<float>(R * g.d_model);
+    c->h = a.take<float>(R * g.d_model);
+    c->y = a.take<float>(R * g.d_model);
+    c->qkv = a.take<float>(R * (g.n_heads + 2 * g.n_kv_heads) * 64);
+    c->q = a.take<float>(R * g.n_heads * 64);
+    c->o = a.take<float>(R * g.n_heads * 64);
+    c->u = a.take<float>(R * g.d_ff);
+    c->logits = a.take<float>((size_t)batch * g.vocab);
+    if (pass == 0) {
+      a.size = round_up(a.used, 256);
+      cudaError_t e = cudaMalloc(&a.base, a.size);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete c;
+        return fail(e == cudaErrorMemoryAllocation ? MS_ERR_OOM : MS_ERR_CUDA, "ms_cache_create: cudaMalloc(%zu): %s",
+                    a.size, cudaGetErrorString(e));
+      }
+    }
+  }
+  // RoPE table: angle = pos * base^(-2i/64), computed in double, stored fp32.
+  std::vector<float> cs((size_t)capacity * 32), sn((size_t)capacity * 32);
+  for (int p = 0; p < capacity; ++p)
+    for (int i = 0; i < 32; ++i) {
+      const double th = std::pow((double)g.rope_base, -2.0 * i / 64.0);
+      const double ang = (double)p * th;
+      cs[(size_t)p * 32 + i] = (float)std::cos(ang);
+      sn[(size_t)p * 32 + i] = (float)std::sin(ang);
+    }
+  cudaError_t e = cudaMemset(c->arena.base, 0, c->arena.size);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->gen_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaMemcpy(c->cosv, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->sinv, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    if (c->gen_stream) cudaStreamDestroy(c->gen_stream);
+    if (c->ev_in) cudaEventDestroy(c->ev_in);
+    if (c->ev_out) cudaEventDestroy(c->ev_out);
+    cudaFree(c->arena.base);
+    delete c;
+    return fail(MS_ERR_CUDA, "ms_cache_create: init: %s", cudaGetErrorString(e));
+  }
+  *out = c;
+  return MS_OK;
+}
+
+ms_status ms_cache_destroy(ms_cache* c) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_destroy: null cache");
+  DeviceGuard dg(c->m->device);
+  if (c->gen_exec) cudaGraphExecDestroy(c->gen_exec);
+  if (c->gen_stream) {
+    cudaStreamSynchronize(c->gen_stream);
+    cudaStreamDestroy(c->gen_stream);
+  }
+  if (c->ev_in) cudaEventDestroy(c->ev_in);
+  if (c->ev_out) cudaEventDestroy(c->ev_out);
+  cudaDeviceSynchronize();
+  cudaFree(c->arena.base);
+  delete c;
+  return MS_OK;
+}
+
+ms_status ms_cache_reset(ms_cache* c) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_reset: null cache");
+  DeviceGuard dg(c->m->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  int zero = 0;
+  CUDA_TRY(cudaMemcpy(c->dlen, &zero, sizeof(int), cudaMemcpyHostToDevice));
+  c->len = 0;
+  c->has_next = false;
+  return MS_OK;
+}
+
+int ms_cache_length(const ms_cache* c) { return c ? c->len : -1; }
+uint64_t ms_cache_kernel_launches(const ms_cache* c) { return c ? c->launches : 0; }
+int ms_cache_capacity(const ms_cache* c) { return c ? c->cap : -1; }
+int ms_cache_batch(const ms_cache* c) { return c ? c->B : -1; }
+
+ms_status ms_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, const float* prefix, int P,
+                     float* logits, int32_t* argmax, void* stream) {
+  if (!m || !c) return fail(MS_ERR_INVALID_ARG, "ms_prefill: null model or cache");
+  if (c->m != m) return fail(MS_ERR_INVALID_ARG, "ms_prefill: cache belongs to another model");
+  if (S < 0 || P < 0 || P + S < 1) return fail(MS_ERR_SHAPE, "ms_prefill: need S >= 0, P >= 0, P + S >= 1");
+  if (S > 0 && !tokens) return fail(MS_ERR_INVALID_ARG, "ms_prefill: null tokens with S > 0");
+  if (P > 0 && !prefix) return fail(MS_ERR_INVALID_ARG, "ms_prefill: null prefix with P > 0");
+  if ((long long)c->len + P + S > c->cap)
+    return fail(MS_ERR_CACHE_FULL, "ms_prefill: %d + %d positions exceed capacity %d", c->len, P + S, c->cap);
+  DeviceGuard dg(m->device);
+  const unsigned long long before = ms::launch_counter().load();
+  cudaError_t e = run_prefill(m, c, tokens, S, prefix, P, logits, argmax, (cudaStream_t)stream);
+  c->launches += ms::launch_counter().load() - before;
+  if (e != cudaSuccess) return check_launch(e, "ms_prefill launch");
+  c->len += P + S;
+  c->has_next = true;
+  return MS_OK;
+}
+
+ms_status ms_decode_step(ms_model* m, ms_cache* c, const int32_t* tokens, float* logits, int32_t* argmax,
+                         void* stream) {
+  if (!m || !c) return fail(MS_ERR_INVALID_ARG, "ms_decode_step: null model or cache");
+  if (c->m != m) return fail(MS_ERR_INVALID_ARG, "ms_decode_step: cache belongs to another model");
+  if (!tokens) return fail(MS_ERR_INVALID_ARG, "ms_decode_step: null tokens");
+  if (c->len + 1 > c->cap) return fail(MS_ERR_CACHE_FULL, "ms_decode_step: cache full (%d)", c->cap);
+  DeviceGuard dg(m->device);
+  const unsigned long long before = ms::launch_counter().load();
+  cudaError_t e = run_decode(m, c, tokens, logits, argmax, (cudaStream_t)stream, false);
+  c->launches += ms::launch_counter().load() - before;
+  if (e != cudaSuccess) return check_launch(e, "ms_decode_step launch");
+  c->len += 1;
+  c->has_next = true;
+  return MS_OK;
+}
+
+ms_status ms_generate(ms_model* m, ms_cache* c, int n_steps, int32_t* out_tokens, float* logits, void* stream) {
+  if (!m || !c) return fail(MS_ERR_INVALID_ARG, "ms_generate: null model or cache");
+  if (c->m != m) return fail(MS_ERR_INVALID_ARG, "ms_generate: cache belongs to another model");
+  if (n_steps < 0) return fail(MS_ERR_SHAPE, "ms_generate: n_steps < 0");
+  if (n_steps == 0) return MS_OK;
+  if (!out_tokens) return fail(MS_ERR_INVALID_ARG, "ms_generate: null out_tokens");
+  if (!c->has_next) return fail(MS_ERR_INVALID_ARG, "ms_generate: no previous argmax on this cache (prefill first)");
+  if ((long long)c->len + n_steps > c->cap)
+    return fail(MS_ERR_CACHE_FULL, "ms_generate: %d + %d positions exceed capacity %d", c->len, n_steps, c->cap);
+  DeviceGuard dg(m->device);
+  const bool legacy = stream == nullptr;
+  cudaStream_t st = legacy ? c->gen_stream : (cudaStream_t)stream;
+  const int len0 = c->len;
+  if (legacy) {
+    // the graph runs on the cache's own stream, ordered after and before the legacy stream
+    CUDA_TRY(cudaEventRecord(c->ev_in, nullptr));
+    CUDA_TRY(cudaStreamWaitEvent(st, c->ev_in, 0));
+  }
+  {
+    if (!c->gen_exec) {
+      cudaGraph_t graph = nullptr;
+      CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+      cudaError_t e = run_decode(m, c, nullptr, c->logits, nullptr, st, false);
+      cudaError_t e2 = cudaStreamEndCapture(st, &graph);
+      if (e != cudaSuccess || e2 != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return fail(MS_ERR_CUDA, "ms_generate: capture: %s", cudaGetErrorString(e != cudaSuccess ? e : e2));
+      }
+      size_t nodes = 0;
+      cudaGraphGetNodes(graph, nullptr, &nodes);
+      c->gen_nodes = nodes;
+      e = cudaGraphInstantiate(&c->gen_exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (e != cudaSuccess) {
+        c->gen_exec = nullptr;
+        return fail(MS_ERR_CUDA, "ms_generate: instantiate: %s", cudaGetErrorString(e));
+      }
+    }
+    for (int i = 0; i < n_steps; ++i) {
+      CUDA_TRY(cudaGraphLaunch(c->gen_exec, st));
+      c->launches += c->gen_nodes;
+    }
+  }
+  CUDA_TRY(cudaMemcpyAsync(out_tokens, c->hist + (size_t)len0 * c->B, (size_t)n_steps * c->B * sizeof(int32_t),
+                           cudaMemcpyDeviceToDevice, st));
+  if (logits)
+    CUDA_TRY(cudaMemcpyAsync(logits, c->logits, (size_t)c->B * m->cfg.vocab * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  if (legacy) {
+    CUDA_TRY(cudaEventRecord(c->ev_out, st));
+    CUDA_TRY(cudaStreamWaitEvent(nullptr, c->ev_out, 0));
+  }
+  c->len += n_steps;
+  return MS_OK;
+}
+
+ms_status ms_cache_export(const ms_cache* c, float* k, float* v) {
+  if (!c || !k || !v) return fail(MS_ERR_INVALID_ARG, "ms_cache_export: null argument");
+  DeviceGuard dg(c->m->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  const ms_config& g = c->m->cfg;
+  const int T = c->len, Hk = g.n_kv_heads;
+  std::vector<float> buf((size_t)T * 64);
+  for (int which = 0; which < 2; ++which) {
+    const float* src = which ? c->v : c->k;
+    float* dst = which ? v : k;
+    for (int l = 0; l < g.n_layers; ++l)
+      for (int b = 0; b < c->B; ++b)
+        for (int gg = 0; gg < Hk; ++gg) {
+          const float* s = src + l * layer_stride(c) + (((size_t)b * Hk + gg) * c->cap) * 64;
+          if (T > 0) CUDA_TRY(cudaMemcpy(buf.data(), s, (size_t)T * 64 * 4, cudaMemcpyDeviceToHost));
+          for (int t = 0; t < T; ++t)
+            memcpy(dst + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64, buf.data() + (size_t)t * 64, 64 * 4);
+        }
+  }
+  return MS_OK;
+}
+
+ms_status ms_cache_import(ms_cache* c, const float* k, const float* v, int T) {
+  if (!c || (T > 0 && (!k || !v))) return fail(MS_ERR_INVALID_ARG, "ms_cache_import: null argument");
+  if (T < 0 || T > c->cap) return fail(MS_ERR_CACHE_FULL, "ms_cache_import: T = %d outside [0, %d]", T, c->cap);
+  DeviceGuard dg(c->m->device);
+  CUDA_TRY(cudaDeviceSynchronize());
+  const ms_config& g = c->m->cfg;
+  const int Hk = g.n_kv_heads;
+  std::vector<float> buf((size_t)T * 64);
+  for (int which = 0; which < 2; ++which) {
+    float* dst = which ? c->v : c->k;
+    const float* src = which ? v : k;
+    for (int l = 0; l < g.n_layers; ++l)
+      for (int b = 0; b < c->B; ++b)
+        for (int gg = 0; gg < Hk; ++gg) {
+          for (int t = 0; t < T; ++t)
+            memcpy(buf.data() + (size_t)t * 64, src + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64, 64 * 4);
+          float* d = dst + l * layer_stride(c) + (((size_t)b * Hk + gg) * c->cap) * 64;
+          if (T > 0) CUDA_TRY(cudaMemcpy(d, buf.data(), (size_t)T * 64 * 4, cudaMemcpyHostToDevice));
+        }
+  }
+  CUDA_TRY(cudaMemcpy(c->dlen, &T, sizeof(int), cudaMemcpyHostToDevice));
+  c->len = T;
+  c->has_next = false;
+  return MS_OK;
+}
+
+ms_status ms_device_status(ms_cache* c, void* stream) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_device_status: null cache");
+  DeviceGuard dg(c->m->device);
+  CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned w = 0;
+  CUDA_TRY(cudaMemcpy(&w, c->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  const unsigned zero = 0;
+  CUDA_TRY(cudaMemcpy(c->status, &zero, sizeof(unsigned), cudaMemcpyHostToDevice));
+  if (w & ms::kErrTimeoutBit) return fail(MS_ERR_TIMEOUT, "a device-side wait ran out (status 0x%x)", w);
+  if (w & ms::kErrTokenBit) return fail(MS_ERR_TOKEN_RANGE, "a token id was outside [0, vocab) (status 0x%x)", w);
+  if (w & ms::kErrShapeBit) return fail(MS_ERR_SHAPE, "a device-side size check failed (status 0x%x)", w);
+  return MS_OK;
+}
+
+// ---- single operations ---------------------------------------------------------------
+ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, const float* scales, int N, float* y,
+                          void* stream) {
+  if (!x || !packed || !scales || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_w4: null pointer");
+  if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: need M, N >= 1, K a multiple of 256");
+  CUDA_TRY(ensure_kernel_attributes());
+  ms::WView w{packed, scales, nullptr, N, K, ms::kInt4};
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
+    return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
+  if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: N must be a multiple of 64 for this M");
+  return check_launch(ms::launch_gemm(L, w, x, K, M, y, N, ms::kStore), "gemm");
+}
+
+ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y, void* stream) {
+  if (!x || !w16 || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_f16: null pointer");
+  if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: need M, N >= 1, K a multiple of 256");
+  CUDA_TRY(ensure_kernel_attributes());
+  ms::WView w{nullptr, nullptr, w16, N, K, ms::kFp16};
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
+    return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
+  if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: N must be a multiple of 64 for this M");
+  return check_launch(ms::launch_gemm(L, w, x, K, M, y, N, ms::kStore), "gemm");
+}
+
+ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta, float eps, int R, int d,
+                               float* h, void* stream) {
+  if (!x || !gamma || !beta || !h) return fail(MS_ERR_INVALID_ARG, "ms_op_skip_layernorm: null pointer");
+  if (R < 0 || d < 128 || d % 128 != 0 || d > 2048) return fail(MS_ERR_SHAPE, "ms_op_skip_layernorm: d must be a multiple of 128 up to 2048");
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  return check_launch(ms::launch_skipln(L, x, y, gamma, beta, eps, R, d, h), "skip_layernorm");
+}
+
+ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const float* gamma, const float* beta, float eps,
+                               const float* W, int V, float* logits, int32_t* argmax, void* stream) {
+  if (!x || !W) return fail(MS_ERR_INVALID_ARG, "ms_op_lm_head_argmax: null pointer");
+  if ((gamma == nullptr) != (beta == nullptr)) return fail(MS_ERR_INVALID_ARG, "ms_op_lm_head_argmax: gamma and beta go together");
+  if (M < 1 || M > 64 || V < 1 || d < 128 || d % 128 != 0 || ldx < d || ldx % 4 != 0)
+    return fail(MS_ERR_SHAPE, "ms_op_lm_head_argmax: bad sizes");
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(ensure_kernel_attributes());
+  OpScratch sc;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if ((int)g_scratch.size() <= dev) g_scratch.resize(dev + 1);
+    OpScratch& s = g_scratch[dev];
+    if (!s.counter) {
+      // sized for the largest grid any V can give (one CTA per SM's worth of rows)
+      CUDA_TRY(cudaMalloc(&s.part_val, 1024 * 64 * sizeof(float)));
+      CUDA_TRY(cudaMalloc(&s.part_idx, 1024 * 64 * sizeof(int)));
+      CUDA_TRY(cudaMalloc(&s.counter, 256));
+      CUDA_TRY(cudaMemset(s.counter, 0, 256));
+    }
+    sc = s;
+  }
+  if (ms::lm_head_grid(V) > 1024) return fail(MS_ERR_SHAPE, "ms_op_lm_head_argmax: V too large");
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  ms::LmHeadWork w{sc.part_val, sc.part_idx, sc.counter};
+  return check_launch(ms::launch_lm_head(L, x, ldx, M, d, gamma, beta, eps, W, V, logits, argmax, nullptr, M, 0, nullptr,
+                                         0, w),
+                      "lm_head");
+}
+
+}  // extern "C"

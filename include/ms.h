@@ -1,0 +1,209 @@
+/*
+ * ms.h — C ABI of the MuScriptor KV-cached INT4 decoder step on NVIDIA B200 (sm_100a).
+ *
+ * The decoder is the one the pages describe:
+ *   - "MuScriptor small — ONNX conversion", section "muscriptor-small-lm.onnx": one
+ *     branch-free call takes tokens [1,S], the conditioner prefix [1,P,d] (P = 0 after
+ *     the first call) and the KV cache, and returns last-position logits [1,1393] and
+ *     the grown cache; positions are implicit in the cache length.
+ *   - "MuScriptor Medium — optimized W4A32 ONNX Runtime", section "Model variant":
+ *     backbone MatMuls in symmetric RTN INT4 with group size 32, activations, KV cache,
+ *     embeddings and LM head in fp32, a fixed-capacity cache shared in place between
+ *     past and present; section "Quick smoke test": capacity chosen by the caller.
+ *   - "MuScriptor — small (≈100M)" model card, "Model description": greedy (argmax)
+ *     decoding; "Model variants": the three shapes.
+ *
+ * Conventions for every call:
+ *   - Return value: MS_OK or an error code.  On error nothing was launched and no state
+ *     changed, unless the description says otherwise; ms_last_error() gives a message
+ *     for the calling thread.
+ *   - "device" pointers are CUDA device memory of the model's device; "host" pointers
+ *     are ordinary host memory; "any" pointers may be either (the library copies with
+ *     cudaMemcpyDefault).  The caller keeps ownership of everything it passes in.
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default stream).  Calls
+ *     that take a stream are asynchronous on it; device-side errors (a token id out of
+ *     range, a wait that ran out) are recorded in a status word read by ms_device_status.
+ *   - Calls on one ms_cache must not overlap on the GPU (they share its work buffers);
+ *     different caches of one model may run on different streams.
+ *
+ * Error behaviour common to all calls: a NULL handle or required pointer gives
+ * MS_ERR_INVALID_ARG; a size that does not fit the model or the cache gives MS_ERR_SHAPE;
+ * a call that would grow the cache past its capacity gives MS_ERR_CACHE_FULL and changes
+ * nothing; a failed CUDA runtime call gives MS_ERR_CUDA (the message names the call).
+ */
+#ifndef MS_H
+#define MS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ms_model ms_model;
+typedef struct ms_cache ms_cache;
+
+typedef enum {
+  MS_OK = 0,
+  MS_ERR_INVALID_ARG = 1,
+  MS_ERR_SHAPE = 2,
+  MS_ERR_CACHE_FULL = 3,
+  MS_ERR_TOKEN_RANGE = 4,
+  MS_ERR_OOM = 5,
+  MS_ERR_CUDA = 6,
+  MS_ERR_TIMEOUT = 7,
+  MS_ERR_UNSUPPORTED = 8
+} ms_status;
+
+/* Backbone weight storage.  INT4_G32: the W4A32 page's format.  FP16: the same matrices
+ * rounded to IEEE half ("MuScriptor for Core AI (.aimodel)", file table: the large model
+ * with weights cast to half), fp32 accumulation. */
+typedef enum { MS_W_INT4_G32 = 0, MS_W_FP16 = 1 } ms_weight_format;
+
+/* Model shape.  head_dim must be 64; vocab is 1393 for MuScriptor but any value >= 1 is
+ * accepted.  d_model must be a multiple of 256, d_ff a multiple of 256, n_heads a
+ * multiple of n_kv_heads, n_heads * 64 a multiple of 256. */
+typedef struct {
+  int n_layers;
+  int d_model;
+  int n_heads;
+  int n_kv_heads;
+  int head_dim;
+  int d_ff;
+  int vocab;
+  float rope_base; /* 1e4 */
+  float ln_eps;    /* 1e-5 */
+  int weight_format; /* ms_weight_format */
+} ms_config;
+
+/* One layer's weights ("any" pointers, copied at ms_model_create).
+ * Matrix order in w/s/w16: 0 = fused QKV [(H + 2 Hk) * 64][d], 1 = O [d][H * 64],
+ * 2 = FC1 [d_ff][d], 3 = FC2 [d][d_ff]; each matrix is [N][K] with row n = output
+ * feature n.  INT4: w[i] is uint8 [N][K/2], nibble u = q + 8, element 2j in the low
+ * nibble of byte j; s[i] is fp32 [N][K/32], one scale per 32 consecutive K elements.
+ * FP16: w16[i] is IEEE half bits [N][K].  The unused format's pointers may be NULL. */
+typedef struct {
+  const float* ln1_g;
+  const float* ln1_b;
+  const float* ln2_g;
+  const float* ln2_b;
+  const uint8_t* w[4];
+  const float* s[4];
+  const uint16_t* w16[4];
+} ms_layer_weights;
+
+typedef struct {
+  const float* tok_emb;  /* fp32 [vocab][d] */
+  const float* lm_head;  /* fp32 [vocab][d], logits = LN_f(x) . lm_head^T */
+  const float* ln_f_g;   /* fp32 [d] */
+  const float* ln_f_b;   /* fp32 [d] */
+  const ms_layer_weights* layers; /* host array of n_layers entries */
+} ms_weights;
+
+/* ---- INT4 quantiser -------------------------------------------------------------
+ * Symmetric round-to-nearest INT4, group 32 along K ("MuScriptor Medium — optimized
+ * W4A32 ONNX Runtime", Model variant): per group scale = absmax / 7 and
+ * q = clamp(rint(w / scale), -7, 7), both divisions IEEE fp32, ties to even; an all-zero
+ * group gets scale 0 and q = 0.  w: device fp32 [N][K] row-major; packed: device uint8
+ * [N][K/2]; scales: device fp32 [N][K/32].  K must be a multiple of 32, N >= 1.
+ * Asynchronous on stream. */
+ms_status ms_quantize_int4_g32(const float* w, int N, int K, uint8_t* packed, float* scales,
+                               void* stream);
+
+/* ---- model -------------------------------------------------------------------------
+ * Copies the weights to `device` in the library's own layout.  Synchronous.  Returns
+ * MS_ERR_SHAPE for an unsupported shape, MS_ERR_OOM when device memory runs out. */
+ms_status ms_model_create(const ms_config* cfg, const ms_weights* weights, int device,
+                          ms_model** out);
+ms_status ms_model_destroy(ms_model* model);
+/* Bytes of device memory the model's weights occupy. */
+size_t ms_model_weight_bytes(const ms_model* model);
+
+/* ---- cache -------------------------------------------------------------------------
+ * A fixed-capacity fp32 KV cache for `batch` independent streams that advance together
+ * (every call appends the same number of positions to each stream), plus the work
+ * buffers one call needs.  Layout on the device: K and V each [L][batch][Hk][capacity][64].
+ * Allocates device memory; length starts at 0.  Synchronous. */
+ms_status ms_cache_create(ms_model* model, int batch, int capacity, ms_cache** out);
+ms_status ms_cache_reset(ms_cache* cache); /* length = 0; no device work */
+int ms_cache_length(const ms_cache* cache);   /* positions held (host view), -1 on NULL */
+int ms_cache_capacity(const ms_cache* cache);
+int ms_cache_batch(const ms_cache* cache);
+ms_status ms_cache_destroy(ms_cache* cache);
+/* Bytes of K plus V for a cache of this shape (no allocation): 2 * L * batch * Hk *
+ * capacity * 64 * 4.  For the medium model with Hk = 16 and capacity 2504 this is the
+ * W4A32 page's "about 469.5 MiB". Returns 0 on an invalid argument. */
+size_t ms_cache_kv_bytes(const ms_config* cfg, int batch, int capacity);
+
+/* ---- one decoder call ----------------------------------------------------------------
+ * Prefill: appends P prefix rows followed by S token rows to every stream (positions
+ * len .. len + P + S - 1), then returns the logits of the last new position and their
+ * argmax.  tokens: device int64 [batch][S] (S >= 0); prefix: device fp32 [batch][P][d]
+ * or NULL with P = 0; P + S >= 1.  logits: device fp32 [batch][vocab] or NULL; argmax:
+ * device int32 [batch] or NULL.  Token ids are device data: an id outside [0, vocab) is
+ * clamped on the device and flagged in the status word (ms_device_status then returns
+ * MS_ERR_TOKEN_RANGE).  MS_ERR_CACHE_FULL if len + P + S > capacity. */
+ms_status ms_prefill(ms_model* model, ms_cache* cache, const int64_t* tokens, int S,
+                     const float* prefix, int P, float* logits, int32_t* argmax, void* stream);
+
+/* Decode step: appends one token per stream (device int32 [batch]; may alias the
+ * previous call's argmax buffer) and returns the new position's logits and argmax
+ * (either may be NULL).  The cache is updated in place. */
+ms_status ms_decode_step(ms_model* model, ms_cache* cache, const int32_t* tokens, float* logits,
+                         int32_t* argmax, void* stream);
+
+/* Greedy loop: n_steps decode steps, each feeding the previous argmax back (the first
+ * step takes the argmax of the last prefill or decode call on this cache).  out_tokens:
+ * device int32 [n_steps][batch] receives every step's argmax; logits: device fp32
+ * [batch][vocab] receives the last step's logits, or NULL.  Runs from a CUDA graph of
+ * one step that is captured on first use and replayed; no host synchronisation. */
+ms_status ms_generate(ms_model* model, ms_cache* cache, int n_steps, int32_t* out_tokens,
+                      float* logits, void* stream);
+
+/* ---- cache transfer (host pointers, synchronous) --------------------------------------
+ * Export in the pages' layout [L][batch][T][Hk][64] (T = current length);
+ * import T positions in the same layout and set the length to T. */
+ms_status ms_cache_export(const ms_cache* cache, float* k, float* v);
+ms_status ms_cache_import(ms_cache* cache, const float* k, const float* v, int T);
+
+/* ---- status -------------------------------------------------------------------------
+ * Synchronises `stream`, reads and clears the device-side status word of `cache` and
+ * returns MS_ERR_TOKEN_RANGE or MS_ERR_TIMEOUT if a kernel recorded one, else MS_OK. */
+ms_status ms_device_status(ms_cache* cache, void* stream);
+/* Number of CUDA kernels the calls on this cache have launched so far: direct launches
+ * plus, for every replay of a captured graph, the kernels in that graph.  Host counter,
+ * no device work. */
+uint64_t ms_cache_kernel_launches(const ms_cache* cache);
+/* Message of the last error on the calling thread ("" if none). */
+const char* ms_last_error(void);
+
+/* ---- single operations (the kernels the calls above are made of) ----------------------
+ * For kernel-level tests and for callers that assemble their own pipeline.  All
+ * pointers are device pointers of the current device; all calls are asynchronous. */
+
+/* y[m][n] = sum_k x[m][k] * W[n][k] with W the INT4 g32 dequantised matrix
+ * (W[n][k] = q[n][k] * s[n][k/32]).  x fp32 [M][K], y fp32 [M][N].  M <= 8 runs the
+ * decode GEMV, larger M the prefill GEMM.  K a multiple of 256. */
+ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, const float* scales,
+                          int N, float* y, void* stream);
+/* The same with IEEE half weights w16 [N][K]. */
+ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y,
+                           void* stream);
+/* SkipLayerNorm ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model variant):
+ * s = x + y (y may be NULL: plain LayerNorm), x <- s, h = (s - mean) / sqrt(var + eps)
+ * * gamma + beta with the biased variance, per row of d.  x, y, h fp32 [R][d]. */
+ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta,
+                               float eps, int R, int d, float* h, void* stream);
+/* LM head and greedy choice: logits[m][v] = LN(x_m) . W[v] (LN skipped when gamma is
+ * NULL), argmax[m] = lowest index of the largest logit.  x fp32 rows at stride ldx
+ * floats, W fp32 [V][d].  M <= 64. */
+ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const float* gamma,
+                               const float* beta, float eps, const float* W, int V, float* logits,
+                               int32_t* argmax, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MS_H */

@@ -1,0 +1,246 @@
+"""Decoder-level parity through the C ABI against the oracle.
+
+Acceptance, from the benchmark spec of parity: teacher-forced logits within max-abs 2e-3
+at every compared step; greedy tokens equal wherever the oracle's top-2 logit margin is
+above 1e-2 (after the first step below that margin the greedy runs may legitimately part,
+so the comparison stops there and the teacher-forced check carries on).  Teacher forcing
+uses the oracle's own greedy tokens or a seeded token sequence, never tokens produced by
+the GPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import ms_oracle as O
+
+pytestmark = pytest.mark.gpu
+ms = pytest.importorskip("decoder_only_transformer_int4_b200")
+
+TOL = 2e-3
+MARGIN = 1e-2
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _build(shape, fmt="int4", ln_random=False, seed=0, std=0.02):
+    draw = synth.make_weights(shape, seed=seed, std=std, ln_random=ln_random)
+    return draw, O.OracleModel(draw, fmt), ms.Model.from_draw(draw, fmt)
+
+
+def _greedy_agree(gpu_tokens, ora_tokens, ora_logits):
+    """Compare greedy tokens up to (and including) the first low-margin step."""
+    margins = O.top2_margin(ora_logits)
+    for i, (a, b) in enumerate(zip(gpu_tokens, ora_tokens)):
+        if margins[i] <= MARGIN:
+            return i
+        assert a == b, f"step {i}: gpu {a} oracle {b} (margin {margins[i]:.4f})"
+    return len(ora_tokens)
+
+
+def _run_teacher_forced(gm, batch, cap, prefix, forced, start):
+    """Prefill [prefix; start] then decode the forced tokens one by one.  Returns logits
+    [steps + 1, B, V] (row 0 from the prefill)."""
+    cache = ms.Cache(gm, batch, cap)
+    lg, am = cache.prefill(_dev(start.reshape(batch, 1).astype(np.int64)), _dev(prefix))
+    rows = [lg.cpu().numpy()]
+    for i in range(forced.shape[1]):
+        lg, am = cache.decode_step(_dev(forced[:, i].astype(np.int32)))
+        rows.append(lg.cpu().numpy())
+    assert cache.device_status() == ms.MS_OK
+    return np.stack(rows), cache
+
+
+TINY = [
+    # (layers, d, heads, kv heads, d_ff, vocab)
+    (2, 256, 4, 4, 512, 300),
+    (2, 256, 4, 2, 512, 300),
+    (2, 256, 4, 1, 512, 1393),
+    (1, 768, 12, 4, 1024, 500),     # 3 query heads per kv head
+    (1, 512, 8, 1, 512, 257),       # 8 query heads per kv head
+]
+
+
+@pytest.mark.parametrize("dims", TINY)
+@pytest.mark.parametrize("batch", [1, 3])
+def test_tiny_teacher_forced_and_greedy(dims, batch):
+    L, d, H, Hk, F, V = dims
+    sh = synth.Shape("tiny", L, d, H, Hk, F, vocab=V)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    P, steps, cap = 70, 12, 100
+    prefix = synth.make_prefix(sh, batch, prefix_len=P, seed=11)
+    start = synth.make_start_tokens(batch, vocab=V, seed=12)
+    ref_tok, ref_lg = [], []
+    for b in range(batch):
+        t, lgs = om.greedy(prefix[b], int(start[b]), steps, capacity=cap)
+        ref_tok.append(t)
+        ref_lg.append(lgs)
+    ref_tok, ref_lg = np.stack(ref_tok), np.stack(ref_lg)       # [B, steps+1], [B, steps+1, V]
+    forced = ref_tok[:, :steps]
+    got, cache = _run_teacher_forced(gm, batch, cap, prefix, forced, start)
+    err = np.abs(got.transpose(1, 0, 2) - ref_lg)
+    assert err.max() <= TOL, err.max()
+    # the cache holds the post-RoPE keys and the values of every position
+    k, v = cache.export()
+    for b in range(batch):
+        c = om.new_cache(cap)
+        om.prefill(c, prefix[b], [int(start[b])])
+        for t in forced[b]:
+            om.decode_step(c, int(t))
+        ok, ov = c.export()
+        assert np.max(np.abs(k[:, b] - ok[:, 0])) < 1e-4 and np.max(np.abs(v[:, b] - ov[:, 0])) < 1e-4
+    # free-running greedy from a fresh cache, graph-replayed
+    cache2 = ms.Cache(gm, batch, cap)
+    _, am = cache2.prefill(_dev(start.reshape(batch, 1)), _dev(prefix))
+    toks, last = cache2.generate(steps)
+    gpu_tok = np.concatenate([am.cpu().numpy()[None], toks.cpu().numpy()], 0).T   # [B, steps+1]
+    for b in range(batch):
+        _greedy_agree(gpu_tok[b], ref_tok[b], ref_lg[b])
+    assert cache2.length == P + 1 + steps
+
+
+@pytest.mark.parametrize("batch", [1, 2, 4, 8, 16])
+def test_batched_streams_are_independent(batch):
+    sh = synth.Shape("tiny-b", 2, 256, 4, 2, 512, vocab=211)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    P, steps, cap = 33, 6, 48
+    prefix = synth.make_prefix(sh, batch, prefix_len=P, seed=21)
+    start = synth.make_start_tokens(batch, vocab=211, seed=22)
+    forced = synth.make_token_sequence(steps, batch, vocab=211, seed=23)
+    got, _ = _run_teacher_forced(gm, batch, cap, prefix, forced, start)
+    for b in range(batch):
+        ref = om.teacher_forced(prefix[b], [int(start[b])] + list(forced[b]))
+        assert np.abs(got[:, b] - ref).max() <= TOL
+
+
+def test_fp16_weights_variant():
+    sh = synth.Shape("tiny-h", 2, 512, 8, 2, 1024, vocab=400)
+    draw, om, gm = _build(sh, fmt="fp16", ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, 2, prefix_len=40, seed=31)
+    start = synth.make_start_tokens(2, vocab=400, seed=32)
+    forced = synth.make_token_sequence(5, 2, vocab=400, seed=33)
+    got, _ = _run_teacher_forced(gm, 2, 64, prefix, forced, start)
+    for b in range(2):
+        ref = om.teacher_forced(prefix[b], [int(start[b])] + list(forced[b]))
+        assert np.abs(got[:, b] - ref).max() <= TOL
+
+
+def test_prefill_in_pieces_equals_one_call():
+    sh = synth.Shape("tiny-p", 2, 256, 4, 1, 512, vocab=97)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, 1, prefix_len=65, seed=41)
+    toks = synth.make_token_sequence(9, 1, vocab=97, seed=42)
+    c1 = ms.Cache(gm, 1, 128)
+    lg1, _ = c1.prefill(_dev(toks), _dev(prefix))
+    c2 = ms.Cache(gm, 1, 128)
+    c2.prefill(None, _dev(prefix))
+    c2.prefill(_dev(toks[:, :4]), None)
+    lg2, _ = c2.prefill(_dev(toks[:, 4:]), None)
+    ref = om.teacher_forced(prefix[0], list(toks[0]))[-1]
+    assert np.abs(lg1.cpu().numpy()[0] - ref).max() <= TOL
+    assert np.abs(lg2.cpu().numpy()[0] - ref).max() <= TOL
+    assert c1.length == c2.length == 74
+
+
+def test_cache_import_resumes_decoding():
+    sh = synth.Shape("tiny-i", 2, 256, 4, 2, 512, vocab=150)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, 1, prefix_len=20, seed=51)
+    c = om.new_cache(64)
+    om.prefill(c, prefix[0], [3])
+    k, v = c.export()
+    cache = ms.Cache(gm, 1, 64)
+    cache.import_(k.astype(np.float32), v.astype(np.float32))
+    assert cache.length == 21
+    lg, _ = cache.decode_step(_dev(np.array([7], np.int32)))
+    ref = om.decode_step(c, 7)
+    assert np.abs(lg.cpu().numpy()[0] - ref).max() <= TOL
+
+
+def test_errors_cache_full_and_token_range():
+    sh = synth.Shape("tiny-e", 1, 256, 4, 4, 512, vocab=50)
+    draw, om, gm = _build(sh)
+    prefix = synth.make_prefix(sh, 1, prefix_len=10, seed=61)
+    cache = ms.Cache(gm, 1, 12)
+    cache.prefill(_dev(np.array([[1]], np.int64)), _dev(prefix))
+    cache.decode_step(_dev(np.array([2], np.int32)))
+    with pytest.raises(ms.MsError) as e:
+        cache.decode_step(_dev(np.array([2], np.int32)))
+    assert e.value.status == ms.MS_ERR_CACHE_FULL and cache.length == 12
+    with pytest.raises(ms.MsError) as e:
+        cache.generate(1)
+    assert e.value.status == ms.MS_ERR_CACHE_FULL
+    # an out-of-range token id is device data: the kernel clamps it and flags the status word
+    c2 = ms.Cache(gm, 1, 12)
+    c2.prefill(_dev(np.array([[5000]], np.int64)), _dev(prefix))
+    assert c2.device_status() == ms.MS_ERR_TOKEN_RANGE
+    assert c2.device_status() == ms.MS_OK              # reading clears it
+
+
+def test_generate_graph_equals_eager_steps():
+    sh = synth.Shape("tiny-g", 2, 256, 4, 2, 512, vocab=300)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, 2, prefix_len=50, seed=71)
+    start = synth.make_start_tokens(2, vocab=300, seed=72)
+    c1 = ms.Cache(gm, 2, 80)
+    c1.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
+    toks, lg = c1.generate(20)
+    c2 = ms.Cache(gm, 2, 80)
+    _, am = c2.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
+    eager = []
+    for _ in range(20):
+        lg2, am = c2.decode_step(am.clone())
+        eager.append(am.cpu().numpy())
+    assert np.array_equal(toks.cpu().numpy(), np.stack(eager))
+    assert np.array_equal(lg.cpu().numpy(), lg2.cpu().numpy())
+    # a second generate call continues from where the first stopped
+    more, _ = c1.generate(5)
+    for _ in range(5):
+        _, am = c2.decode_step(am.clone())
+        eager.append(am.cpu().numpy())
+    assert np.array_equal(more.cpu().numpy(), np.stack(eager[20:]))
+
+
+# ---- the benchmark workloads at full size ---------------------------------------------
+
+def _full_config(key, steps_checked, teacher_steps):
+    wl = synth.WORKLOADS[key]
+    sh = wl.shape
+    draw, om, gm = _build(sh, fmt=wl.weight_format)
+    B = wl.batch
+    prefix = synth.make_prefix(sh, B, seed=1)
+    start = synth.make_start_tokens(B, seed=2)
+    # greedy through the graph path, as the benchmark runs it
+    cache = ms.Cache(gm, B, wl.capacity)
+    _, am = cache.prefill(_dev(start.reshape(B, 1)), _dev(prefix))
+    toks, _ = cache.generate(wl.decode_steps)
+    gpu_tok = np.concatenate([am.cpu().numpy()[None], toks.cpu().numpy()], 0).T
+    assert cache.device_status() == ms.MS_OK
+    for b in range(min(B, 2)):
+        t, lgs = om.greedy(prefix[b], int(start[b]), steps_checked, capacity=wl.capacity)
+        _greedy_agree(gpu_tok[b, : steps_checked + 1], t, lgs)
+    # teacher-forced on a seeded sequence, logits compared at every forced step
+    forced = synth.make_token_sequence(teacher_steps, B, seed=3)
+    got, _ = _run_teacher_forced(gm, B, wl.capacity, prefix, forced, start)
+    for b in range(min(B, 2)):
+        ref = om.teacher_forced(prefix[b], [int(start[b])] + list(forced[b]))
+        err = np.abs(got[:, b] - ref).max()
+        assert err <= TOL, (key, b, err)
+    return gpu_tok
+
+
+def test_full_c1_small_two_layers():
+    _full_config("c1", 8, 8)
+
+
+@pytest.mark.slow
+def test_full_c2_small():
+    _full_config("c2", 64, 64)
+
+
+@pytest.mark.slow
+def test_full_c3_medium_gqa():
+    tok = _full_config("c3", 24, 40)
+    assert tok.shape == (1, 2001)
