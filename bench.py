@@ -45,6 +45,9 @@ def _args():
     ap.add_argument("--workload", default="c3", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="override the workload's decode steps (short runs for profiling)")
     ap.add_argument("--cpu-decode-steps", type=int, default=16,
                     help="decode steps in the oracle's timed sample")
     return ap.parse_args()
@@ -228,6 +231,9 @@ def run_ours(a):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wl = synth.WORKLOADS[a.workload]
+    if a.decode_steps is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, decode_steps=a.decode_steps)
     sh, B = wl.shape, wl.batch
 
     draw = synth.make_weights(sh, seed=0)
@@ -300,7 +306,7 @@ def run_ours(a):
     out_h = torch.empty((wl.decode_steps, B), dtype=torch.int32).pin_memory()
     am_h = torch.empty((B,), dtype=torch.int32).pin_memory()
     e2e_ms = []
-    for i in range(max(1, min(a.steps, 3))):
+    for i in range(0 if a.no_e2e else max(1, min(a.steps, 3))):
         cache.reset()
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -316,7 +322,7 @@ def run_ours(a):
         e2e_ms.append(e0.elapsed_time(e1))
     h2d = prefix_h.numel() * 4 + start_h.numel() * 8
     d2h = out_h.numel() * 4 + am_h.numel() * 4
-    e2e_val = world * tokens_per_step / (statistics.mean(e2e_ms) / 1e3)
+    e2e_val = world * tokens_per_step / (statistics.mean(e2e_ms) / 1e3) if e2e_ms else None
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

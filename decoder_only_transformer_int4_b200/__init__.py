@@ -72,6 +72,8 @@ _PROTOS = {
     "ms_cache_capacity": (_I, [_P]),
     "ms_cache_batch": (_I, [_P]),
     "ms_cache_kernel_launches": (ctypes.c_uint64, [_P]),
+    "ms_cache_set_decode_path": (_I, [_P, _I]),
+    "ms_cache_decode_path": (_I, [_P]),
     "ms_cache_destroy": (_I, [_P]),
     "ms_cache_kv_bytes": (ctypes.c_size_t, [ctypes.POINTER(Config), _I, _I]),
     "ms_prefill": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _P]),
@@ -263,6 +265,16 @@ class Cache:
     @property
     def kernel_launches(self) -> int:
         return int(_lib.ms_cache_kernel_launches(self._h))
+
+    PATH_AUTO, PATH_PERSISTENT, PATH_PER_OP = 0, 1, 2
+
+    def set_decode_path(self, path: int):
+        """0 automatic, 1 persistent decode kernel, 2 one kernel per operation."""
+        _check(_lib.ms_cache_set_decode_path(self._h, path), "ms_cache_set_decode_path")
+
+    @property
+    def decode_path(self) -> int:
+        return int(_lib.ms_cache_decode_path(self._h))
 
     def reset(self):
         _check(_lib.ms_cache_reset(self._h), "ms_cache_reset")

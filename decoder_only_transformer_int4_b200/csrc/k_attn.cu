@@ -24,6 +24,7 @@ constexpr int kDecThreads = 128;
 constexpr int kDecSub = 64;        // positions staged in shared memory at a time
 constexpr int kMinPerSplit = 16;   // smallest run of positions worth a CTA
 constexpr int kDecTargetCtas = 2 * 148;
+constexpr int kMaxSplits = 128;    // partials one (stream, kv head) may have
 
 struct AttnDecArgs {
   const float* q;
@@ -43,6 +44,7 @@ int attn_decode_splits(int B, int Hk, int cap) {
   int s = (kDecTargetCtas + B * Hk - 1) / (B * Hk);
   const int most = (cap + kMinPerSplit - 1) / kMinPerSplit;
   if (s > most) s = most;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s < 1) s = 1;
   return s;
 }
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
   __shared__ __align__(16) float Vs[kDecSub][64];
   __shared__ float sc[HPG][kDecSub];
   __shared__ float mh[HPG], lh[HPG], corr[HPG];
+  __shared__ float mwbuf[HPG * kMaxSplits], lbuf[HPG * kMaxSplits];
   __shared__ unsigned last;
   constexpr int kSlots = (HPG * 64 + kDecThreads - 1) / kDecThreads;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -65,8 +68,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
   int s_act = (T + kMinPerSplit - 1) / kMinPerSplit;
   if (s_act > (int)gridDim.x) s_act = gridDim.x;
   if (s_act < 1) s_act = 1;
-  if (split >= s_act) return;
   const int chunk = (T + s_act - 1) / s_act;
+  s_act = (T + chunk - 1) / chunk;  // every active split gets at least one position
+  if (split >= s_act) return;
   const int t0 = split * chunk;
   const int t1 = min(T, t0 + chunk);
 
@@ -157,19 +161,36 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
   __syncthreads();
   if (!last) return;
   __threadfence();
+  // Merge: weight of split s for head h is exp(m_s - M) with M the largest m_s; the
+  // loads of every split go out together (one round trip per step of the merge).
   const float* p0 = a.part + ((size_t)b * a.Hk + g) * a.splits * HPG * 66;
+  __shared__ float Linv[HPG];
+  for (int i = tid; i < HPG * s_act; i += kDecThreads) {
+    const int h = i / s_act, s = i - h * s_act;
+    mwbuf[h * kMaxSplits + s] = __ldcg(p0 + ((size_t)s * HPG + h) * 66);
+    lbuf[h * kMaxSplits + s] = __ldcg(p0 + ((size_t)s * HPG + h) * 66 + 1);
+  }
+  __syncthreads();
+  for (int h = warp; h < HPG; h += kDecThreads / 32) {
+    float mx = -INFINITY;
+    for (int s = lane; s < s_act; s += 32) mx = fmaxf(mx, mwbuf[h * kMaxSplits + s]);
+    mx = warp_max(mx);
+    float l = 0.f;
+    for (int s = lane; s < s_act; s += 32) {
+      const float w = expf(mwbuf[h * kMaxSplits + s] - mx);
+      mwbuf[h * kMaxSplits + s] = w;
+      l = fmaf(w, lbuf[h * kMaxSplits + s], l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) Linv[h] = 1.0f / l;
+  }
+  __syncthreads();
   for (int idx = tid; idx < HPG * 64; idx += kDecThreads) {
     const int h = idx >> 6, dd = idx & 63;
-    float M = -INFINITY;
-    for (int s = 0; s < s_act; ++s) M = fmaxf(M, __ldcg(p0 + ((size_t)s * HPG + h) * 66));
-    float Lsum = 0.f, O = 0.f;
-    for (int s = 0; s < s_act; ++s) {
-      const float* ps = p0 + ((size_t)s * HPG + h) * 66;
-      const float w = expf(__ldcg(ps) - M);
-      Lsum = fmaf(w, __ldcg(ps + 1), Lsum);
-      O = fmaf(w, __ldcg(ps + 2 + dd), O);
-    }
-    a.o[((size_t)b * a.H + g * HPG + h) * 64 + dd] = O / Lsum;
+    float O = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < s_act; ++s) O = fmaf(mwbuf[h * kMaxSplits + s], __ldcg(p0 + ((size_t)s * HPG + h) * 66 + 2 + dd), O);
+    a.o[((size_t)b * a.H + g * HPG + h) * 64 + dd] = O * Linv[h];
   }
   if (tid == 0) *ctr = 0u;
 }

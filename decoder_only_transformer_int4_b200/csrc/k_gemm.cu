@@ -15,6 +15,7 @@ struct GemmArgs {
   const float* ws;
   const uint16_t* wh;
   int N, K;
+  int ldq, lds;
   const float* x;
   int ldx, M;
   float* y;
@@ -55,8 +56,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
       const int r = tid >> 2, wd = tid & 3;
       const int n = n0 + r;
       if (FMT == kInt4) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(a.wq + (size_t)n * (K / 2) + k0 / 2 + wd * 4);
-        const float s = a.ws[(size_t)n * (K / 32) + k0 / 32];
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(a.wq + (size_t)n * a.ldq + k0 / 2 + wd * 4);
+        const float s = a.ws[(size_t)n * a.lds + k0 / 32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) Bs[wd * 8 + e][r] = nib_to_q((w >> (4 * e)) & 15u) * s;
       } else {
@@ -117,6 +118,8 @@ cudaError_t launch_gemm(const Launch& L, const WView& w, const float* x, int ldx
   a.wh = w.h;
   a.N = w.N;
   a.K = w.K;
+  a.ldq = w.ldq;
+  a.lds = w.lds;
   a.x = x;
   a.ldx = ldx;
   a.M = M;

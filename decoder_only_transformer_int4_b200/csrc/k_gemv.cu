@@ -22,6 +22,8 @@ struct GemvArgs {
   const float* ws;
   const uint16_t* wh;
   int N, K, rpc;
+  int ldq, lds;       // INT4 row strides (bytes, floats)
+  int inter;          // 1: scales follow each row's nibbles (one copy per slice)
   const float* x;
   int ldx;
   const float* ln_g;
@@ -32,11 +34,13 @@ struct GemvArgs {
   unsigned* status;
 };
 
-size_t gemv_row_bytes(int fmt, int K) { return fmt == kInt4 ? (size_t)K / 2 : (size_t)K * 2; }
-
+// Shared memory: the slice's rows (INT4: nibbles + scales), then M activation rows.
 size_t gemv_smem(int fmt, int K, int rpc, int M) {
-  size_t s = 16 + align16((size_t)rpc * gemv_row_bytes(fmt, K));
-  if (fmt == kInt4) s += align16((size_t)rpc * (K / 8));
+  size_t s = 16;
+  if (fmt == kInt4)
+    s += align16((size_t)rpc * (K / 2)) + align16((size_t)rpc * (K / 8));
+  else
+    s += align16((size_t)rpc * K * 2);
   s += (size_t)M * K * 4 + 64 * 4;
   return s;
 }
@@ -62,12 +66,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
   const int K = a.K;
   const int n0 = blockIdx.x * a.rpc;
   const int rows = min(a.rpc, a.N - n0);
-  const size_t wrow = FMT == kInt4 ? (size_t)K / 2 : (size_t)K * 2;
+  // Shared layout.  Interleaved INT4: rows of ldq bytes (nibbles then scales) back to
+  // back.  Separate INT4: all rows' nibbles, then all rows' scales.  FP16: rows of 2K bytes.
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
   unsigned char* wsm = smem + 16;
-  float* ssm = reinterpret_cast<float*>(wsm + align16((size_t)a.rpc * wrow));
-  float* xsm = ssm + (FMT == kInt4 ? align16((size_t)a.rpc * (K / 8)) / 4 : 0);
+  const size_t wregion = FMT == kInt4 ? align16((size_t)a.rpc * (K / 2)) + align16((size_t)a.rpc * (K / 8))
+                                      : align16((size_t)a.rpc * K * 2);
+  float* xsm = reinterpret_cast<float*>(wsm + wregion);
   float* red = xsm + (size_t)M * K;
+  const size_t wstride = FMT == kInt4 ? (a.inter ? (size_t)a.ldq : (size_t)K / 2) : (size_t)K * 2;
+  const float* ssm_sep = reinterpret_cast<const float*>(wsm + align16((size_t)a.rpc * (K / 2)));
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -75,13 +83,21 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
   }
   __syncthreads();
   if (tid == 0) {
-    const uint32_t wb = (uint32_t)(rows * wrow);
-    const uint32_t sb = FMT == kInt4 ? (uint32_t)(rows * (K / 8)) : 0u;
-    mbar_expect_tx(bar, wb + sb);
-    const unsigned char* wsrc = FMT == kInt4 ? reinterpret_cast<const unsigned char*>(a.wq)
-                                             : reinterpret_cast<const unsigned char*>(a.wh);
-    bulk_g2s_pieces(wsm, wsrc + (size_t)n0 * wrow, wb, bar);
-    if (sb) bulk_g2s_pieces(ssm, a.ws + (size_t)n0 * (K / 32), sb, bar);
+    if (FMT == kFp16) {
+      const uint32_t wb = (uint32_t)((size_t)rows * K * 2);
+      mbar_expect_tx(bar, wb);
+      bulk_g2s_pieces(wsm, reinterpret_cast<const unsigned char*>(a.wh) + (size_t)n0 * K * 2, wb, bar);
+    } else if (a.inter) {
+      const uint32_t wb = (uint32_t)((size_t)rows * a.ldq);
+      mbar_expect_tx(bar, wb);
+      bulk_g2s_pieces(wsm, a.wq + (size_t)n0 * a.ldq, wb, bar);
+    } else {
+      const uint32_t wb = (uint32_t)((size_t)rows * (K / 2));
+      const uint32_t sb = (uint32_t)((size_t)rows * (K / 8));
+      mbar_expect_tx(bar, wb + sb);
+      bulk_g2s_pieces(wsm, a.wq + (size_t)n0 * (K / 2), wb, bar);
+      bulk_g2s_pieces(const_cast<float*>(ssm_sep), a.ws + (size_t)n0 * (K / 32), sb, bar);
+    }
   }
 
   pdl_wait();
@@ -134,8 +150,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
 #pragma unroll
     for (int m = 0; m < M; ++m) acc[m] = 0.f;
     if (FMT == kInt4) {
-      const uint32_t* wr = reinterpret_cast<const uint32_t*>(wsm + (size_t)r * wrow);
-      const float* sr = ssm + (size_t)r * (K / 32);
+      const uint32_t* wr = reinterpret_cast<const uint32_t*>(wsm + (size_t)r * wstride);
+      const float* sr = a.inter ? reinterpret_cast<const float*>(wsm + (size_t)r * wstride + K / 2)
+                                : ssm_sep + (size_t)r * (K / 32);
 #pragma unroll 2
       for (int j = 0; j < JW; ++j) {
         const int c = lane + 32 * j;
@@ -160,7 +177,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
         }
       }
     } else {
-      const uint4* wr = reinterpret_cast<const uint4*>(wsm + (size_t)r * wrow);
+      const uint4* wr = reinterpret_cast<const uint4*>(wsm + (size_t)r * wstride);
 #pragma unroll 2
       for (int j = 0; j < JW; ++j) {
         const int c = lane + 32 * j;
@@ -260,6 +277,9 @@ cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx
   a.N = w.N;
   a.K = w.K;
   a.rpc = gemv_rpc(w.N);
+  a.ldq = w.ldq;
+  a.lds = w.lds;
+  a.inter = w.interleaved() ? 1 : 0;
   a.x = x;
   a.ldx = ldx;
   a.ln_g = ln_g;
@@ -457,18 +477,35 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
   if (!last) return;
   __threadfence();
   const int len = a.dlen ? *reinterpret_cast<volatile int*>(a.dlen) : 0;
-  if (tid < M) {
-    const int mg = a.m_base + tid;
+  // every thread takes a share of the per-CTA results, then a block argmax
+  for (int m = 0; m < M; ++m) {
+    const int mg = a.m_base + m;
     float bv = -FLT_MAX;
     int bx = INT_MAX;
-    for (int c = 0; c < (int)gridDim.x; ++c) {
+    for (int c = tid; c < (int)gridDim.x; c += kLmThreads) {
       const float v = __ldcg(a.part_val + (size_t)c * 64 + mg);
       const int i = __ldcg(a.part_idx + (size_t)c * 64 + mg);
-      if (better(v, i, bv, bx)) {
+      if (argmax_better(v, i, bv, bx)) {
         bv = v;
         bx = i;
       }
     }
+    warp_argmax(bv, bx);
+    if (lane == 0) {
+      bval[warp * M + m] = bv;
+      bidx[warp * M + m] = bx;
+    }
+  }
+  __syncthreads();
+  if (tid < M) {
+    const int mg = a.m_base + tid;
+    float bv = -FLT_MAX;
+    int bx = INT_MAX;
+    for (int w = 0; w < kLmWarps; ++w)
+      if (argmax_better(bval[w * M + tid], bidx[w * M + tid], bv, bx)) {
+        bv = bval[w * M + tid];
+        bx = bidx[w * M + tid];
+      }
     if (bx == INT_MAX) bx = 0;
     if (a.argmax) a.argmax[mg] = bx;
     if (a.hist) a.hist[(size_t)(len + a.hist_off) * a.hist_B + mg] = bx;

@@ -13,8 +13,8 @@ constexpr unsigned kErrTimeout = kErrTimeoutBit;
 constexpr unsigned kErrShape = kErrShapeBit;
 
 // Iteration limit for every spin on an mbarrier: far above any legitimate wait
-// (a few microseconds), far below a hang.
-constexpr long long kSpinLimit = 1ll << 26;
+// (a few microseconds), far below a hang (seconds at most).
+constexpr long long kSpinLimit = 1ll << 22;
 
 __device__ __forceinline__ void flag_error(unsigned* status, unsigned bit) {
   if (status) atomicOr(status, bit);
@@ -103,6 +103,23 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   __syncthreads();
   float t = lane < nw ? red[lane] : 0.f;
   return warp_sum(t);
+}
+
+// Greedy choice order: larger value first, lower index on ties.
+__device__ __forceinline__ bool argmax_better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+// (value, index) argmax over a warp; every lane gets the result.
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+    if (argmax_better(v2, i2, v, i)) {
+      v = v2;
+      i = i2;
+    }
+  }
 }
 
 // fp32 INT4 nibble -> exact float of q = u - 8 (u in [0, 15]): 2^23 + u has u in its low

@@ -20,13 +20,23 @@ struct Launch {
   unsigned* status;   // device status word (may be null)
 };
 
-// A backbone matrix [N][K] (row n = output feature n) in the library's device layout.
+// A backbone matrix [N][K] (row n = output feature n).  INT4: row n's nibbles start at
+// q + n * ldq (bytes) and its K/32 scales at s + n * lds (floats).  The model keeps each
+// row as [K/2 nibble bytes | K/32 fp32 scales] (ldq = 5K/8, s = q + K/2, lds = ldq / 4),
+// so one contiguous copy moves a slice of rows with their scales; the single-operation
+// entry points pass the C ABI's separate arrays (ldq = K/2, lds = K/32).  FP16: row n at
+// h + n * K.
 struct WView {
-  const uint8_t* q;   // INT4 nibbles [N][K/2]
-  const float* s;     // INT4 scales [N][K/32]
-  const uint16_t* h;  // fp16 [N][K]
+  const uint8_t* q;
+  const float* s;
+  const uint16_t* h;
   int N, K;
   int fmt;            // WFmt
+  int ldq;            // bytes between INT4 rows
+  int lds;            // floats between scale rows
+  bool interleaved() const {
+    return fmt == kInt4 && reinterpret_cast<const uint8_t*>(s) == q + K / 2 && lds * 4 == ldq;
+  }
 };
 
 // Opt every kernel that needs it into large dynamic shared memory on the current device.

@@ -33,9 +33,18 @@ constexpr size_t kMaxDynSmem = 227 * 1024;
 
 // Raise the kernel's dynamic shared memory limit when it needs more than 48 KiB.  Done once
 // per device before any launch (never during stream capture).
+// `bytes` is capped at the device's opt-in limit minus the kernel's static shared memory.
 template <typename... KArgs>
 inline cudaError_t allow_smem(void (*kernel)(KArgs...), size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa;
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+  if (e != cudaSuccess) return e;
+  const size_t most = (size_t)optin > fa.sharedSizeBytes ? (size_t)optin - fa.sharedSizeBytes : 0;
+  if (bytes > most) bytes = most;
   return cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel),
                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }

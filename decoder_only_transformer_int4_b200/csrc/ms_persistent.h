@@ -1,0 +1,59 @@
+// Arguments of the persistent decode kernel (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ms {
+
+// One layer as the persistent kernel sees it.  w[i]: rows of matrix i (QKV, O, FC1, FC2);
+// INT4 rows are [K/2 nibble bytes | K/32 fp32 scales], fp16 rows are K halves.
+struct PLayer {
+  const float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+  const uint8_t* w[4];
+};
+
+struct PersistArgs {
+  int L, d, H, Hk, F, V, fmt;
+  float eps;
+  const float* tok_emb;
+  const float* lm_head;
+  const float* lnf_g;
+  const float* lnf_b;
+  const PLayer* layers;      // device array [L]
+  int cap;
+  float* kc;                 // K cache base; layer l at kc + l * layer_stride
+  float* vc;
+  size_t layer_stride;
+  const float* cosv;         // RoPE table [cap][32]
+  const float* sinv;
+  int* dlen;                 // cache length (device)
+  int32_t* hist;             // token history [cap][B]: argmax of position p at p * B + b
+  unsigned* status;
+  float* x;                  // residual [B][d]
+  float* qkv;                // [B][(H + 2Hk) * 64]
+  float* o;                  // [B][H * 64]
+  float* u;                  // [B][d_ff]
+  float* part;               // attention partials [B][Hk][att_splits][hpg][66]
+  unsigned* att_counters;    // [B][Hk]
+  int att_splits;
+  float* lm_val;             // [grid][64]
+  int* lm_idx;
+  unsigned* lm_counter;
+  unsigned* bar_count;       // grid barrier: arrivals, completed epoch, abort word
+  unsigned* bar_flag;
+  unsigned* abort;
+  const int32_t* tokens_in;  // tokens of the first step [B], or null: take hist[(len - 1) * B + b]
+  float* logits;             // [B][V] written every step, or null
+  int32_t* argmax_out;       // [B] last step's argmax, or null
+  int n_steps;
+  int nslot;
+};
+
+cudaError_t init_attrs_persistent();
+// Ring slots that fit next to the kernel's other shared memory (0: the kernel does not fit).
+int persistent_slots(int M, int d, int H, int F, size_t smem_optin);
+size_t persistent_smem(int M, int d, int H, int F, int nslot);
+int persistent_max_ctas(int M, int fmt, size_t smem);
+cudaError_t launch_decode_persistent(const PersistArgs& a, int M, int grid, size_t smem, cudaStream_t st);
+
+}  // namespace ms

@@ -15,6 +15,7 @@
 #include "../../include/ms.h"
 #include "ms_kernels.h"
 #include "ms_launch.cuh"
+#include "ms_persistent.h"
 
 namespace ms {
 std::atomic<unsigned long long>& launch_counter() {
@@ -138,6 +139,7 @@ cudaError_t ensure_kernel_attributes() {
   if (g_attr_done[dev]) return cudaSuccess;
   e = ms::init_attrs_gemv();
   if (e == cudaSuccess) e = ms::init_attrs_attn();
+  if (e == cudaSuccess) e = ms::init_attrs_persistent();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -150,6 +152,7 @@ struct ms_model {
   Arena arena;
   float *tok_emb = nullptr, *lm_head = nullptr, *ln_f_g = nullptr, *ln_f_b = nullptr;
   std::vector<DevLayer> layers;
+  ms::PLayer* d_players = nullptr;  // the same pointers, on the device, for the persistent kernel
 };
 
 struct ms_cache {
@@ -175,6 +178,11 @@ struct ms_cache {
   size_t gen_nodes = 0;
   cudaStream_t gen_stream = nullptr;     // used when the caller passes the legacy stream
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+  // persistent decode kernel
+  unsigned* sync3 = nullptr;             // grid barrier count, completed epoch, abort word
+  int persist_grid = 0, persist_nslot = 0;
+  size_t persist_smem = 0;
+  int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
 };
 
@@ -260,6 +268,62 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
   return e;
 }
 
+bool use_persistent(const ms_cache* c) {
+  if (c->path_request == 2) return false;
+  return c->persist_grid > 0;
+}
+
+// n_steps greedy steps in one launch of the persistent kernel.  tokens: the first step's
+// tokens (device int32 [B]) or null to continue from the token history.
+cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int n_steps, float* logits,
+                           int32_t* argmax, cudaStream_t st) {
+  const ms_config& g = m->cfg;
+  cudaError_t e = cudaMemsetAsync(c->sync3, 0, 3 * sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  ms::PersistArgs a;
+  a.L = g.n_layers;
+  a.d = g.d_model;
+  a.H = g.n_heads;
+  a.Hk = g.n_kv_heads;
+  a.F = g.d_ff;
+  a.V = g.vocab;
+  a.fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
+  a.eps = g.ln_eps;
+  a.tok_emb = m->tok_emb;
+  a.lm_head = m->lm_head;
+  a.lnf_g = m->ln_f_g;
+  a.lnf_b = m->ln_f_b;
+  a.layers = m->d_players;
+  a.cap = c->cap;
+  a.kc = c->k;
+  a.vc = c->v;
+  a.layer_stride = layer_stride(c);
+  a.cosv = c->cosv;
+  a.sinv = c->sinv;
+  a.dlen = c->dlen;
+  a.hist = c->hist;
+  a.status = c->status;
+  a.x = c->x;
+  a.qkv = c->qkv;
+  a.o = c->o;
+  a.u = c->u;
+  a.part = c->att_part;
+  a.att_counters = c->att_counters;
+  a.att_splits = c->splits;
+  a.lm_val = c->lm_val;
+  a.lm_idx = c->lm_idx;
+  a.lm_counter = c->lm_counter;
+  a.bar_count = c->sync3;
+  a.bar_flag = c->sync3 + 1;
+  a.abort = c->sync3 + 2;
+  a.tokens_in = tokens;
+  a.logits = logits;
+  a.argmax_out = argmax;
+  a.n_steps = n_steps;
+  a.nslot = c->persist_nslot;
+  return ms::launch_decode_persistent(a, c->B, c->persist_grid, c->persist_smem, st);
+}
+
 ms_status check_launch(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return MS_OK;
   return fail(MS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -329,6 +393,7 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
     m->lm_head = a.take<float>((size_t)V * d);
     m->ln_f_g = a.take<float>(d);
     m->ln_f_b = a.take<float>(d);
+    m->d_players = a.take<ms::PLayer>(c.n_layers > 0 ? c.n_layers : 1);
     m->layers.assign(c.n_layers, DevLayer{});
     for (int l = 0; l < c.n_layers; ++l) {
       DevLayer& L = m->layers[l];
@@ -347,9 +412,14 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
         w.s = nullptr;
         w.h = nullptr;
         if (w.fmt == ms::kInt4) {
-          w.q = a.take<uint8_t>((size_t)N * K / 2);
-          w.s = a.take<float>((size_t)N * K / 32);
+          // each row: K/2 nibble bytes then K/32 fp32 scales
+          w.ldq = K / 2 + K / 8;
+          w.lds = w.ldq / 4;
+          w.q = a.take<uint8_t>((size_t)N * w.ldq);
+          w.s = w.q ? reinterpret_cast<const float*>(w.q + K / 2) : nullptr;
         } else {
+          w.ldq = 0;
+          w.lds = 0;
           w.h = a.take<uint16_t>((size_t)N * K);
         }
       }
@@ -383,12 +453,27 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
     for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
       const ms::WView& w = L.w[i];
       if (w.fmt == ms::kInt4) {
-        e = cp(const_cast<uint8_t*>(w.q), lw.w[i], (size_t)w.N * w.K / 2);
-        if (e == cudaSuccess) e = cp(const_cast<float*>(w.s), lw.s[i], (size_t)w.N * w.K / 32 * 4);
+        e = cudaMemcpy2D(const_cast<uint8_t*>(w.q), w.ldq, lw.w[i], w.K / 2, w.K / 2, w.N, cudaMemcpyDefault);
+        if (e == cudaSuccess)
+          e = cudaMemcpy2D(const_cast<uint8_t*>(w.q) + w.K / 2, w.ldq, lw.s[i], w.K / 8, w.K / 8, w.N,
+                           cudaMemcpyDefault);
       } else {
         e = cp(const_cast<uint16_t*>(w.h), lw.w16[i], (size_t)w.N * w.K * 2);
       }
     }
+  }
+  if (e == cudaSuccess && c.n_layers > 0) {
+    std::vector<ms::PLayer> pl(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const DevLayer& L = m->layers[l];
+      pl[l].ln1_g = L.ln1_g;
+      pl[l].ln1_b = L.ln1_b;
+      pl[l].ln2_g = L.ln2_g;
+      pl[l].ln2_b = L.ln2_b;
+      for (int i = 0; i < 4; ++i)
+        pl[l].w[i] = L.w[i].fmt == ms::kInt4 ? L.w[i].q : reinterpret_cast<const uint8_t*>(L.w[i].h);
+    }
+    e = cudaMemcpy(m->d_players, pl.data(), pl.size() * sizeof(ms::PLayer), cudaMemcpyHostToDevice);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -424,9 +509,40 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
   c->cap = capacity;
   c->splits = ms::attn_decode_splits(batch, g.n_kv_heads, capacity);
   c->rows_cap = (size_t)batch * capacity;
+  {
+    // persistent decode kernel: one CTA per SM if its shared memory fits
+    int dev = m->device, nsm = 0, optin = 0, coop = 0;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    const bool mb = batch == 1 || batch == 2 || batch == 4 || batch == 8;
+    // every weight row (and LM head row) must fit one 16 KiB ring slot
+    int kmax = g.d_model > g.d_ff ? g.d_model : g.d_ff;
+    if (g.n_heads * 64 > kmax) kmax = g.n_heads * 64;
+    const size_t rowmax = g.weight_format == MS_W_FP16 ? (size_t)kmax * 2 : (size_t)kmax / 2 + kmax / 8;
+    const bool rows_fit = rowmax <= 16384 && (size_t)g.d_model * 4 <= 16384;
+    if (mb && rows_fit && coop && nsm > 0 && g.n_layers > 0) {
+      // leave room for the kernel's static shared memory (under 1 KiB)
+      const int ns = ms::persistent_slots(batch, g.d_model, g.n_heads, g.d_ff, (size_t)optin - 2048);
+      if (ns >= 4) {
+        const size_t sm_bytes = ms::persistent_smem(batch, g.d_model, g.n_heads, g.d_ff, ns);
+        const int fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
+        if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1) {
+          c->persist_grid = nsm;
+          c->persist_nslot = ns;
+          c->persist_smem = sm_bytes;
+          int s = nsm / (batch * g.n_kv_heads);
+          if (s > 128) s = 128;
+          if (s > c->splits) c->splits = s;
+        }
+      }
+    }
+    cudaGetLastError();
+  }
   const int hpg = g.n_heads / g.n_kv_heads;
   const size_t R = c->rows_cap;
-  const int lmg = ms::lm_head_grid(g.vocab);
+  int lmg = ms::lm_head_grid(g.vocab);
+  if (lmg < 1024) lmg = 1024;  // room for the persistent kernel's one entry per CTA
   for (int pass = 0; pass < 2; ++pass) {
     Arena& a = c->arena;
     a.used = 0;
@@ -437,6 +553,7 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->dlen = a.take<int>(4);
     c->status = a.take<unsigned>(4);
     c->lm_counter = a.take<unsigned>(4);
+    c->sync3 = a.take<unsigned>(4);
     c->att_counters = a.take<unsigned>((size_t)batch * g.n_kv_heads);
     c->hist = a.take<int32_t>((size_t)capacity * batch);
     c->att_part = a.take<float>((size_t)batch * g.n_kv_heads * c->splits * hpg * 66);
@@ -518,6 +635,20 @@ ms_status ms_cache_reset(ms_cache* c) {
 
 int ms_cache_length(const ms_cache* c) { return c ? c->len : -1; }
 uint64_t ms_cache_kernel_launches(const ms_cache* c) { return c ? c->launches : 0; }
+
+ms_status ms_cache_set_decode_path(ms_cache* c, int path) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_decode_path: null cache");
+  if (path < 0 || path > 2) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_decode_path: path must be 0, 1 or 2");
+  if (path == 1 && c->persist_grid == 0)
+    return fail(MS_ERR_UNSUPPORTED, "ms_cache_set_decode_path: the persistent kernel does not fit this model/batch");
+  c->path_request = path;
+  return MS_OK;
+}
+
+int ms_cache_decode_path(const ms_cache* c) {
+  if (!c) return -1;
+  return use_persistent(c) ? 1 : 2;
+}
 int ms_cache_capacity(const ms_cache* c) { return c ? c->cap : -1; }
 int ms_cache_batch(const ms_cache* c) { return c ? c->B : -1; }
 
@@ -548,7 +679,8 @@ ms_status ms_decode_step(ms_model* m, ms_cache* c, const int32_t* tokens, float*
   if (c->len + 1 > c->cap) return fail(MS_ERR_CACHE_FULL, "ms_decode_step: cache full (%d)", c->cap);
   DeviceGuard dg(m->device);
   const unsigned long long before = ms::launch_counter().load();
-  cudaError_t e = run_decode(m, c, tokens, logits, argmax, (cudaStream_t)stream, false);
+  cudaError_t e = use_persistent(c) ? run_persistent(m, c, tokens, 1, logits, argmax, (cudaStream_t)stream)
+                                    : run_decode(m, c, tokens, logits, argmax, (cudaStream_t)stream, false);
   c->launches += ms::launch_counter().load() - before;
   if (e != cudaSuccess) return check_launch(e, "ms_decode_step launch");
   c->len += 1;
@@ -566,6 +698,26 @@ ms_status ms_generate(ms_model* m, ms_cache* c, int n_steps, int32_t* out_tokens
   if ((long long)c->len + n_steps > c->cap)
     return fail(MS_ERR_CACHE_FULL, "ms_generate: %d + %d positions exceed capacity %d", c->len, n_steps, c->cap);
   DeviceGuard dg(m->device);
+  if (use_persistent(c)) {
+    cudaStream_t ps = (cudaStream_t)stream;
+    const int len0 = c->len;
+    const int chunk = 128;  // steps per launch
+    for (int done = 0; done < n_steps;) {
+      const int k = n_steps - done < chunk ? n_steps - done : chunk;
+      const unsigned long long before = ms::launch_counter().load();
+      cudaError_t e = run_persistent(m, c, nullptr, k, c->logits, nullptr, ps);
+      c->launches += ms::launch_counter().load() - before;
+      if (e != cudaSuccess) return check_launch(e, "ms_generate persistent launch");
+      done += k;
+    }
+    CUDA_TRY(cudaMemcpyAsync(out_tokens, c->hist + (size_t)len0 * c->B, (size_t)n_steps * c->B * sizeof(int32_t),
+                             cudaMemcpyDeviceToDevice, ps));
+    if (logits)
+      CUDA_TRY(cudaMemcpyAsync(logits, c->logits, (size_t)c->B * m->cfg.vocab * sizeof(float), cudaMemcpyDeviceToDevice,
+                               ps));
+    c->len += n_steps;
+    return MS_OK;
+  }
   const bool legacy = stream == nullptr;
   cudaStream_t st = legacy ? c->gen_stream : (cudaStream_t)stream;
   const int len0 = c->len;
@@ -680,7 +832,7 @@ ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, c
   if (!x || !packed || !scales || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_w4: null pointer");
   if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: need M, N >= 1, K a multiple of 256");
   CUDA_TRY(ensure_kernel_attributes());
-  ms::WView w{packed, scales, nullptr, N, K, ms::kInt4};
+  ms::WView w{packed, scales, nullptr, N, K, ms::kInt4, K / 2, K / 32};
   ms::Launch L{(cudaStream_t)stream, false, nullptr};
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
@@ -692,7 +844,7 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
   if (!x || !w16 || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_f16: null pointer");
   if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: need M, N >= 1, K a multiple of 256");
   CUDA_TRY(ensure_kernel_attributes());
-  ms::WView w{nullptr, nullptr, w16, N, K, ms::kFp16};
+  ms::WView w{nullptr, nullptr, w16, N, K, ms::kFp16, 0, 0};
   ms::Launch L{(cudaStream_t)stream, false, nullptr};
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");

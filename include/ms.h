@@ -161,6 +161,16 @@ ms_status ms_decode_step(ms_model* model, ms_cache* cache, const int32_t* tokens
 ms_status ms_generate(ms_model* model, ms_cache* cache, int n_steps, int32_t* out_tokens,
                       float* logits, void* stream);
 
+/* Decode path for ms_decode_step and ms_generate on this cache: 0 = automatic (the
+ * persistent kernel when it fits, else one kernel per operation), 1 = the persistent
+ * kernel (MS_ERR_UNSUPPORTED when it does not fit: batch not 1, 2, 4 or 8, or its shared
+ * memory does not fit), 2 = one kernel per operation.  Both paths compute the same
+ * arithmetic; the choice only changes how the work is launched.  Host state only. */
+ms_status ms_cache_set_decode_path(ms_cache* cache, int path);
+/* The path the next decode call will take: 1 persistent kernel, 2 one kernel per
+ * operation; -1 on NULL. */
+int ms_cache_decode_path(const ms_cache* cache);
+
 /* ---- cache transfer (host pointers, synchronous) --------------------------------------
  * Export in the pages' layout [L][batch][T][Hk][64] (T = current length);
  * import T positions in the same layout and set the length to T. */

@@ -40,10 +40,11 @@ def _greedy_agree(gpu_tokens, ora_tokens, ora_logits):
     return len(ora_tokens)
 
 
-def _run_teacher_forced(gm, batch, cap, prefix, forced, start):
+def _run_teacher_forced(gm, batch, cap, prefix, forced, start, path=0):
     """Prefill [prefix; start] then decode the forced tokens one by one.  Returns logits
     [steps + 1, B, V] (row 0 from the prefill)."""
     cache = ms.Cache(gm, batch, cap)
+    cache.set_decode_path(path)
     lg, am = cache.prefill(_dev(start.reshape(batch, 1).astype(np.int64)), _dev(prefix))
     rows = [lg.cpu().numpy()]
     for i in range(forced.shape[1]):
@@ -63,9 +64,12 @@ TINY = [
 ]
 
 
+@pytest.mark.parametrize("path", [1, 2])
 @pytest.mark.parametrize("dims", TINY)
-@pytest.mark.parametrize("batch", [1, 3])
-def test_tiny_teacher_forced_and_greedy(dims, batch):
+@pytest.mark.parametrize("batch", [1, 2, 3])
+def test_tiny_teacher_forced_and_greedy(dims, batch, path):
+    if path == 1 and batch == 3:
+        pytest.skip("the persistent kernel serves 1, 2, 4 or 8 streams")
     L, d, H, Hk, F, V = dims
     sh = synth.Shape("tiny", L, d, H, Hk, F, vocab=V)
     draw, om, gm = _build(sh, ln_random=True, std=0.05)
@@ -79,7 +83,8 @@ def test_tiny_teacher_forced_and_greedy(dims, batch):
         ref_lg.append(lgs)
     ref_tok, ref_lg = np.stack(ref_tok), np.stack(ref_lg)       # [B, steps+1], [B, steps+1, V]
     forced = ref_tok[:, :steps]
-    got, cache = _run_teacher_forced(gm, batch, cap, prefix, forced, start)
+    got, cache = _run_teacher_forced(gm, batch, cap, prefix, forced, start, path)
+    assert cache.decode_path == (path if batch != 3 else 2)
     err = np.abs(got.transpose(1, 0, 2) - ref_lg)
     assert err.max() <= TOL, err.max()
     # the cache holds the post-RoPE keys and the values of every position
@@ -93,6 +98,7 @@ def test_tiny_teacher_forced_and_greedy(dims, batch):
         assert np.max(np.abs(k[:, b] - ok[:, 0])) < 1e-4 and np.max(np.abs(v[:, b] - ov[:, 0])) < 1e-4
     # free-running greedy from a fresh cache, graph-replayed
     cache2 = ms.Cache(gm, batch, cap)
+    cache2.set_decode_path(path)
     _, am = cache2.prefill(_dev(start.reshape(batch, 1)), _dev(prefix))
     toks, last = cache2.generate(steps)
     gpu_tok = np.concatenate([am.cpu().numpy()[None], toks.cpu().numpy()], 0).T   # [B, steps+1]
@@ -179,15 +185,18 @@ def test_errors_cache_full_and_token_range():
     assert c2.device_status() == ms.MS_OK              # reading clears it
 
 
-def test_generate_graph_equals_eager_steps():
+@pytest.mark.parametrize("path", [1, 2])
+def test_generate_equals_step_by_step(path):
     sh = synth.Shape("tiny-g", 2, 256, 4, 2, 512, vocab=300)
     draw, om, gm = _build(sh, ln_random=True, std=0.05)
     prefix = synth.make_prefix(sh, 2, prefix_len=50, seed=71)
     start = synth.make_start_tokens(2, vocab=300, seed=72)
     c1 = ms.Cache(gm, 2, 80)
+    c1.set_decode_path(path)
     c1.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
     toks, lg = c1.generate(20)
     c2 = ms.Cache(gm, 2, 80)
+    c2.set_decode_path(path)
     _, am = c2.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
     eager = []
     for _ in range(20):
@@ -201,6 +210,37 @@ def test_generate_graph_equals_eager_steps():
         _, am = c2.decode_step(am.clone())
         eager.append(am.cpu().numpy())
     assert np.array_equal(more.cpu().numpy(), np.stack(eager[20:]))
+
+
+@pytest.mark.parametrize("batch", [1, 2, 4, 8])
+def test_decode_paths_agree(batch):
+    """The persistent kernel and the one-kernel-per-operation path compute the same
+    arithmetic; only the attention split count (so the merge order) differs."""
+    sh = synth.Shape("tiny-pp", 3, 512, 8, 2, 1024, vocab=700)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, batch, prefix_len=90, seed=81)
+    start = synth.make_start_tokens(batch, vocab=700, seed=82)
+    forced = synth.make_token_sequence(10, batch, vocab=700, seed=83)
+    a, ca = _run_teacher_forced(gm, batch, 128, prefix, forced, start, path=1)
+    b, cb = _run_teacher_forced(gm, batch, 128, prefix, forced, start, path=2)
+    assert ca.decode_path == 1 and cb.decode_path == 2
+    assert np.abs(a - b).max() < 1e-4
+    ka, va = ca.export()
+    kb, vb = cb.export()
+    assert np.abs(ka - kb).max() < 1e-5 and np.abs(va - vb).max() < 1e-5
+    for b_ in range(batch):
+        ref = om.teacher_forced(prefix[b_], [int(start[b_])] + list(forced[b_]))
+        assert np.abs(a[:, b_] - ref).max() <= TOL
+
+
+def test_persistent_path_unsupported_batch_is_rejected():
+    sh = synth.Shape("tiny-u", 1, 256, 4, 4, 512, vocab=50)
+    draw, om, gm = _build(sh)
+    c = ms.Cache(gm, 3, 16)
+    with pytest.raises(ms.MsError) as e:
+        c.set_decode_path(1)
+    assert e.value.status == ms.MS_ERR_UNSUPPORTED
+    assert c.decode_path == 2
 
 
 # ---- the benchmark workloads at full size ---------------------------------------------
