@@ -86,6 +86,7 @@ _PROTOS = {
     "ms_op_matmul_f16": (_I, [_P, _I, _I, _P, _I, _P, _P]),
     "ms_op_skip_layernorm": (_I, [_P, _P, _P, _P, _F, _I, _I, _P, _P]),
     "ms_op_lm_head_argmax": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
+    "ms_op_lm_head_argmax_static": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _fn = getattr(_lib, _name)
@@ -179,6 +180,23 @@ def lm_head_argmax(x: torch.Tensor, W: torch.Tensor, gamma: Optional[torch.Tenso
     _check(_lib.ms_op_lm_head_argmax(_ptr(x), d, m, d, _ptr(gamma), _ptr(beta), eps, _ptr(W), v, _ptr(logits),
                                      _ptr(am), _stream()), "ms_op_lm_head_argmax")
     return logits, am
+
+
+def lm_head_argmax_static(x: torch.Tensor, W: torch.Tensor, gamma: Optional[torch.Tensor] = None,
+                          beta: Optional[torch.Tensor] = None, eps: float = 1e-5, logits: Optional[torch.Tensor] = None,
+                          argmax: Optional[torch.Tensor] = None):
+    """ms_op_lm_head_argmax_static: the LM head + argmax without any device allocation by
+    the library (its scratch is a fixed array inside the library).  Output tensors may be
+    passed in so that the call allocates nothing on the Python side either."""
+    m, d = x.shape
+    v = W.shape[0]
+    if logits is None:
+        logits = torch.empty((m, v), dtype=torch.float32, device=x.device)
+    if argmax is None:
+        argmax = torch.empty((m,), dtype=torch.int32, device=x.device)
+    _check(_lib.ms_op_lm_head_argmax_static(_ptr(x), d, m, d, _ptr(gamma), _ptr(beta), eps, _ptr(W), v,
+                                            _ptr(logits), _ptr(argmax), _stream()), "ms_op_lm_head_argmax_static")
+    return logits, argmax
 
 
 # ---- model and cache -------------------------------------------------------------------

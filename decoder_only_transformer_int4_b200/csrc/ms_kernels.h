@@ -39,6 +39,9 @@ struct WView {
   }
 };
 
+// Sets the message ms_last_error() returns on the calling thread.
+void set_last_error(const char* msg);
+
 // Opt every kernel that needs it into large dynamic shared memory on the current device.
 cudaError_t init_attrs_gemv();
 cudaError_t init_attrs_attn();

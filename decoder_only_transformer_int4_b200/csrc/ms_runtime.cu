@@ -146,6 +146,10 @@ cudaError_t ensure_kernel_attributes() {
 
 }  // namespace
 
+namespace ms {
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace ms
+
 struct ms_model {
   ms_config cfg;
   int device = 0;

@@ -212,6 +212,27 @@ ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const floa
                                const float* beta, float eps, const float* W, int V, float* logits,
                                int32_t* argmax, void* stream);
 
+/* The same LM head and greedy choice for callers that cannot allocate device memory.
+ * No passage of the pages corresponds to this entry point; it exists for callers such as
+ * code that runs while a CUDA stream is being captured into a graph (cudaMalloc is not
+ * allowed there), code whose device memory is owned by another allocator that must see
+ * every allocation, and latency-critical paths where an allocation could synchronise
+ * the device.  ms_op_lm_head_argmax allocates a scratch buffer on its first call; this
+ * variant instead uses a fixed scratch array compiled into the library (about 128 KiB:
+ * per-CTA results for up to 256 CTAs and 64 rows, plus a counter), which every GPU that
+ * loads the library holds until the process exits.  Arguments and results are those of
+ * ms_op_lm_head_argmax.  Limits: M <= 64 and V small enough for 256 CTAs (always the
+ * case for vocabularies that fit the kernel's shared memory); larger sizes return
+ * MS_ERR_SHAPE with a message.  The first call on a device looks up the array's device
+ * address (with that device current), so make that first call before any stream
+ * capture.  Every call shares the one array and keeps the last call's contents; the
+ * counter that must start at zero is cleared on the stream before each launch.  Calls
+ * that overlap on the GPU (different streams, or different host threads) race on the
+ * array: order them on one stream.  It calls no cudaMalloc or cudaFree. */
+ms_status ms_op_lm_head_argmax_static(const float* x, int ldx, int M, int d, const float* gamma,
+                                      const float* beta, float eps, const float* W, int V,
+                                      float* logits, int32_t* argmax, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
