@@ -29,10 +29,13 @@ struct PersistArgs {
   int* dlen;                 // cache length (device)
   int32_t* hist;             // token history [cap][B]: argmax of position p at p * B + b
   unsigned* status;
-  float* x;                  // residual [B][d]
-  float* qkv;                // [B][(H + 2Hk) * 64]
-  float* o;                  // [B][H * 64]
-  float* u;                  // [B][d_ff]
+  // Activation vectors handed from phase to phase as {value, epoch} 64-bit words.
+  uint64_t* qkv_s;           // [B][(H + 2Hk) * 64]
+  uint64_t* o_s;             // [B][H * 64]
+  uint64_t* xc_s;            // residual after attention [B][d]
+  uint64_t* xe_s;            // residual after the FFN [B][d]
+  uint64_t* u_s;             // [B][d_ff]
+  unsigned epoch_base;       // epochs of this launch: epoch_base + 1 ...
   float* part;               // attention partials [B][Hk][att_splits][hpg][66]
   unsigned* att_counters;    // [B][Hk]
   int att_splits;
@@ -54,6 +57,7 @@ cudaError_t init_attrs_persistent();
 int persistent_slots(int M, int d, int H, int F, size_t smem_optin);
 size_t persistent_smem(int M, int d, int H, int F, int nslot);
 int persistent_max_ctas(int M, int fmt, size_t smem);
+size_t persistent_static_smem(int M, int fmt);  // (size_t)-1 on error
 cudaError_t launch_decode_persistent(const PersistArgs& a, int M, int grid, size_t smem, cudaStream_t st);
 
 }  // namespace ms

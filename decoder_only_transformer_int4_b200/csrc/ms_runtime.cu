@@ -184,6 +184,9 @@ struct ms_cache {
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
   // persistent decode kernel
   unsigned* sync3 = nullptr;             // grid barrier count, completed epoch, abort word
+  uint64_t *qkv_s = nullptr, *o_s = nullptr, *xc_s = nullptr, *xe_s = nullptr, *u_s = nullptr;
+  size_t stamp_bytes = 0;                // the five stamped vectors, contiguous
+  unsigned epoch_next = 0;               // first unused epoch of the stamped vectors
   int persist_grid = 0, persist_nslot = 0;
   size_t persist_smem = 0;
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
@@ -284,6 +287,14 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   const ms_config& g = m->cfg;
   cudaError_t e = cudaMemsetAsync(c->sync3, 0, 3 * sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
+  // epochs of the stamped vectors: fresh for every launch; restart from zeroed words
+  // before the 32-bit counter would wrap
+  const unsigned long long need = (unsigned long long)n_steps * 5ull * (unsigned long long)g.n_layers + 2ull;
+  if ((unsigned long long)c->epoch_next + need >= 0xFFFFFFF0ull) {
+    e = cudaMemsetAsync(c->qkv_s, 0, c->stamp_bytes, st);
+    if (e != cudaSuccess) return e;
+    c->epoch_next = 0;
+  }
   ms::PersistArgs a;
   a.L = g.n_layers;
   a.d = g.d_model;
@@ -307,10 +318,13 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.dlen = c->dlen;
   a.hist = c->hist;
   a.status = c->status;
-  a.x = c->x;
-  a.qkv = c->qkv;
-  a.o = c->o;
-  a.u = c->u;
+  a.qkv_s = c->qkv_s;
+  a.o_s = c->o_s;
+  a.xc_s = c->xc_s;
+  a.xe_s = c->xe_s;
+  a.u_s = c->u_s;
+  a.epoch_base = c->epoch_next;
+  c->epoch_next += (unsigned)need;
   a.part = c->att_part;
   a.att_counters = c->att_counters;
   a.att_splits = c->splits;
@@ -525,13 +539,16 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     if (g.n_heads * 64 > kmax) kmax = g.n_heads * 64;
     const size_t rowmax = g.weight_format == MS_W_FP16 ? (size_t)kmax * 2 : (size_t)kmax / 2 + kmax / 8;
     const bool rows_fit = rowmax <= 16384 && (size_t)g.d_model * 4 <= 16384;
-    if (mb && rows_fit && coop && nsm > 0 && g.n_layers > 0) {
-      // leave room for the kernel's static shared memory (under 1 KiB)
-      const int ns = ms::persistent_slots(batch, g.d_model, g.n_heads, g.d_ff, (size_t)optin - 2048);
+    if (mb && rows_fit && coop && nsm > 0 && g.n_layers > 0 && g.n_layers <= 64) {
+      // the ring gets what the kernel's static shared memory and its other regions leave
+      const int fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
+      const size_t st_smem = ms::persistent_static_smem(batch, fmt);
+      const int ns = st_smem < (size_t)optin
+                         ? ms::persistent_slots(batch, g.d_model, g.n_heads, g.d_ff, (size_t)optin - st_smem - 256)
+                         : 0;
       if (ns >= 4) {
         const size_t sm_bytes = ms::persistent_smem(batch, g.d_model, g.n_heads, g.d_ff, ns);
-        const int fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
-        if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1) {
+        if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1 && (g.d_model + nsm - 1) / nsm <= 16) {
           c->persist_grid = nsm;
           c->persist_nslot = ns;
           c->persist_smem = sm_bytes;
@@ -558,6 +575,18 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->status = a.take<unsigned>(4);
     c->lm_counter = a.take<unsigned>(4);
     c->sync3 = a.take<unsigned>(4);
+    {
+      const size_t n_qkv = (size_t)batch * (g.n_heads + 2 * g.n_kv_heads) * 64;
+      const size_t n_o = (size_t)batch * g.n_heads * 64;
+      const size_t n_x = (size_t)batch * g.d_model;
+      const size_t n_u = (size_t)batch * g.d_ff;
+      c->qkv_s = a.take<uint64_t>(n_qkv + n_o + 2 * n_x + n_u);
+      c->o_s = c->qkv_s ? c->qkv_s + n_qkv : nullptr;
+      c->xc_s = c->o_s ? c->o_s + n_o : nullptr;
+      c->xe_s = c->xc_s ? c->xc_s + n_x : nullptr;
+      c->u_s = c->xe_s ? c->xe_s + n_x : nullptr;
+      c->stamp_bytes = (n_qkv + n_o + 2 * n_x + n_u) * sizeof(uint64_t);
+    }
     c->att_counters = a.take<unsigned>((size_t)batch * g.n_kv_heads);
     c->hist = a.take<int32_t>((size_t)capacity * batch);
     c->att_part = a.take<float>((size_t)batch * g.n_kv_heads * c->splits * hpg * 66);
