@@ -45,6 +45,7 @@ void set_last_error(const char* msg);
 // Opt every kernel that needs it into large dynamic shared memory on the current device.
 cudaError_t init_attrs_gemv();
 cudaError_t init_attrs_attn();
+cudaError_t init_attrs_gemm_tc();
 
 cudaError_t launch_quantize_int4(const float* w, int N, int K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
@@ -72,9 +73,9 @@ cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx
                         const float* ln_g, const float* ln_b, float eps, float* y, int ldy, int epi);
 bool gemv_fits(const WView& w, int M);
 
-// General-M path (prefill, batched decode).
-cudaError_t launch_gemm(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y,
-                        int ldy, int epi);
+// General-M path on the tensor cores (tcgen05, 3xTF32): prefill and batched decode.
+cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y,
+                           int ldy, int epi);
 
 // Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
 // the combine done by the last CTA of each (stream, kv head).

@@ -140,6 +140,7 @@ cudaError_t ensure_kernel_attributes() {
   e = ms::init_attrs_gemv();
   if (e == cudaSuccess) e = ms::init_attrs_attn();
   if (e == cudaSuccess) e = ms::init_attrs_persistent();
+  if (e == cudaSuccess) e = ms::init_attrs_gemm_tc();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -215,13 +216,13 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
     float* kc = c->k + l * layer_stride(c);
     float* vc = c->v + l * layer_stride(c);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o);
-    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu);
-    if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore);
   }
   if (e == cudaSuccess)
     e = ms::launch_skipln(L, c->x, g.n_layers > 0 ? c->y : nullptr, m->ln_f_g, m->ln_f_b, g.ln_eps, R, d, c->h);
@@ -253,7 +254,7 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
       e = ms::launch_gemv(L, ly.w[0], c->x, d, B, ly.ln1_g, ly.ln1_b, g.ln_eps, c->qkv, nq, ms::kStore);
     } else {
       e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
     }
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o);
@@ -262,10 +263,10 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[3], c->u, F, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
     } else {
-      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
       if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
-      if (e == cudaSuccess) e = ms::launch_gemm(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
     }
   }
   ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
@@ -870,7 +871,7 @@ ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, c
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
   if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: N must be a multiple of 64 for this M");
-  return check_launch(ms::launch_gemm(L, w, x, K, M, y, N, ms::kStore), "gemm");
+  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore), "gemm");
 }
 
 ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y, void* stream) {
@@ -882,7 +883,7 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
   if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: N must be a multiple of 64 for this M");
-  return check_launch(ms::launch_gemm(L, w, x, K, M, y, N, ms::kStore), "gemm");
+  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore), "gemm");
 }
 
 ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta, float eps, int R, int d,
