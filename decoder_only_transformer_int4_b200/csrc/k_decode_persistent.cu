@@ -9,16 +9,17 @@
 // ring; the slot the eight warps have just finished with is refilled at once with the slice
 // nslot places ahead, so the copies run ahead of use across phase, layer and step
 // boundaries.  And the hand-off between phases needs no barrier: every activation
-// vector a phase produces (qkv, o, x, u) is written as 64-bit words {value, epoch}, each
-// element stored once, and the next phase polls the words it needs until they carry the
-// current epoch — the wait and the read are one round trip.  One grid barrier per step
-// (after the LM head) orders the rest (cache append, token history).
+// vector a phase produces (qkv, o, x, u, attention partials) is written as 64-bit words
+// {value, epoch}, each element stored once, and the consumer polls the words it needs —
+// all of them in flight at once — until they carry the current epoch: the wait and the read
+// are one round trip.  One grid barrier per step (after the LM head) orders the rest (cache
+// append, token history).
 //
 // Phases of one step (token position pos, T = pos + 1 keys):
 //   A  LN1 of x, QKV rows (raw q, k, v)                                 -> qkv
 //   B  attention unit (stream, kv head, split): RoPE of q (and of the new k, which the
 //      last split appends to the cache with v), scores over its run of positions, partial
-//      (m, l, o); the last unit of a (stream, kv head) merges the partials  -> o
+//      (m, l, o); one CTA per head then merges the splits' partials     -> o
 //   C  O rows, residual                                                  x += o Wo^T -> xc
 //   D  LN2 of x, FC1 rows, GELU                                          -> u
 //   E  FC2 rows, residual                                                x += u W2^T -> xe
@@ -26,8 +27,18 @@
 // other CTAs read them from the stamped copies.
 //   after the last layer: LN_f of x, LM head rows, per-CTA argmax, last CTA picks the token,
 //   records it in the token history and advances the cache length.
-// The arithmetic per element is the same as the separate kernels' (fp32, INT4 codes
-// converted exactly, one scale FMA per 32-element group).
+//
+// Matrix-vector products.  A CTA owns whole tiles of 8 weight rows; the tile-packed weights
+// (records of 8 rows x 32 columns, one group of INT4 scales each) stream through the ring,
+// and the eight warps split each slot's records evenly.  Per record a warp runs two
+// m16n8k16 tensor-core MMAs with the weights as B (8 rows = the 8 columns n; INT4 codes
+// turned into exact fp16 integers with one mask and one fp16 op per pair) and the
+// activation as A: the fp32 vector, scaled by a power of two so that its largest element is
+// below 2^14, is written once per phase as an fp16 pair hi + lo (hi = fp16(x), lo =
+// fp16(x - hi)), i.e. 22 significant bits, in rows 2m and 2m + 1 of A for stream m.  The
+// products are exact and accumulate in fp32; the group's scale multiplies each record's
+// result in fp32, as in the plain dequantised product.  This replaces ~5.6 instructions per
+// weight of a CUDA-core dot product by ~2.
 //
 // Every wait is bounded: the grid barrier's spin, the stamp polls and the ring's mbarrier
 // waits give up after a limit, set the status word's timeout bit and an abort word that
@@ -41,18 +52,39 @@
 namespace ms {
 
 namespace {
-constexpr int kConsumers = 256;
-constexpr int kThreads = kConsumers;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr int kSlot = 16384;
-constexpr long long kGridSpinLimit = 1ll << 24;  // polls of the barrier flag (~10 s)
+constexpr long long kGridSpinLimit = 1ll << 24;  // polls of the barrier count (~10 s)
 constexpr int kAttSub = 64;
 constexpr int kAttMaxSplits = 128;
 constexpr int kMinPerSplit = 16;
-constexpr int kMaxOwnRows = 16;   // residual rows a CTA owns: ceil(d_model / CTAs) <= 16
-constexpr int kMaxLayers = 64;    // layer table kept in shared memory
+constexpr int kMaxTiles = 8;              // 8-row tiles of one matrix per CTA
+constexpr int kMaxOwn = 8 * kMaxTiles;    // residual rows a CTA owns
+constexpr int kMaxLayers = 64;            // layer table kept in shared memory
+constexpr int kPairBatch = 8;             // element pairs a thread has in flight per round
+constexpr int kRecInt4 = 160;             // tile-packed record: 32 code words + 8 scales
+constexpr int kRecF16 = 512;              // tile-packed record: 32 x 16 bytes of halves
+constexpr int kUnroll = 4;                // records a warp has in flight (2 for more than 4 streams)
+
+// Attention scratch (floats): q, scores, per-head running stats, the new k and v; then either
+// the staged keys/values or, for a merge, the splits' partials.
+constexpr int kAttQs = 0;
+constexpr int kAttSc = kAttQs + 8 * 64;
+constexpr int kAttSmall = kAttSc + 8 * kAttSub;   // mh[8] lh[8] corr[8] pad[8] knew[64] vnew[64]
+constexpr int kAttU = kAttSmall + 160;
+constexpr int kAttKs = kAttU;                     // [64][65]
+constexpr int kAttVs = kAttKs + kAttSub * 65;     // [64][64]
+constexpr int kMrgMw = kAttU;                     // [128]
+constexpr int kMrgLw = kMrgMw + kAttMaxSplits;    // [128]
+constexpr int kMrgOv = kMrgLw + kAttMaxSplits;    // [128][64]
+constexpr int kMrgP4 = kMrgOv + kAttMaxSplits * 64;  // [4][64]
+constexpr int kMrgLin = kMrgP4 + 256;
+constexpr int kAttFloats = (kAttVs + kAttSub * 64 > kMrgLin + 4 ? kAttVs + kAttSub * 64 : kMrgLin + 4);
+static_assert((kAttVs * 4) % 16 == 0 && (kMrgOv * 4) % 16 == 0, "float4 alignment of the attention scratch");
 
 __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// Named barrier of the consumer warps that also ORs a flag over them.
+// Named barrier of the CTA's threads that also ORs a flag over them.
 __device__ __forceinline__ bool consumer_bar_or(bool pred) {
   unsigned r;
   asm volatile(
@@ -63,50 +95,22 @@ __device__ __forceinline__ bool consumer_bar_or(bool pred) {
   return r != 0;
 }
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // No routine of this kernel is called out of line: with nearly all of the SM's unified L1
 // given to shared memory, a call's register saves (local memory) would cost a round trip
-// to L2.  Each routine has a single call site, so inlining does not grow the code.
+// to L2.
 __device__ __forceinline__ float ex(float x) { return expf(x); }
 __device__ __forceinline__ float gelu_ool(float u) { return gelu_erf(u); }
 
-// Rows [n0, n1) of an N-row matrix owned by CTA c of G (contiguous, balanced).
-__device__ __forceinline__ void partition(int N, int c, int G, int& n0, int& n1) {
-  n0 = (int)(((long long)N * c) / G);
-  n1 = (int)(((long long)N * (c + 1)) / G);
-}
-
-// Shapes of matrix mi (0 QKV, 1 O, 2 FC1, 3 FC2) and of the LM head (mi 4), as scalar
-// selects: a small array indexed at run time would live in local memory.
+// Shapes of matrix mi (0 QKV, 1 O, 2 FC1, 3 FC2), as scalar selects: a small array indexed
+// at run time would live in local memory.
 __device__ __forceinline__ int mat_N(const PersistArgs& a, int mi) {
-  return mi == 0 ? (a.H + 2 * a.Hk) * 64 : mi == 2 ? a.F : mi == 4 ? a.V : a.d;
+  return mi == 0 ? (a.H + 2 * a.Hk) * 64 : mi == 2 ? a.F : a.d;
 }
 __device__ __forceinline__ int mat_K(const PersistArgs& a, int mi) {
   return mi == 1 ? a.H * 64 : mi == 3 ? a.F : a.d;
 }
-__device__ __forceinline__ int mat_rowb(const PersistArgs& a, int mi) {
-  if (mi == 4) return a.d * 4;
-  const int K = mat_K(a, mi);
-  return a.fmt == kInt4 ? K / 2 + K / 8 : K * 2;
-}
 
-// Ring position shared by the producer and the consumers (each keeps its own copy).
+// Ring position (each consumer thread keeps its own copy).
 struct RingPos {
   int slot = 0;
   uint32_t phase = 0;
@@ -119,50 +123,64 @@ struct RingPos {
 };
 
 struct Smem {
-  uint64_t* full;
-  uint64_t* empty;
+  uint64_t* full;          // ring mbarriers [16]
+  float* red;              // reduction slots [2][8][4]
   unsigned char* ring;
-  float* act;      // activation rows / attention scratch
-  float* red;      // 64 floats
+  unsigned char* region;   // activation planes, staging, partial sums / attention scratch / LM head input
 };
 
 __device__ __forceinline__ Smem carve(unsigned char* base, int nslot) {
   Smem s;
   s.full = reinterpret_cast<uint64_t*>(base);
-  s.empty = s.full + 16;
-  s.red = reinterpret_cast<float*>(s.empty + 16);
+  s.red = reinterpret_cast<float*>(base + 128);
   s.ring = base + 1024;
-  s.act = reinterpret_cast<float*>(s.ring + (size_t)nslot * kSlot);
+  s.region = s.ring + (size_t)nslot * kSlot;
   return s;
 }
 
+// Shared-memory region of the matrix phases: A planes (2M rows of K halves, row stride
+// K/2 + 16 words so that rows 2m and 2m + 1 fall in different banks), the thread-private
+// staging of the loaded vector, and the warps' partial sums [tile][warp][m][8].
+__host__ __device__ __forceinline__ size_t plane_bytes(int M, int kmax) {
+  return align16((size_t)2 * M * (2 * kmax + 64));
+}
+__host__ __device__ __forceinline__ size_t xin_bytes(int kmax) { return align16((size_t)kmax * 4); }
+__host__ __device__ __forceinline__ size_t part_bytes(int M) { return (size_t)kMaxTiles * kWarps * M * 8 * 4; }
+__host__ __device__ __forceinline__ size_t gb_bytes(int d) { return align16((size_t)d * 8); }
+
+struct Region {
+  uint32_t* planes;
+  float2* xin;    // staged input pairs (each thread reads back only the pairs it wrote)
+  float4* gb;     // staged LayerNorm (gamma, gamma, beta, beta) per pair, likewise
+  float* part;
+};
+
 // ---------------------------------------------------------------------------------
-// Weight schedule: the CTA's slices in consumption order (per step: per layer the rows of
-// QKV, O, FC1, FC2; then the LM head rows), one ring slot each.  Thread 0 keeps a cursor
-// and issues the next slice whenever a slot comes free.
+// Weight schedule: the CTA's slices in consumption order (per step: per layer the records
+// of QKV, O, FC1, FC2; then the LM head rows), one ring slot each.  sched[s] and sched[5 + s]
+// bound the CTA's units of stage s (records for s < 4, LM head rows for s = 4).  Thread 0
+// keeps a cursor and issues the next slice whenever a slot comes free.
 // ---------------------------------------------------------------------------------
 struct Cursor {
-  int step = 0, l = 0, stage = 0, p = -1;  // stage 0..3: matrices, 4: LM head
-  const PLayer* layers = nullptr;          // the layer table (a shared-memory copy)
-  __device__ bool next(const PersistArgs& a, int c, int G, const unsigned char** src, uint32_t* bytes) {
+  int step = 0, l = 0, stage = 0, p = -1;
+  const PLayer* layers = nullptr;   // the layer table (a shared-memory copy)
+  const int* sched = nullptr;
+  __device__ bool next(const PersistArgs& a, const unsigned char** src, uint32_t* bytes) {
     for (;;) {
       if (step >= a.n_steps) return false;
-      const int N = mat_N(a, stage);
-      const int rb = mat_rowb(a, stage);
-      int n0, n1;
-      partition(N, c, G, n0, n1);
-      const int rpp = kSlot / rb;
-      p = p < 0 ? n0 : p + rpp;
-      if (p < n1) {
-        const int rows = min(rpp, n1 - p);
+      const int ub = stage == 4 ? a.d * 4 : (a.fmt == kInt4 ? kRecInt4 : kRecF16);
+      const int per = kSlot / ub;
+      p = p < 0 ? sched[stage] : p + per;
+      if (p < sched[5 + stage]) {
+        const int n = min(per, sched[5 + stage] - p);
         const PLayer& ly = layers[l];
         const unsigned char* base = stage == 0   ? ly.w[0]
                                     : stage == 1 ? ly.w[1]
                                     : stage == 2 ? ly.w[2]
                                     : stage == 3 ? ly.w[3]
                                                  : reinterpret_cast<const unsigned char*>(a.lm_head);
-        *src = base + (size_t)p * rb;
-        *bytes = (uint32_t)(rows * rb);
+        *src = base + (size_t)p * ub;
+        *bytes = (uint32_t)(n * ub);
         return true;
       }
       p = -1;
@@ -181,19 +199,8 @@ struct Cursor {
 };
 
 // ---------------------------------------------------------------------------------
-// Consumer helpers
+// Stamped words and reductions
 // ---------------------------------------------------------------------------------
-constexpr long long kPollLimit = 1ll << 22;  // re-reads of one stamped word (>= 512 ns apart) before giving up
-
-__device__ __forceinline__ float csum(float v, float* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_sum(v);
-  consumer_bar();
-  if (lane == 0) red[warp] = v;
-  consumer_bar();
-  float t = lane < kConsumers / 32 ? red[lane] : 0.f;
-  return warp_sum(t);
-}
 
 // {value, epoch} words: the value's bits in the low half, the epoch in the high half; one
 // 64-bit store / load each, so a reader sees either the old or the new word whole.
@@ -206,214 +213,351 @@ __device__ __forceinline__ uint64_t ld_stamp(const uint64_t* p) {
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
   return w;
 }
-
-// Read element i of a stamped vector, waiting until it carries epoch ep.  Returns false
-// if the wait ran out or another CTA gave up.
-// Waiting threads back off (64 ns doubling to 512 ns) so that a CTA's spinning threads do
-// not flood the L2 slices that hold the words being produced.
-__device__ __forceinline__ bool poll_slow(const uint64_t* p, unsigned ep, float& v, const PersistArgs& a);
-__device__ __forceinline__ bool poll_one(const uint64_t* p, unsigned ep, float& v, const PersistArgs& a) {
-  const uint64_t w = ld_stamp(p);
-  if ((unsigned)(w >> 32) == ep) {
-    v = __uint_as_float((unsigned)w);
-    return true;
-  }
-  return poll_slow(p, ep, v, a);
+// Two consecutive words (16-byte aligned); each element is read whole.
+__device__ __forceinline__ void ld_stamp2(const uint64_t* p, uint64_t& w0, uint64_t& w1) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
 }
-__device__ __forceinline__ bool poll_slow(const uint64_t* p, unsigned ep, float& v, const PersistArgs& a) {
-  uint64_t w = ld_stamp(p);
-  long long it = 0;
+
+// Waits until every word a thread has loaded carries epoch ep: the stale ones are read
+// again together (all in flight), with one backoff per round — never one round trip per
+// word.  Pairs (two consecutive words per load) and single words.  Returns false if the
+// wait ran out or another CTA gave up.
+constexpr long long kSettleLimit = 1ll << 23;  // rounds (each >= 64 ns apart) before giving up
+__device__ __forceinline__ bool stale2(uint64_t w0, uint64_t w1, unsigned ep) {
+  return ((unsigned)(w0 >> 32) != ep) | ((unsigned)(w1 >> 32) != ep);
+}
+__device__ __forceinline__ bool settle_wait(long long it, unsigned& ns, const PersistArgs& a) {
+  if ((it & 15) == 15) {
+    if (*reinterpret_cast<volatile unsigned*>(a.abort)) return false;
+    if (it > kSettleLimit) {
+      flag_error(a.status, kErrTimeout);
+      atomicExch(a.abort, 1u);
+      return false;
+    }
+  }
+  __nanosleep(ns);
+  if (ns < 256) ns <<= 1;
+  return true;
+}
+template <int N>
+__device__ __forceinline__ bool settle_pairs(uint64_t (&w0)[N], uint64_t (&w1)[N], const uint64_t* const (&pp)[N],
+                                             const bool (&use)[N], unsigned ep, const PersistArgs& a) {
   unsigned ns = 64;
-  while ((unsigned)(w >> 32) != ep) {
-    __nanosleep(ns);
-    if (ns < 512) ns <<= 1;
-    if ((++it & 63) == 0) {
-      if (*reinterpret_cast<volatile unsigned*>(a.abort)) return false;
-      if (it > kPollLimit) {
-        flag_error(a.status, kErrTimeout);
-        atomicExch(a.abort, 1u);
-        return false;
-      }
-    }
-    w = ld_stamp(p);
+  for (long long it = 0;; ++it) {
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < N; ++j) stale |= use[j] && stale2(w0[j], w1[j], ep);
+    if (!stale) return true;
+    if (!settle_wait(it, ns, a)) return false;
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if (use[j] && stale2(w0[j], w1[j], ep)) ld_stamp2(pp[j], w0[j], w1[j]);
   }
-  v = __uint_as_float((unsigned)w);
-  return true;
+}
+template <int N>
+__device__ __forceinline__ bool settle_words(uint64_t (&w)[N], const uint64_t* const (&pp)[N], const bool (&use)[N],
+                                             unsigned ep, const PersistArgs& a) {
+  unsigned ns = 64;
+  for (long long it = 0;; ++it) {
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < N; ++j) stale |= use[j] && (unsigned)(w[j] >> 32) != ep;
+    if (!stale) return true;
+    if (!settle_wait(it, ns, a)) return false;
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+      if (use[j] && (unsigned)(w[j] >> 32) != ep) w[j] = ld_stamp(pp[j]);
+  }
 }
 
-// Rows m < M of a stamped vector (row stride ld words) into act: de-interleaved by
-// 8-element words (elements 8c..8c+3 in one float4 array, 8c+4..8c+7 in the next) or, with
-// natural, in plain order; optionally LayerNorm'd.  All the loads of a thread go out before
-// it waits on any of them.  Returns false (for every consumer thread) on a failed wait.
-template <int M>
-__device__ __forceinline__ bool poll_act(float* act, float* red, const uint64_t* src, int ld, int K, unsigned ep,
-                                      const float* g, const float* b, float eps, bool natural, const PersistArgs& a) {
-  const int tid = threadIdx.x, KW = K / 8;
-  bool ok = true;
-  for (int m = 0; m < M; ++m) {
-    const uint64_t* s0 = src + (size_t)m * ld;
-    float* dm = act + (size_t)m * K;
-    auto slot = [&](int k) -> float& {
-      if (natural) return dm[k];
-      const int c = k >> 3, e = k & 7;
-      return dm[((e >> 2) * KW + c) * 4 + (e & 3)];
-    };
-    constexpr int kBatch = 4;
-    for (int k0 = tid; k0 < K; k0 += kConsumers * kBatch) {
-      uint64_t w[kBatch];
+// Block-wide reduction with one barrier: x summed, y and z maxed.  The slots alternate
+// between two halves, so a reduction's slots are never rewritten before every thread has
+// passed the next reduction's barrier (and so has read them).
+struct Red {
+  float* buf;
+  int par;
+};
+__device__ __forceinline__ float3 block_red(float x, float y, float z, Red& r) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int k = k0 + j * kConsumers;
-        w[j] = k < K ? ld_stamp(s0 + k) : 0;
-      }
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int k = k0 + j * kConsumers;
-        if (k < K && ok) {
-          float v = __uint_as_float((unsigned)w[j]);
-          if ((unsigned)(w[j] >> 32) != ep) ok = poll_one(s0 + k, ep, v, a);
-          slot(k) = v;
-        }
-      }
-    }
+  for (int o = 16; o; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y = fmaxf(y, __shfl_xor_sync(0xffffffffu, y, o));
+    z = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, o));
   }
-  if (consumer_bar_or(!ok)) return false;
-  if (g) {
-    for (int m = 0; m < M; ++m) {
-      float* dm = act + (size_t)m * K;
-      float s = 0.f;
-      for (int k = tid; k < K; k += kConsumers) s += dm[k];  // order-free sum over the row
-      const float mean = csum(s, red) / K;
-      float q = 0.f;
-      for (int k = tid; k < K; k += kConsumers) {
-        const float t = dm[k] - mean;
-        q += t * t;
-      }
-      const float rstd = 1.0f / sqrtf(csum(q, red) / K + eps);
-      // normalise in place; the gamma/beta index is the element's position in the row
-      for (int k = tid; k < K; k += kConsumers) {
-        int e;  // element index of storage slot k
-        if (natural) {
-          e = k;
-        } else {
-          const int half = (k >> 2) / KW, c = (k >> 2) - half * KW;
-          e = c * 8 + half * 4 + (k & 3);
-        }
-        dm[k] = (dm[k] - mean) * rstd * g[e] + b[e];
-      }
-    }
-    consumer_bar();
-  }
-  return true;
-}
-
-// Plain fp32 rows (the token embedding) into act, de-interleaved, LayerNorm'd.
-__device__ __forceinline__ void embed_act(float* act, float* red, const float* src, int K, const float* g, const float* b,
-                                       float eps) {
-  const int tid = threadIdx.x, KW = K / 8;
-  float4* d4 = reinterpret_cast<float4*>(act);
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-  float s = 0.f;
-  for (int f = tid; f < K / 4; f += kConsumers) {
-    const float4 v = s4[f];
-    d4[(f & 1) * KW + (f >> 1)] = v;
-    s += (v.x + v.y) + (v.z + v.w);
-  }
-  const float mean = csum(s, red) / K;
-  float q = 0.f;
-  for (int f = tid; f < K / 4; f += kConsumers) {
-    const float4 v = d4[(f & 1) * KW + (f >> 1)];
-    const float p0 = v.x - mean, p1 = v.y - mean, p2 = v.z - mean, p3 = v.w - mean;
-    q += (p0 * p0 + p1 * p1) + (p2 * p2 + p3 * p3);
-  }
-  const float rstd = 1.0f / sqrtf(csum(q, red) / K + eps);
-  const float4* g4 = reinterpret_cast<const float4*>(g);
-  const float4* b4 = reinterpret_cast<const float4*>(b);
-  for (int f = tid; f < K / 4; f += kConsumers) {
-    float4 v = d4[(f & 1) * KW + (f >> 1)];
-    const float4 gg = g4[f], bb = b4[f];
-    v.x = (v.x - mean) * rstd * gg.x + bb.x;
-    v.y = (v.y - mean) * rstd * gg.y + bb.y;
-    v.z = (v.z - mean) * rstd * gg.z + bb.z;
-    v.w = (v.w - mean) * rstd * gg.w + bb.w;
-    d4[(f & 1) * KW + (f >> 1)] = v;
-  }
+  float* slot = r.buf + r.par * 32;
+  if (lane == 0) *reinterpret_cast<float4*>(slot + warp * 4) = make_float4(x, y, z, 0.f);
   consumer_bar();
+  float X = 0.f, Y = 0.f, Z = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float4 v = *reinterpret_cast<const float4*>(slot + w * 4);
+    X += v.x;
+    Y = fmaxf(Y, v.y);
+    Z = fmaxf(Z, v.z);
+  }
+  r.par ^= 1;
+  return make_float3(X, Y, Z);
 }
 
-// Dot products of RB weight rows (rows r, r + 8, ... of the slot) with the M activation
-// rows.  Lane l takes the 4-byte words l + 32 j of each row; two words are loaded ahead and
-// each word's 8 products go into two chains, so a warp keeps several independent FMA
-// chains in flight.
-template <int M, int FMT>
-__device__ __forceinline__ void word_fma(const unsigned char* row, int c, int K, const float4* xa, const float4* xb,
-                                         float* acc) {
-  float q[8];
-  float sc = 1.f;
-  if (FMT == kInt4) {
-    const uint32_t wd = reinterpret_cast<const uint32_t*>(row)[c];
-    sc = reinterpret_cast<const float*>(row + K / 2)[c >> 2];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = nib_to_q((wd >> (4 * e)) & 15u);
-  } else {
-    const uint4 hv = reinterpret_cast<const uint4*>(row)[c];
-    const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f2 = __half22float2(h2[e]);
-      q[2 * e] = f2.x;
-      q[2 * e + 1] = f2.y;
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    float p0 = q[0] * xa[m].x, p1 = q[1] * xa[m].y;
-    p0 = fmaf(q[2], xa[m].z, p0);
-    p1 = fmaf(q[3], xa[m].w, p1);
-    p0 = fmaf(q[4], xb[m].x, p0);
-    p1 = fmaf(q[5], xb[m].y, p1);
-    p0 = fmaf(q[6], xb[m].z, p0);
-    p1 = fmaf(q[7], xb[m].w, p1);
-    acc[m] = FMT == kInt4 ? fmaf(sc, p0 + p1, acc[m]) : acc[m] + (p0 + p1);
-  }
+// e such that bound * 2^e < 2^14 (fp16 hi/lo pairs then stay far from overflow and keep
+// ~22 significant bits); clamped so that 2^e and 2^-e are normal floats.
+__device__ __forceinline__ int act_exp(float bound) {
+  const unsigned bits = __float_as_uint(bound);
+  if ((bits & 0x7F800000u) == 0) return 100;  // zero or subnormal bound
+  const int E = (int)((bits >> 23) & 0xFFu) - 126;   // bound < 2^E
+  return min(max(14 - E, -100), 100);
+}
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((unsigned)(127 + e) << 23); }
+// Two floats to an fp16 pair (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float half_lo(uint32_t h) {
+  float f;
+  asm("{ .reg .b16 l, u;\n mov.b32 {l, u}, %1;\n cvt.f32.f16 %0, l; }" : "=f"(f) : "r"(h));
+  return f;
+}
+__device__ __forceinline__ float half_hi(uint32_t h) {
+  float f;
+  asm("{ .reg .b16 l, u;\n mov.b32 {l, u}, %1;\n cvt.f32.f16 %0, u; }" : "=f"(f) : "r"(h));
+  return f;
+}
+// Word of pair p (elements 2p, 2p + 1) in a plane row: within each 32-element group, lane
+// quad t's four pairs (2t + 8i, i = 0..3) are adjacent, so one 16-byte load fetches a lane's
+// A fragments of both k16 steps.
+__device__ __forceinline__ int plane_word(int p) {
+  const int q = p & 15;
+  return (p >> 4) * 16 + (q & 3) * 4 + (q >> 2);
 }
 
-template <int M, int FMT, int RB>
-__device__ __forceinline__ void rows_dot(const unsigned char* buf, int rb, int r0, int nr, const float4* act, int K,
-                                         float (&acc)[RB][M]) {
-  const int lane = threadIdx.x & 31;
-  const int KW = K / 8, JW = KW / 32;
-  float acc2[RB][M];
-#pragma unroll
-  for (int i = 0; i < RB; ++i)
-#pragma unroll
-    for (int m = 0; m < M; ++m) acc[i][m] = acc2[i][m] = 0.f;
+// Source of a vector row: stamped words (wait for epoch ep) or plain floats.
+struct VecSrc {
+  const uint64_t* st;
+  const float* pl;
+  unsigned ep;
+};
+
+// Loads one vector row of K elements, optionally LayerNorm'd (g != null), into shared
+// memory: as the fp16 hi/lo A rows phi/plo scaled by 2^e (PLANES; *inv = 2^-e), or as plain
+// fp32 at act.  Every load of a round is in flight before the thread waits on any; the
+// values (and gamma, beta) are staged in shared memory, each thread reading back only the
+// pairs it wrote.  Returns false (this thread) on a failed wait; the caller ORs the outcome
+// over the CTA.
+template <bool PLANES>
+__device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* g, const float* bt, float eps,
+                                         uint32_t* phi, uint32_t* plo, float* inv, float* act, const Region& rg,
+                                         Red& red, const PersistArgs& a) {
+  const int tid = threadIdx.x, P = K >> 1;
+  float2* xin = rg.xin;
+  bool ok = true;
 #pragma unroll 1
-  for (int j = 0; j < JW; j += 2) {
-    const int c0 = lane + 32 * j, c1 = c0 + 32;
-    const bool two = j + 1 < JW;
-    float4 xa0[M], xb0[M], xa1[M], xb1[M];
+  for (int base = 0; base < P; base += kThreads * kPairBatch) {
+    uint64_t w0[kPairBatch], w1[kPairBatch];
+    const uint64_t* pp[kPairBatch];
+    bool use[kPairBatch];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      xa0[m] = act[(size_t)m * 2 * KW + c0];
-      xb0[m] = act[(size_t)m * 2 * KW + KW + c0];
-      xa1[m] = two ? act[(size_t)m * 2 * KW + c1] : make_float4(0.f, 0.f, 0.f, 0.f);
-      xb1[m] = two ? act[(size_t)m * 2 * KW + KW + c1] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int i = 0; i < RB; ++i) {
-      if (i < nr) {
-        const unsigned char* row = buf + (size_t)(r0 + 8 * i) * rb;
-        word_fma<M, FMT>(row, c0, K, xa0, xb0, acc[i]);
-        if (two) word_fma<M, FMT>(row, c1, K, xa1, xb1, acc2[i]);
+    for (int j = 0; j < kPairBatch; ++j) {
+      const int p = base + tid + j * kThreads;
+      use[j] = p < P;
+      pp[j] = src.st + 2 * (use[j] ? p : 0);
+      w0[j] = w1[j] = 0;
+      if (use[j]) {
+        if (src.st) {
+          ld_stamp2(pp[j], w0[j], w1[j]);
+        } else {
+          const float2 f = reinterpret_cast<const float2*>(src.pl)[p];
+          w0[j] = __float_as_uint(f.x);
+          w1[j] = __float_as_uint(f.y);
+        }
       }
     }
+    if (g)
+      for (int p = base + tid; p < min(P, base + kThreads * kPairBatch); p += kThreads) {
+        const float2 gv = reinterpret_cast<const float2*>(g)[p], bv = reinterpret_cast<const float2*>(bt)[p];
+        rg.gb[p] = make_float4(gv.x, gv.y, bv.x, bv.y);
+      }
+    if (src.st && ok) ok = settle_pairs<kPairBatch>(w0, w1, pp, use, src.ep, a);
+#pragma unroll
+    for (int j = 0; j < kPairBatch; ++j) {
+      const int p = base + tid + j * kThreads;
+      if (use[j]) xin[p] = make_float2(__uint_as_float((unsigned)w0[j]), __uint_as_float((unsigned)w1[j]));
+    }
+  }
+  float mean = 0.f, rstd = 1.f, bound = 0.f;
+  if (g) {
+    float s = 0.f;
+    for (int p = tid; p < P; p += kThreads) {
+      const float2 x = xin[p];
+      s += x.x + x.y;
+    }
+    mean = block_red(s, 0.f, 0.f, red).x / K;
+    float q = 0.f, am = 0.f, bm = 0.f;
+    for (int p = tid; p < P; p += kThreads) {
+      const float2 x = xin[p];
+      const float4 gb = rg.gb[p];
+      const float d0 = x.x - mean, d1 = x.y - mean;
+      q += d0 * d0 + d1 * d1;
+      am = fmaxf(am, fmaxf(fabsf(d0) * fabsf(gb.x), fabsf(d1) * fabsf(gb.y)));
+      bm = fmaxf(bm, fmaxf(fabsf(gb.z), fabsf(gb.w)));
+    }
+    const float3 r = block_red(q, am, bm, red);
+    rstd = 1.0f / sqrtf(r.x / K + eps);
+    bound = rstd * r.y + r.z;   // |LN(x)_k| <= rstd |x_k - mean| |g_k| + |b_k|
+  } else if (PLANES) {
+    float am = 0.f;
+    for (int p = tid; p < P; p += kThreads) {
+      const float2 x = xin[p];
+      am = fmaxf(am, fmaxf(fabsf(x.x), fabsf(x.y)));
+    }
+    bound = block_red(0.f, am, 0.f, red).y;
+  }
+  float sc = 1.f;
+  if (PLANES) {
+    const int e = act_exp(bound);
+    sc = exp2i(e);
+    if (tid == 0) *inv = exp2i(-e);
+  }
+  for (int p = tid; p < P; p += kThreads) {
+    const float2 x = xin[p];
+    float y0 = x.x, y1 = x.y;
+    if (g) {
+      const float4 gb = rg.gb[p];
+      y0 = (x.x - mean) * rstd * gb.x + gb.z;
+      y1 = (x.y - mean) * rstd * gb.y + gb.w;
+    }
+    if (PLANES) {
+      y0 *= sc;
+      y1 *= sc;
+      const uint32_t hi = pack_half2(y0, y1);
+      const int wd = plane_word(p);
+      phi[wd] = hi;
+      plo[wd] = pack_half2(y0 - half_lo(hi), y1 - half_hi(hi));
+    } else {
+      reinterpret_cast<float2*>(act)[p] = make_float2(y0, y1);
+    }
+  }
+  return ok;
+}
+
+// ---------------------------------------------------------------------------------
+// Matrix phases
+// ---------------------------------------------------------------------------------
+// Shared-memory loads by 32-bit shared address (volatile: never merged with a load of the
+// same address from before a barrier, where the ring slot or the planes held other data).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {  // (a & b) | c
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+// Codes u (= q + 8) in bits 0-3 and 16-19 -> halves q: 0x6400 | u is 1024 + u, minus 1032.
+__device__ __forceinline__ uint32_t q_pair_a(uint32_t w) {
+  const uint32_t h = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  uint32_t r;
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64086408u));
+  return r;
+}
+// Codes in bits 4-7 and 20-23 -> halves q: 0x6400 | (u << 4) is 1024 + 16u; / 16 - 72.
+__device__ __forceinline__ uint32_t q_pair_b(uint32_t w) {
+  const uint32_t h = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(h), "r"(0x2C002C00u), "r"(0xD480D480u));
+  return r;
+}
+// D += A B for one m16n8k16 step (A rows = activation planes, B columns = weight rows).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One record (tile, group g) of the warp's share: its contribution r (scaled by the group's
+// INT4 scales).  Lane (q = lane / 4, t = lane % 4) gets r[0], r[1] = rows 2t, 2t + 1 of the
+// tile for A row q, and r[2], r[3] the same for A row q + 8 (streams 4..7).
+template <int M, int FMT>
+__device__ __forceinline__ void mv_record(uint32_t rec, uint32_t planes, int pw, int g, float (&r)[4]) {
+  // Branch-free, so that the records a warp has in flight overlap: lanes whose A row does
+  // not exist (r >= 2M) read row 0 and zero it.
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
+  const bool alive = gid < 2 * M;
+  uint4 alo = lds_u4(planes + 4u * ((alive ? gid : 0) * pw + g * 16 + tq * 4));
+  if (M < 4) {
+    alo.x = alive ? alo.x : 0u;
+    alo.y = alive ? alo.y : 0u;
+    alo.z = alive ? alo.z : 0u;
+    alo.w = alive ? alo.w : 0u;
+  }
+  uint4 ahi = make_uint4(0u, 0u, 0u, 0u);
+  if (M > 4) ahi = lds_u4(planes + 4u * ((gid + 8) * pw + g * 16 + tq * 4));   // 2M = 16 rows
+  r[0] = r[1] = r[2] = r[3] = 0.f;
+  if (FMT == kInt4) {
+    const uint32_t w = lds_u32(rec + 4u * lane);
+    const float2 s = lds_f2(rec + 128u + 8u * tq);
+    mma16816(r, alo.x, ahi.x, alo.y, ahi.y, q_pair_a(w), q_pair_b(w));
+    mma16816(r, alo.z, ahi.z, alo.w, ahi.w, q_pair_a(w >> 8), q_pair_b(w >> 8));
+    r[0] *= s.x;
+    r[1] *= s.y;
+    r[2] *= s.x;
+    r[3] *= s.y;
+  } else {
+    const uint4 b = lds_u4(rec + 16u * lane);
+    mma16816(r, alo.x, ahi.x, alo.y, ahi.y, b.x, b.y);
+    mma16816(r, alo.z, ahi.z, alo.w, ahi.w, b.z, b.w);
+  }
+}
+
+// Adds a warp's sums for tile tl into its partial slots: hi and lo rows (lanes 4 apart)
+// first, then stream m = r / 2 (and m + 4) from the lanes with even r.
+template <int M>
+__device__ __forceinline__ void flush_tile(float (&acc)[4], float* part, int tl) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gid = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
+  if ((gid & 1) == 0) {
+    const int m = gid >> 1;
+    float* pp = part + (size_t)(tl * kWarps + warp) * M * 8;
+    if (m < M) {
+      pp[m * 8 + 2 * tq] += acc[0];
+      pp[m * 8 + 2 * tq + 1] += acc[1];
+    }
+    if (M > 4 && m + 4 < M) {
+      pp[(m + 4) * 8 + 2 * tq] += acc[2];
+      pp[(m + 4) * 8 + 2 * tq + 1] += acc[3];
+    }
   }
 #pragma unroll
-  for (int i = 0; i < RB; ++i)
-#pragma unroll
-    for (int m = 0; m < M; ++m) acc[i][m] = warp_sum(acc[i][m] + acc2[i][m]);
+  for (int i = 0; i < 4; ++i) acc[i] = 0.f;
 }
+
+// Where a matrix phase's outputs go.  mode: 0 store, 1 residual (x += value, kept in the
+// CTA's own rows and published), 2 GELU.  Outputs are {value, epoch} words at out[m * ldo + n].
+struct OutSpec {
+  int mode;
+  uint64_t* out;
+  int ldo;
+  unsigned ep;
+  float* xown;   // residual rows of this CTA, [M][kMaxOwn], first row xr0
+  int xr0;
+};
 
 // Consumer side of the ring: wait for a slot's bytes, hand it back when done.  Every
 // consumer thread waits (bounded) on its own; release() ORs the outcome over all of them
@@ -426,12 +570,11 @@ struct Consumer {
   bool got = false;
   // thread 0 only: the schedule cursor and the number of slices issued
   Cursor cur;
-  int c = 0, G = 1;
   long long issued = 0, consumed = 0;
   __device__ void issue_next() {
     const unsigned char* src;
     uint32_t bytes;
-    if (!cur.next(*a, c, G, &src, &bytes)) return;
+    if (!cur.next(*a, &src, &bytes)) return;
     const int slot = (int)(issued % a->nslot);
     mbar_expect_tx(&sm.full[slot], bytes);
     bulk_g2s(sm.ring + (size_t)slot * kSlot, src, bytes, &sm.full[slot]);
@@ -441,10 +584,11 @@ struct Consumer {
     if (threadIdx.x == 0)
       for (int i = 0; i < a->nslot; ++i) issue_next();
   }
+  // The slot's address (valid only if got: check it before reading).
   __device__ const unsigned char* acquire() {
     got = mbar_wait(&sm.full[rp.slot], rp.phase, a->status);
     if (!got) atomicExch(a->abort, 1u);
-    return got ? sm.ring + (size_t)rp.slot * kSlot : nullptr;
+    return sm.ring + (size_t)rp.slot * kSlot;
   }
   // All consumers are done with the slot: refill it with the slice nslot places ahead.
   __device__ bool release() {
@@ -469,55 +613,87 @@ struct Consumer {
   }
 };
 
-// Where a matrix phase's outputs go.  mode: 0 store, 1 residual (x += value, kept in the
-// CTA's own rows and published), 2 GELU.  Outputs are {value, epoch} words at out[m * ldo + n].
-struct OutSpec {
-  int mode;
-  uint64_t* out;
-  int ldo;
-  unsigned ep;
-  float* xown;   // residual rows of this CTA, [M][kMaxOwnRows], first row xr0
-  int xr0;
-};
-
-// One matrix phase: rows [n0, n1) of a matrix, slot by slot from the ring.  Warp w takes
-// rows w, w+8, w+16, w+24 of a slot together; lane m writes output m of each row.
+// One matrix phase over the CTA's records [rbeg, rend) (whole tiles, K/32 records each),
+// slot by slot from the ring; the A planes hold the phase's input.  The warps split each
+// slot's records into eight contiguous runs; a run's sums go to the warp's partial slots at
+// each tile change; the CTA then adds the eight warps' partials in a fixed order, scales by
+// the input's 2^-e and applies the output mode.
 template <int M, int FMT>
-__device__ __forceinline__ bool gemv_phase(Consumer& cs, const float4* act, int K, int rb, int n0, int n1,
-                                        const OutSpec e) {
-  constexpr int RB = M <= 2 ? 2 : 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rpp = kSlot / rb;
-  for (int p = n0; p < n1; p += rpp) {
-    const int rows = min(rpp, n1 - p);
-    const unsigned char* buf = cs.acquire();
-    for (int r0 = warp; buf && r0 < rows; r0 += 8 * RB) {
-      const int nr = min(RB, (rows - r0 + 7) / 8);
-      float acc[RB][M];
-      rows_dot<M, FMT, RB>(buf, rb, r0, nr, act, K, acc);
-      if (lane < M) {
+__device__ __forceinline__ bool mv_phase(Consumer& cs, const Region& rg, int K, int rbeg, int rend, const OutSpec& e,
+                                         const float* inv_s) {
+  constexpr int RB = FMT == kInt4 ? kRecInt4 : kRecF16;
+  constexpr int PER = kSlot / RB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int KG = K >> 5;
+  const int t0 = rbeg / KG, nt = (rend - rbeg) / KG;
+  const int pw = (K >> 1) + 16;
+  const uint32_t planes_s = smem_u32(rg.planes);
+  for (int i = lane; i < nt * M * 8; i += 32) {
+    const int tl = i / (M * 8);
+    rg.part[(size_t)(tl * kWarps + warp) * M * 8 + (i - tl * M * 8)] = 0.f;
+  }
+  __syncwarp();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int cur = -1;
+  for (int p = rbeg; p < rend; p += PER) {
+    const int n = min(PER, rend - p);
+    const uint32_t buf_s = smem_u32(cs.acquire());
+    if (cs.got) {
+      const int c0 = (n * warp) >> 3, c1 = (n * (warp + 1)) >> 3;
+      const int r0 = p + c0 - rbeg;
+      int tl = r0 / KG, g = r0 - tl * KG;
+      // U records at a time: their loads, conversions and MMAs are independent, so
+      // their latencies overlap; the sums then go into the accumulators in order.
+      constexpr int U = M > 4 ? kUnroll / 2 : kUnroll;
+      for (int i = c0; i < c1; i += U) {
+        float rr[U][4];
+        int gj = g;
 #pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          if (i < nr) {
-            float v = acc[i][0];
+        for (int j = 0; j < U; ++j) {
+          // past the run's end: read the run's last record (in bounds); not accumulated
+          const int ij = min(i + j, c1 - 1);
+          mv_record<M, FMT>(buf_s + (uint32_t)(ij * RB), planes_s, pw, gj, rr[j]);
+          gj = gj + 1 == KG ? 0 : gj + 1;
+        }
 #pragma unroll
-            for (int m = 1; m < M; ++m)
-              if (lane == m) v = acc[i][m];
-            const int n = p + r0 + 8 * i;
-            if (e.mode == 1) {
-              float* xo = e.xown + lane * kMaxOwnRows + (n - e.xr0);
-              v += *xo;
-              *xo = v;
-            } else if (e.mode == 2) {
-              v = gelu_ool(v);
+        for (int j = 0; j < U; ++j) {
+          if (i + j < c1) {
+            if (tl != cur) {
+              if (cur >= 0) flush_tile<M>(acc, rg.part, cur);
+              cur = tl;
             }
-            st_stamp(e.out + (size_t)lane * e.ldo + n, v, e.ep);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] += rr[j][k];
+            if (++g == KG) {
+              g = 0;
+              ++tl;
+            }
           }
         }
       }
     }
     if (!cs.release()) return false;
   }
+  if (cur >= 0) flush_tile<M>(acc, rg.part, cur);
+  consumer_bar();
+  for (int o = threadIdx.x; o < nt * 8 * M; o += kThreads) {
+    const int tl = o / (8 * M), rem = o - tl * 8 * M, m = rem >> 3, cc = rem & 7;
+    const float* pp = rg.part + (size_t)tl * kWarps * M * 8 + m * 8 + cc;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += pp[w * M * 8];
+    v *= inv_s[m];
+    const int nn = (t0 + tl) * 8 + cc;
+    if (e.mode == 1) {
+      float* xo = e.xown + m * kMaxOwn + (nn - e.xr0);
+      v += *xo;
+      *xo = v;
+    } else if (e.mode == 2) {
+      v = gelu_ool(v);
+    }
+    st_stamp(e.out + (size_t)m * e.ldo + nn, v, e.ep);
+  }
+  consumer_bar();  // the region is reused by the next phase
   return true;
 }
 
@@ -556,35 +732,38 @@ __device__ bool grid_sync(const PersistArgs& a, unsigned& epoch, int* ok_s) {
   return *ok_s != 0;
 }
 
+// Active splits of a (stream, kv head) over T keys (at least kMinPerSplit positions each, no
+// empty split) and the positions per split.
+__device__ __forceinline__ void att_split_count(int T, int S, int& s_act, int& chunk) {
+  s_act = (T + kMinPerSplit - 1) / kMinPerSplit;
+  if (s_act > S) s_act = S;
+  chunk = (T + s_act - 1) / s_act;
+  s_act = (T + chunk - 1) / chunk;
+}
+
 // Attention for one (stream b, kv head g, split) unit over keys [0, T) of layer slices
 // kc/vc; the new position pos = T - 1 comes from the stamped qkv words (epoch ep).  The
 // split holding pos appends the new key (RoPE'd) and value to the cache and uses them
-// directly.  Writes the split's partial; the last split of (b, g) to finish merges them into
-// the stamped o words (epoch ep_out).  Returns false on a failed wait.
-__device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scratch, int b, int g, int split, int S, int T,
-                                            int pos, float* kc, float* vc, unsigned ep, unsigned ep_out,
-                                            unsigned* ticket_s) {
+// directly.  With one active split it writes the normalised output o; otherwise its partial
+// (m, l, o) per head as stamped words (epoch ep_out) for the merge.  Returns false on a
+// failed wait.
+__device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scratch, int b, int g, int split, int S,
+                                            int s_act, int chunk, int T, int pos, float* kc, float* vc, unsigned ep,
+                                            unsigned ep_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = a.H, Hk = a.Hk, hpg = H / Hk;
-  int s_act = (T + kMinPerSplit - 1) / kMinPerSplit;
-  if (s_act > S) s_act = S;
-  const int chunk = (T + s_act - 1) / s_act;
-  s_act = (T + chunk - 1) / chunk;  // every active split gets at least one position
   if (split >= s_act) return true;
   const int t0 = split * chunk, t1 = min(T, t0 + chunk);
   const bool owner = t1 == T;  // this split holds the new position
-  float* qs = scratch;                         // [8][64]
-  float* Ks = qs + 8 * 64;                     // [64][65]
-  float* Vs = Ks + kAttSub * 65;               // [64][64]
-  float* sc = Vs + kAttSub * 64;               // [8][64]
-  float* mh = sc + 8 * kAttSub;                // [8]
+  float* qs = scratch + kAttQs;    // [8][64]
+  float* sc = scratch + kAttSc;    // [8][64]
+  float* mh = scratch + kAttSmall; // [8]
   float* lh = mh + 8;
   float* corr = lh + 8;
-  float* mw = corr + 8;                        // [8][kAttMaxSplits]
-  float* lw = mw + 8 * kAttMaxSplits;          // [8][kAttMaxSplits]
-  float* linv = lw + 8 * kAttMaxSplits;        // [8]
-  float* knew = linv + 8;                      // [64]
-  float* vnew = knew + 64;                     // [64]
+  float* knew = corr + 16;         // [64]
+  float* vnew = knew + 64;         // [64]
+  float* Ks = scratch + kAttKs;    // [64][65]
+  float* Vs = scratch + kAttVs;    // [64][64]
   const int nq = (H + 2 * Hk) * 64;
   const uint64_t* row = a.qkv_s + (size_t)b * nq;
   const float* cs = a.cosv + (size_t)pos * 32;
@@ -598,7 +777,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
   }
   // first run of cached keys: issue these loads before waiting on this step's q
   auto stage = [&](int c0, int cn) {
-    for (int i = tid; i < cn * 16; i += kConsumers) {
+    for (int i = tid; i < cn * 16; i += kThreads) {
       const int p = i >> 4, f = i & 15;
       if (c0 + p == pos) continue;  // the new position comes from qkv
       const float4 kv = __ldcg(reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64) + f);
@@ -610,25 +789,35 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     }
   };
   stage(t0, min(kAttSub, t1 - t0));
-  bool ok = true;
-  for (int i = tid; i < hpg * 32; i += kConsumers) {
-    const int h = i >> 5, j = i & 31;
-    float x0 = 0.f, x1 = 0.f;
-    ok = ok && poll_one(row + (g * hpg + h) * 64 + j, ep, x0, a);
-    ok = ok && poll_one(row + (g * hpg + h) * 64 + j + 32, ep, x1, a);
-    const float c = cs[j], s = sn[j];
-    qs[h * 64 + j] = (x0 * c - x1 * s) * 0.125f;
-    qs[h * 64 + j + 32] = (x0 * s + x1 * c) * 0.125f;
+  // this thread's words of q (pair j, j + 32 of head tid / 32; hpg * 32 <= 256 threads)
+  // and, in the split that holds pos, of the new v and k: all loaded, then settled together
+  const int qh = tid >> 5, qj = tid & 31;
+  uint64_t w[5];
+  const uint64_t* pp[5];
+  bool use[5];
+  pp[0] = row + (g * hpg + (tid < hpg * 32 ? qh : 0)) * 64 + qj;
+  pp[1] = pp[0] + 32;
+  pp[2] = row + (H + Hk + g) * 64 + (tid & 63);
+  pp[3] = row + (H + g) * 64 + qj;
+  pp[4] = pp[3] + 32;
+  use[0] = use[1] = tid < hpg * 32;
+  use[2] = owner && tid < 64;
+  use[3] = use[4] = owner && tid < 32;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) w[k] = use[k] ? ld_stamp(pp[k]) : 0;
+  const bool ok = settle_words<5>(w, pp, use, ep, a);
+  if (use[0]) {
+    const float x0 = __uint_as_float((unsigned)w[0]), x1 = __uint_as_float((unsigned)w[1]);
+    const float c = cs[qj], s = sn[qj];
+    qs[qh * 64 + qj] = (x0 * c - x1 * s) * 0.125f;
+    qs[qh * 64 + qj + 32] = (x0 * s + x1 * c) * 0.125f;
   }
-  if (owner && tid < 64) {
-    float v = 0.f;
-    ok = ok && poll_one(row + (H + Hk + g) * 64 + tid, ep, v, a);
+  if (use[2]) {
+    const float v = __uint_as_float((unsigned)w[2]);
     vnew[tid] = v;
     vb[(size_t)pos * 64 + tid] = v;
-    if (tid < 32) {
-      float x0 = 0.f, x1 = 0.f;
-      ok = ok && poll_one(row + (H + g) * 64 + tid, ep, x0, a);
-      ok = ok && poll_one(row + (H + g) * 64 + tid + 32, ep, x1, a);
+    if (use[3]) {
+      const float x0 = __uint_as_float((unsigned)w[3]), x1 = __uint_as_float((unsigned)w[4]);
       const float c = cs[tid], s = sn[tid];
       const float k0 = x0 * c - x1 * s, k1 = x0 * s + x1 * c;
       knew[tid] = k0;
@@ -651,7 +840,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
       Vs[p * 64 + tid] = vnew[tid];
     }
     consumer_bar();
-    for (int i = tid; i < hpg * kAttSub; i += kConsumers) {
+    for (int i = tid; i < hpg * kAttSub; i += kThreads) {
       const int h = i / kAttSub, p = i - h * kAttSub;
       float s = -INFINITY;
       if (p < cn) {
@@ -662,7 +851,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
       sc[h * kAttSub + p] = s;
     }
     consumer_bar();
-    for (int h = warp; h < hpg; h += kConsumers / 32) {
+    for (int h = warp; h < hpg; h += kWarps) {
       const float v0 = sc[h * kAttSub + lane], v1 = sc[h * kAttSub + lane + 32];
       const float mx = warp_max(fmaxf(v0, v1));
       const float mold = mh[h];
@@ -682,7 +871,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     }
     consumer_bar();
     for (int k = 0; k < 2; ++k) {
-      const int idx = tid + k * kConsumers;
+      const int idx = tid + k * kThreads;
       if (idx < hpg * 64) {
         const int h = idx >> 6, dd = idx & 63;
         float acc = oacc[k] * corr[h];
@@ -692,60 +881,105 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
       }
     }
   }
-  consumer_bar();
-  float* pb = a.part + (((size_t)b * Hk + g) * a.att_splits + split) * hpg * 66;
+  if (s_act == 1) {
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int idx = tid + k * kConsumers;
-    if (idx < hpg * 64) pb[(idx >> 6) * 66 + 2 + (idx & 63)] = oacc[k];
+    for (int k = 0; k < 2; ++k) {
+      const int idx = tid + k * kThreads;
+      if (idx < hpg * 64) {
+        const int h = idx >> 6, dd = idx & 63;
+        st_stamp(a.o_s + ((size_t)b * H + g * hpg + h) * 64 + dd, oacc[k] * (1.0f / lh[h]), ep_out);
+      }
+    }
+  } else {
+    uint64_t* pb = a.part_s + (((size_t)b * Hk + g) * S + split) * hpg * 66;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int idx = tid + k * kThreads;
+      if (idx < hpg * 64) st_stamp(pb + (idx >> 6) * 66 + 2 + (idx & 63), oacc[k], ep_out);
+    }
+    if (tid < hpg) {
+      st_stamp(pb + tid * 66 + 0, mh[tid], ep_out);
+      st_stamp(pb + tid * 66 + 1, lh[tid], ep_out);
+    }
   }
-  if (tid < hpg) {
-    pb[tid * 66 + 0] = mh[tid];
-    pb[tid * 66 + 1] = lh[tid];
+  consumer_bar();  // scratch reuse
+  return true;
+}
+
+// Merges head hl of (stream b, kv head g) from the s_act splits' stamped partials (epoch
+// ep): o = sum_s w_s o_s / sum_s w_s l_s, w_s = exp(m_s - max m).  Every load is in flight
+// before the first wait.  Returns false on a failed wait.
+__device__ __forceinline__ bool merge_head(const PersistArgs& a, float* scratch, int b, int g, int hl, int S, int s_act,
+                                        unsigned ep) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = a.H, Hk = a.Hk, hpg = H / Hk;
+  float* mw = scratch + kMrgMw;
+  float* lw = scratch + kMrgLw;
+  float* ov = scratch + kMrgOv;
+  float* p4 = scratch + kMrgP4;
+  float* lin = scratch + kMrgLin;
+  const uint64_t* p0 = a.part_s + ((size_t)b * Hk + g) * S * hpg * 66;
+  const int npairs = s_act * 33;
+  bool ok = true;
+#pragma unroll 1
+  for (int base = 0; base < npairs; base += kThreads * kPairBatch) {
+    uint64_t w0[kPairBatch], w1[kPairBatch];
+    const uint64_t* pp[kPairBatch];
+    bool use[kPairBatch];
+#pragma unroll
+    for (int j = 0; j < kPairBatch; ++j) {
+      const int q = base + tid + j * kThreads;
+      use[j] = q < npairs;
+      const int qq = use[j] ? q : 0;
+      const int s = qq / 33, e2 = qq - s * 33;
+      pp[j] = p0 + ((size_t)s * hpg + hl) * 66 + 2 * e2;
+      w0[j] = w1[j] = 0;
+      if (use[j]) ld_stamp2(pp[j], w0[j], w1[j]);
+    }
+    if (ok) ok = settle_pairs<kPairBatch>(w0, w1, pp, use, ep, a);
+#pragma unroll
+    for (int j = 0; j < kPairBatch; ++j) {
+      const int q = base + tid + j * kThreads;
+      if (use[j]) {
+        const int s = q / 33, e2 = q - s * 33;
+        const float v0 = __uint_as_float((unsigned)w0[j]), v1 = __uint_as_float((unsigned)w1[j]);
+        if (e2 == 0) {
+          mw[s] = v0;
+          lw[s] = v1;
+        } else {
+          ov[s * 64 + 2 * e2 - 2] = v0;
+          ov[s * 64 + 2 * e2 - 1] = v1;
+        }
+      }
+    }
   }
-  __threadfence();
-  consumer_bar();
-  unsigned* ctr = a.att_counters + (size_t)b * Hk + g;
-  if (tid == 0) *ticket_s = (atomicAdd(ctr, 1u) == (unsigned)(s_act - 1)) ? 1u : 0u;
-  consumer_bar();
-  if (!*ticket_s) return true;
-  __threadfence();
-  const float* p0 = a.part + ((size_t)b * Hk + g) * a.att_splits * hpg * 66;
-  for (int i = tid; i < hpg * s_act; i += kConsumers) {
-    const int h = i / s_act, s = i - h * s_act;
-    mw[h * kAttMaxSplits + s] = __ldcg(p0 + ((size_t)s * hpg + h) * 66);
-    lw[h * kAttMaxSplits + s] = __ldcg(p0 + ((size_t)s * hpg + h) * 66 + 1);
-  }
-  consumer_bar();
-  for (int h = warp; h < hpg; h += kConsumers / 32) {
+  if (consumer_bar_or(!ok)) return false;
+  if (warp == 0) {
     float mx = -INFINITY;
-    for (int s = lane; s < s_act; s += 32) mx = fmaxf(mx, mw[h * kAttMaxSplits + s]);
+    for (int s = lane; s < s_act; s += 32) mx = fmaxf(mx, mw[s]);
     mx = warp_max(mx);
     float l = 0.f;
     for (int s = lane; s < s_act; s += 32) {
-      const float w = ex(mw[h * kAttMaxSplits + s] - mx);
-      mw[h * kAttMaxSplits + s] = w;
-      l = fmaf(w, lw[h * kAttMaxSplits + s], l);
+      const float w = ex(mw[s] - mx);
+      mw[s] = w;
+      l = fmaf(w, lw[s], l);
     }
     l = warp_sum(l);
-    if (lane == 0) linv[h] = 1.0f / l;
+    if (lane == 0) *lin = 1.0f / l;
   }
   consumer_bar();
-  for (int idx = tid; idx < hpg * 64; idx += kConsumers) {
-    const int h = idx >> 6, dd = idx & 63;
-    float O = 0.f;
-    for (int s0 = 0; s0 < s_act; s0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        v[j] = s0 + j < s_act ? __ldcg(p0 + ((size_t)(s0 + j) * hpg + h) * 66 + 2 + dd) : 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (s0 + j < s_act) O = fmaf(mw[h * kAttMaxSplits + s0 + j], v[j], O);
-    }
-    st_stamp(a.o_s + ((size_t)b * H + g * hpg + h) * 64 + dd, O * linv[h], ep_out);
+  {
+    const int dd = tid & 63, qq = tid >> 6;
+    float acc = 0.f;
+    for (int s = qq; s < s_act; s += 4) acc = fmaf(mw[s], ov[s * 64 + dd], acc);
+    p4[qq * 64 + dd] = acc;
   }
-  if (tid == 0) *ctr = 0u;
+  consumer_bar();
+  if (tid < 64) {
+    const float O = (p4[tid] + p4[64 + tid]) + (p4[128 + tid] + p4[192 + tid]);
+    st_stamp(a.o_s + ((size_t)b * H + g * hpg + hl) * 64 + tid, O * *lin, ep);
+  }
+  consumer_bar();  // scratch reuse
   return true;
 }
 
@@ -756,54 +990,87 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 }  // namespace
 
 template <int M, int FMT>
-__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers);
+__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers,
+                                             const int* sched);
 
 template <int M, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) decode_persistent_kernel(const __grid_constant__ PersistArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const Smem sm = carve(smem, a.nslot);
   __shared__ PLayer layers_s[kMaxLayers];
+  __shared__ int sched_s[10];
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.nslot; ++i) mbar_init(&sm.full[i], 1);
     mbar_fence_init();
+    const int c = blockIdx.x, G = gridDim.x;
+    for (int s = 0; s < 4; ++s) {
+      const int nt = mat_N(a, s) / 8, KG = mat_K(a, s) / 32;
+      sched_s[s] = (nt * c / G) * KG;
+      sched_s[5 + s] = (nt * (c + 1) / G) * KG;
+    }
+    sched_s[4] = a.V * c / G;
+    sched_s[9] = a.V * (c + 1) / G;
   }
   for (int i = threadIdx.x; i < a.L * (int)(sizeof(PLayer) / 8); i += kThreads)
     reinterpret_cast<uint64_t*>(layers_s)[i] = reinterpret_cast<const uint64_t*>(a.layers)[i];
   __syncthreads();
   Consumer cs;
   cs.cur.layers = layers_s;
+  cs.cur.sched = sched_s;
   cs.a = &a;
   cs.sm = sm;
-  cs.c = blockIdx.x;
-  cs.G = gridDim.x;
   cs.start();
-  if (!decode_steps<M, FMT>(a, cs, sm, layers_s)) cs.drain();
+  if (!decode_steps<M, FMT>(a, cs, sm, layers_s, sched_s)) cs.drain();
 }
 
 template <int M, int FMT>
-__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers) {
+__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers,
+                                             const int* sched) {
   __shared__ int ok_s;
   __shared__ unsigned ticket_s;
   __shared__ float bval[8][8];
   __shared__ int bidx[8][8];
   __shared__ int tok_s[8];
-  __shared__ float xown[8][kMaxOwnRows];   // this CTA's residual rows (same rows in C and E)
+  __shared__ float inv_s[8];
+  __shared__ float xown[8 * kMaxOwn];   // this CTA's residual rows (same rows in C and E)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = gridDim.x;
   const int d = a.d, H = a.H, Hk = a.Hk, F = a.F, V = a.V, B = M;
+  const int hpg = H / Hk;
   const int nq = (H + 2 * Hk) * 64;
+  const int kmax = max(max(d, H * 64), F);
+  Region rg;
+  rg.planes = reinterpret_cast<uint32_t*>(sm.region);
+  rg.xin = reinterpret_cast<float2*>(sm.region + plane_bytes(M, kmax));
+  rg.gb = reinterpret_cast<float4*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax));
+  rg.part = reinterpret_cast<float*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d));
+  float* scratch = reinterpret_cast<float*>(sm.region);
+  Red red{sm.red, 0};
   unsigned epoch = 0;
   const int len0 = *a.dlen;
-  const float4* act4 = reinterpret_cast<const float4*>(sm.act);
-  int xr0, xr1;  // residual rows owned (the O and FC2 phases both have d rows)
-  partition(d, c, G, xr0, xr1);
-  int v0, v1;
-  partition(V, c, G, v0, v1);
+  // residual rows owned: the O and FC2 phases both have d rows and the same tiles
+  const int xr0 = sched[1] / (H * 2) * 8;
+  const int xr1 = sched[6] / (H * 2) * 8;
   const int units = B * Hk;
   int S = G / units;
   if (S < 1) S = 1;
   if (S > a.att_splits) S = a.att_splits;
   const unsigned per_step = 5u * a.L;
+
+  // The phase input: row m of a vector (stamped words, or the token embedding) into A
+  // planes rows 2m, 2m + 1.
+  auto load_planes = [&](const uint64_t* st, const float* emb, int ld, int K, unsigned ep, const float* g,
+                         const float* bt) -> bool {
+    bool ok = true;
+    const int pw = (K >> 1) + 16;
+#pragma unroll 1
+    for (int m = 0; m < M; ++m) {
+      const VecSrc src{st ? st + (size_t)m * ld : nullptr, emb ? emb + (size_t)tok_s[m] * d : nullptr, ep};
+      ok = load_row<true>(src, K, g, bt, a.eps, rg.planes + (2 * m) * pw, rg.planes + (2 * m + 1) * pw, &inv_s[m],
+                          nullptr, rg, red, a) && ok;
+    }
+    return !consumer_bar_or(!ok);
+  };
 
   for (int step = 0; step < a.n_steps; ++step) {
     const int pos = len0 + step;
@@ -818,51 +1085,66 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
       tok_s[tid] = t;
     }
     consumer_bar();
+    int s_act, chunk;
+    att_split_count(T, S, s_act, chunk);
     for (int l = 0; l < a.L; ++l) {
       const PLayer& ly = layers[l];
       float* kc = a.kc + (size_t)l * a.layer_stride;
       float* vc = a.vc + (size_t)l * a.layer_stride;
       const unsigned epA = ep0 + 5u * l;
-      if (l == 0) {
-        for (int m = 0; m < M; ++m)
-          for (int n = xr0 + tid; n < xr1; n += kConsumers) xown[m][n - xr0] = a.tok_emb[(size_t)tok_s[m] * d + n];
-        for (int m = 0; m < M; ++m)
-          embed_act(sm.act + (size_t)m * d, sm.red, a.tok_emb + (size_t)tok_s[m] * d, d, ly.ln1_g, ly.ln1_b, a.eps);
-      }
-      // phases A (QKV), B (attention), C (O + residual), D (FC1 + GELU), E (FC2 + residual)
+      // phases A (LN1 + QKV), B (attention), C (O + residual), D (LN2 + FC1 + GELU),
+      // E (FC2 + residual); one call site for the four matrix phases
+#pragma unroll 1
       for (int ph = 0; ph < 5; ++ph) {
-        const unsigned ep = epA + ph;
         if (ph == 1) {
           for (int u = c; u < units * S; u += G) {
             const int bg = u / S, split = u - bg * S;
-            if (!attention_unit(a, sm.act, bg / Hk, bg % Hk, split, S, T, pos, kc, vc, epA, ep, &ticket_s))
+            if (!attention_unit(a, scratch, bg / Hk, bg % Hk, split, S, s_act, chunk, T, pos, kc, vc, epA, epA + 1))
               return false;
-            consumer_bar();
           }
+          if (s_act > 1)
+            for (int u = c; u < units * S; u += G) {
+              const int bg = u / S, split = u - bg * S;
+              if (split < s_act)
+                for (int hl = split; hl < hpg; hl += s_act)
+                  if (!merge_head(a, scratch, bg / Hk, bg % Hk, hl, S, s_act, epA + 1)) return false;
+            }
           continue;
         }
-        const int mi = ph == 0 ? 0 : ph - 1;  // matrix of the phase
+        const int mi = ph == 0 ? 0 : ph - 1;   // matrix of the phase
         const int K = mat_K(a, mi);
-        if (!(ph == 0 && l == 0)) {
-          const uint64_t* src = ph == 0 ? a.xe_s : ph == 2 ? a.o_s : ph == 3 ? a.xc_s : a.u_s;
-          const float* g = ph == 0 ? ly.ln1_g : ph == 3 ? ly.ln2_g : nullptr;
-          const float* bb = ph == 0 ? ly.ln1_b : ph == 3 ? ly.ln2_b : nullptr;
-          if (!poll_act<M>(sm.act, sm.red, src, K, K, ep - 1, g, bb, a.eps, false, a)) return false;
-        }
+        const bool emb = ph == 0 && l == 0;    // layer 0 reads the token embedding
+        if (emb)
+          for (int m = 0; m < M; ++m)
+            for (int n = xr0 + tid; n < xr1; n += kThreads)
+              xown[m * kMaxOwn + n - xr0] = a.tok_emb[(size_t)tok_s[m] * d + n];
+        const uint64_t* src = emb ? nullptr : ph == 0 ? a.xe_s : ph == 2 ? a.o_s : ph == 3 ? a.xc_s : a.u_s;
+        const float* g = ph == 0 ? ly.ln1_g : ph == 3 ? ly.ln2_g : nullptr;
+        const float* bt = ph == 0 ? ly.ln1_b : ph == 3 ? ly.ln2_b : nullptr;
+        if (!load_planes(src, emb ? a.tok_emb : nullptr, K, K, epA + ph - 1, g, bt)) return false;
         OutSpec e;
         e.mode = (ph == 2 || ph == 4) ? 1 : ph == 3 ? 2 : 0;
         e.out = ph == 0 ? a.qkv_s : ph == 2 ? a.xc_s : ph == 3 ? a.u_s : a.xe_s;
         e.ldo = ph == 0 ? nq : ph == 3 ? F : d;
-        e.ep = ep;
-        e.xown = &xown[0][0];
+        e.ep = epA + ph;
+        e.xown = xown;
         e.xr0 = xr0;
-        int n0, n1;
-        partition(mat_N(a, mi), c, G, n0, n1);
-        if (!gemv_phase<M, FMT>(cs, act4, K, mat_rowb(a, mi), n0, n1, e)) return false;
+        if (!mv_phase<M, FMT>(cs, rg, K, sched[mi], sched[5 + mi], e, inv_s)) return false;
       }
     }
     // ---- LM head + argmax ------------------------------------------------------------
-    if (!poll_act<M>(sm.act, sm.red, a.xe_s, d, d, ep0 + per_step - 1, a.lnf_g, a.lnf_b, a.eps, true, a)) return false;
+    float* act = reinterpret_cast<float*>(sm.region);
+    {
+      bool ok = true;
+#pragma unroll 1
+      for (int m = 0; m < M; ++m) {
+        const VecSrc src{a.xe_s + (size_t)m * d, nullptr, ep0 + per_step - 1};
+        ok = load_row<false>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+                             red, a) && ok;
+      }
+      if (consumer_bar_or(!ok)) return false;
+    }
+    const float4* act4 = reinterpret_cast<const float4*>(act);
     float best[M];
     int bi[M];
 #pragma unroll
@@ -872,10 +1154,10 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
     }
     {
       const int rb = d * 4, rpp = kSlot / rb;
-      for (int p = v0; p < v1; p += rpp) {
-        const int rows = min(rpp, v1 - p);
+      for (int p = sched[4]; p < sched[9]; p += rpp) {
+        const int rows = min(rpp, sched[9] - p);
         const unsigned char* buf = cs.acquire();
-        for (int r = warp; buf && r < rows; r += kConsumers / 32) {
+        for (int r = warp; cs.got && r < rows; r += kWarps) {
           const float4* w4 = reinterpret_cast<const float4*>(buf + (size_t)r * rb);
           float acc[M];
 #pragma unroll
@@ -914,7 +1196,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
     if (tid < M) {
       float bv = -FLT_MAX;
       int bx = INT_MAX;
-      for (int w = 0; w < kConsumers / 32; ++w)
+      for (int w = 0; w < kWarps; ++w)
         if (better(bval[w][tid], bidx[w][tid], bv, bx)) {
           bv = bval[w][tid];
           bx = bidx[w][tid];
@@ -931,7 +1213,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
       for (int m = 0; m < M; ++m) {
         float bv = -FLT_MAX;
         int bx = INT_MAX;
-        for (int k = tid; k < G; k += kConsumers) {
+        for (int k = tid; k < G; k += kThreads) {
           const float v = __ldcg(a.lm_val + (size_t)k * 64 + m);
           const int i = __ldcg(a.lm_idx + (size_t)k * 64 + m);
           if (better(v, i, bv, bx)) {
@@ -949,7 +1231,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
       if (tid < M) {
         float bv = -FLT_MAX;
         int bx = INT_MAX;
-        for (int w = 0; w < kConsumers / 32; ++w)
+        for (int w = 0; w < kWarps; ++w)
           if (better(bval[w][tid], bidx[w][tid], bv, bx)) {
             bv = bval[w][tid];
             bx = bidx[w][tid];
@@ -974,9 +1256,12 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
 // ---------------------------------------------------------------------------------
 namespace {
 size_t persist_region(int M, int d, int H, int F) {
-  size_t act = (size_t)M * 4 * (size_t)max(max(d, H * 64), F);
-  size_t att = sizeof(float) * (8 * 64 + kAttSub * 65 + kAttSub * 64 + 8 * kAttSub + 24 + 2 * 8 * kAttMaxSplits + 8 + 128);
-  return align16(act > att ? act : att);
+  const int kmax = max(max(d, H * 64), F);
+  const size_t mv = plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d) + part_bytes(M);
+  const size_t att = align16(sizeof(float) * (size_t)kAttFloats);
+  const size_t lm = align16((size_t)M * d * 4);
+  size_t r = mv > att ? mv : att;
+  return r > lm ? r : lm;
 }
 }  // namespace
 
@@ -990,6 +1275,24 @@ int persistent_slots(int M, int d, int H, int F, size_t smem_optin) {
 
 size_t persistent_smem(int M, int d, int H, int F, int nslot) {
   return 1024 + (size_t)nslot * kSlot + persist_region(M, d, H, F);
+}
+
+bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, const char** why) {
+  auto no = [&](const char* m) {
+    if (why) *why = m;
+    return false;
+  };
+  if (M != 1 && M != 2 && M != 4 && M != 8) return no("batch must be 1, 2, 4 or 8");
+  if (G < 1) return no("no CTAs");
+  const int Ns[3] = {(H + 2 * Hk) * 64, d, F};
+  for (int N : Ns)
+    if (N % 8 != 0 || (N / 8 + G - 1) / G > kMaxTiles) return no("a matrix needs more than 8 tiles of 8 rows per CTA");
+  if (d % 64 != 0 || F % 64 != 0) return no("d_model and d_ff must be multiples of 64");
+  if (d > 2 * kThreads * kPairBatch) return no("d_model above 4096");
+  if ((size_t)d * 4 > (size_t)kSlot) return no("an LM head row does not fit a ring slot");
+  if (H % Hk != 0 || H / Hk > 8) return no("more than 8 query heads per kv head");
+  if (V < 1) return no("empty vocabulary");
+  return true;
 }
 
 template <int M, int FMT>

@@ -5,8 +5,8 @@
 
 namespace ms {
 
-// One layer as the persistent kernel sees it.  w[i]: rows of matrix i (QKV, O, FC1, FC2);
-// INT4 rows are [K/2 nibble bytes | K/32 fp32 scales], fp16 rows are K halves.
+// One layer as the persistent kernel sees it.  w[i]: tile-packed copy of matrix i (QKV, O,
+// FC1, FC2): records of 8 rows x 32 columns, tile by tile (see launch_repack_tiles).
 struct PLayer {
   const float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
   const uint8_t* w[4];
@@ -36,8 +36,7 @@ struct PersistArgs {
   uint64_t* xe_s;            // residual after the FFN [B][d]
   uint64_t* u_s;             // [B][d_ff]
   unsigned epoch_base;       // epochs of this launch: epoch_base + 1 ...
-  float* part;               // attention partials [B][Hk][att_splits][hpg][66]
-  unsigned* att_counters;    // [B][Hk]
+  uint64_t* part_s;          // attention partials, stamped [B][Hk][att_splits][hpg][66]: m, l, o[64]
   int att_splits;
   float* lm_val;             // [grid][64]
   int* lm_idx;
@@ -56,6 +55,9 @@ cudaError_t init_attrs_persistent();
 // Ring slots that fit next to the kernel's other shared memory (0: the kernel does not fit).
 int persistent_slots(int M, int d, int H, int F, size_t smem_optin);
 size_t persistent_smem(int M, int d, int H, int F, int nslot);
+// Whether the model's shapes suit the kernel for M streams on G CTAs (tiles per CTA,
+// vector lengths); why gets a reason when not.
+bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, const char** why);
 int persistent_max_ctas(int M, int fmt, size_t smem);
 size_t persistent_static_smem(int M, int fmt);  // (size_t)-1 on error
 cudaError_t launch_decode_persistent(const PersistArgs& a, int M, int grid, size_t smem, cudaStream_t st);

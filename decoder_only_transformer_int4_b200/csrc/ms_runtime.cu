@@ -81,6 +81,7 @@ struct Arena {
 struct DevLayer {
   float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
   ms::WView w[4];
+  uint8_t* wt[4];  // tile-packed copies for the persistent decode kernel
 };
 
 bool shape_ok(const ms_config* c, std::string* why) {
@@ -185,7 +186,7 @@ struct ms_cache {
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
   // persistent decode kernel
   unsigned* sync3 = nullptr;             // grid barrier count, completed epoch, abort word
-  uint64_t *qkv_s = nullptr, *o_s = nullptr, *xc_s = nullptr, *xe_s = nullptr, *u_s = nullptr;
+  uint64_t *qkv_s = nullptr, *o_s = nullptr, *xc_s = nullptr, *xe_s = nullptr, *u_s = nullptr, *part_s = nullptr;
   size_t stamp_bytes = 0;                // the five stamped vectors, contiguous
   unsigned epoch_next = 0;               // first unused epoch of the stamped vectors
   int persist_grid = 0, persist_nslot = 0;
@@ -326,8 +327,7 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.u_s = c->u_s;
   a.epoch_base = c->epoch_next;
   c->epoch_next += (unsigned)need;
-  a.part = c->att_part;
-  a.att_counters = c->att_counters;
+  a.part_s = c->part_s;
   a.att_splits = c->splits;
   a.lm_val = c->lm_val;
   a.lm_idx = c->lm_idx;
@@ -441,6 +441,7 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
           w.lds = 0;
           w.h = a.take<uint16_t>((size_t)N * K);
         }
+        L.wt[i] = a.take<uint8_t>(ms::tile_packed_bytes(w));
       }
     }
     if (pass == 0) {
@@ -481,6 +482,10 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
       }
     }
   }
+  // tile-packed copies, made on the device from the rows just copied
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l)
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = ms::launch_repack_tiles(m->layers[l].w[i], m->layers[l].wt[i], 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e == cudaSuccess && c.n_layers > 0) {
     std::vector<ms::PLayer> pl(c.n_layers);
     for (int l = 0; l < c.n_layers; ++l) {
@@ -489,8 +494,7 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
       pl[l].ln1_b = L.ln1_b;
       pl[l].ln2_g = L.ln2_g;
       pl[l].ln2_b = L.ln2_b;
-      for (int i = 0; i < 4; ++i)
-        pl[l].w[i] = L.w[i].fmt == ms::kInt4 ? L.w[i].q : reinterpret_cast<const uint8_t*>(L.w[i].h);
+      for (int i = 0; i < 4; ++i) pl[l].w[i] = L.wt[i];
     }
     e = cudaMemcpy(m->d_players, pl.data(), pl.size() * sizeof(ms::PLayer), cudaMemcpyHostToDevice);
   }
@@ -534,13 +538,9 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
-    const bool mb = batch == 1 || batch == 2 || batch == 4 || batch == 8;
-    // every weight row (and LM head row) must fit one 16 KiB ring slot
-    int kmax = g.d_model > g.d_ff ? g.d_model : g.d_ff;
-    if (g.n_heads * 64 > kmax) kmax = g.n_heads * 64;
-    const size_t rowmax = g.weight_format == MS_W_FP16 ? (size_t)kmax * 2 : (size_t)kmax / 2 + kmax / 8;
-    const bool rows_fit = rowmax <= 16384 && (size_t)g.d_model * 4 <= 16384;
-    if (mb && rows_fit && coop && nsm > 0 && g.n_layers > 0 && g.n_layers <= 64) {
+    const bool shapes = nsm > 0 && ms::persistent_shapes_ok(batch, g.d_model, g.n_heads, g.n_kv_heads, g.d_ff,
+                                                            g.vocab, nsm, nullptr);
+    if (shapes && coop && g.n_layers > 0 && g.n_layers <= 64) {
       // the ring gets what the kernel's static shared memory and its other regions leave
       const int fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
       const size_t st_smem = ms::persistent_static_smem(batch, fmt);
@@ -549,7 +549,7 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
                          : 0;
       if (ns >= 4) {
         const size_t sm_bytes = ms::persistent_smem(batch, g.d_model, g.n_heads, g.d_ff, ns);
-        if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1 && (g.d_model + nsm - 1) / nsm <= 16) {
+        if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1) {
           c->persist_grid = nsm;
           c->persist_nslot = ns;
           c->persist_smem = sm_bytes;
@@ -581,12 +581,14 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
       const size_t n_o = (size_t)batch * g.n_heads * 64;
       const size_t n_x = (size_t)batch * g.d_model;
       const size_t n_u = (size_t)batch * g.d_ff;
-      c->qkv_s = a.take<uint64_t>(n_qkv + n_o + 2 * n_x + n_u);
+      const size_t n_p = (size_t)batch * g.n_kv_heads * c->splits * hpg * 66;  // attention partials
+      c->qkv_s = a.take<uint64_t>(n_qkv + n_o + 2 * n_x + n_u + n_p);
       c->o_s = c->qkv_s ? c->qkv_s + n_qkv : nullptr;
       c->xc_s = c->o_s ? c->o_s + n_o : nullptr;
       c->xe_s = c->xc_s ? c->xc_s + n_x : nullptr;
       c->u_s = c->xe_s ? c->xe_s + n_x : nullptr;
-      c->stamp_bytes = (n_qkv + n_o + 2 * n_x + n_u) * sizeof(uint64_t);
+      c->part_s = c->u_s ? c->u_s + n_u : nullptr;
+      c->stamp_bytes = (n_qkv + n_o + 2 * n_x + n_u + n_p) * sizeof(uint64_t);
     }
     c->att_counters = a.take<unsigned>((size_t)batch * g.n_kv_heads);
     c->hist = a.take<int32_t>((size_t)capacity * batch);
