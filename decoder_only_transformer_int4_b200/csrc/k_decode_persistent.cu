@@ -59,12 +59,13 @@ constexpr long long kGridSpinLimit = 1ll << 24;  // polls of the barrier count (
 constexpr int kAttSub = 64;
 constexpr int kAttMaxSplits = 128;
 constexpr int kMinPerSplit = 16;
-constexpr int kMaxTiles = 8;              // 8-row tiles of one matrix per CTA
-constexpr int kMaxOwn = 8 * kMaxTiles;    // residual rows a CTA owns
+constexpr int kTile = 16;                 // weight rows per tile (the MMA's M)
+constexpr int kMaxTiles = 4;              // tiles of one matrix per CTA
+constexpr int kMaxOwn = kTile * kMaxTiles;  // residual rows a CTA owns
 constexpr int kMaxLayers = 64;            // layer table kept in shared memory
 constexpr int kPairBatch = 8;             // element pairs a thread has in flight per round
-constexpr int kRecInt4 = 160;             // tile-packed record: 32 code words + 8 scales
-constexpr int kRecF16 = 512;              // tile-packed record: 32 x 16 bytes of halves
+constexpr int kRecInt4 = 320;             // tile-packed record: 64 code words + 16 scales
+constexpr int kRecF16 = 1024;             // tile-packed record: 32 x 32 bytes of halves
 constexpr int kUnroll = 4;                // records a warp has in flight (2 for more than 4 streams)
 
 // Attention scratch (floats): q, scores, per-head running stats, the new k and v; then either
@@ -122,18 +123,35 @@ struct RingPos {
   }
 };
 
+// One weight slice of the schedule: a contiguous run of records (or LM head rows).
+struct Slice {
+  const unsigned char* src;
+  uint32_t bytes;
+  uint32_t pad;
+};
+
 struct Smem {
   uint64_t* full;          // ring mbarriers [16]
   float* red;              // reduction slots [2][8][4]
+  unsigned* cnt;           // warps done with each slot, counted up [16]
+  unsigned* niss;          // copies issued into each slot [16]
+  int* ntab;               // slices per step
+  Slice* tab;              // the CTA's slices of one step, in consumption order
   unsigned char* ring;
   unsigned char* region;   // activation planes, staging, partial sums / attention scratch / LM head input
 };
 
-__device__ __forceinline__ Smem carve(unsigned char* base, int nslot) {
+__host__ __device__ __forceinline__ size_t tab_bytes(int cap) { return ((size_t)cap * sizeof(Slice) + 1023) & ~(size_t)1023; }
+
+__device__ __forceinline__ Smem carve(unsigned char* base, int nslot, int cap) {
   Smem s;
   s.full = reinterpret_cast<uint64_t*>(base);
   s.red = reinterpret_cast<float*>(base + 128);
-  s.ring = base + 1024;
+  s.cnt = reinterpret_cast<unsigned*>(base + 384);
+  s.niss = reinterpret_cast<unsigned*>(base + 448);
+  s.ntab = reinterpret_cast<int*>(base + 512);
+  s.tab = reinterpret_cast<Slice*>(base + 1024);
+  s.ring = base + 1024 + tab_bytes(cap);
   s.region = s.ring + (size_t)nslot * kSlot;
   return s;
 }
@@ -145,57 +163,26 @@ __host__ __device__ __forceinline__ size_t plane_bytes(int M, int kmax) {
   return align16((size_t)2 * M * (2 * kmax + 64));
 }
 __host__ __device__ __forceinline__ size_t xin_bytes(int kmax) { return align16((size_t)kmax * 4); }
-__host__ __device__ __forceinline__ size_t part_bytes(int M) { return (size_t)kMaxTiles * kWarps * M * 8 * 4; }
+__host__ __device__ __forceinline__ size_t part_bytes(int M) { return (size_t)kMaxTiles * kWarps * M * kTile * 4; }
 __host__ __device__ __forceinline__ size_t gb_bytes(int d) { return align16((size_t)d * 8); }
+
+// Bytes of the region's aliased part: the matrix phases' planes, staging and partial sums,
+// the attention scratch, or the LM head's input, whichever is largest.  The zero row follows.
+__host__ __device__ __forceinline__ size_t persist_main(int M, int d, int H, int F) {
+  const int kmax = max(max(d, H * 64), F);
+  const size_t mv = plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d) + part_bytes(M);
+  const size_t att = align16(sizeof(float) * (size_t)kAttFloats);
+  const size_t lm = align16((size_t)M * d * 4);
+  const size_t r = mv > att ? mv : att;
+  return r > lm ? r : lm;
+}
 
 struct Region {
   uint32_t* planes;
   float2* xin;    // staged input pairs (each thread reads back only the pairs it wrote)
   float4* gb;     // staged LayerNorm (gamma, gamma, beta, beta) per pair, likewise
   float* part;
-};
-
-// ---------------------------------------------------------------------------------
-// Weight schedule: the CTA's slices in consumption order (per step: per layer the records
-// of QKV, O, FC1, FC2; then the LM head rows), one ring slot each.  sched[s] and sched[5 + s]
-// bound the CTA's units of stage s (records for s < 4, LM head rows for s = 4).  Thread 0
-// keeps a cursor and issues the next slice whenever a slot comes free.
-// ---------------------------------------------------------------------------------
-struct Cursor {
-  int step = 0, l = 0, stage = 0, p = -1;
-  const PLayer* layers = nullptr;   // the layer table (a shared-memory copy)
-  const int* sched = nullptr;
-  __device__ bool next(const PersistArgs& a, const unsigned char** src, uint32_t* bytes) {
-    for (;;) {
-      if (step >= a.n_steps) return false;
-      const int ub = stage == 4 ? a.d * 4 : (a.fmt == kInt4 ? kRecInt4 : kRecF16);
-      const int per = kSlot / ub;
-      p = p < 0 ? sched[stage] : p + per;
-      if (p < sched[5 + stage]) {
-        const int n = min(per, sched[5 + stage] - p);
-        const PLayer& ly = layers[l];
-        const unsigned char* base = stage == 0   ? ly.w[0]
-                                    : stage == 1 ? ly.w[1]
-                                    : stage == 2 ? ly.w[2]
-                                    : stage == 3 ? ly.w[3]
-                                                 : reinterpret_cast<const unsigned char*>(a.lm_head);
-        *src = base + (size_t)p * ub;
-        *bytes = (uint32_t)(n * ub);
-        return true;
-      }
-      p = -1;
-      if (stage < 3) {
-        ++stage;
-      } else if (stage == 3) {
-        if (++l < a.L) stage = 0;
-        else stage = 4;
-      } else {
-        stage = 0;
-        l = 0;
-        ++step;
-      }
-    }
-  }
+  const uint32_t* zero;   // a row of zeros: the B columns of streams that do not exist
 };
 
 // ---------------------------------------------------------------------------------
@@ -445,23 +432,6 @@ __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* 
 // ---------------------------------------------------------------------------------
 // Matrix phases
 // ---------------------------------------------------------------------------------
-// Shared-memory loads by 32-bit shared address (volatile: never merged with a load of the
-// same address from before a barrier, where the ring slot or the planes held other data).
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ float2 lds_f2(uint32_t a) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-  return v;
-}
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {  // (a & b) | c
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
@@ -490,62 +460,81 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One record (tile, group g) of the warp's share: its contribution r (scaled by the group's
-// INT4 scales).  Lane (q = lane / 4, t = lane % 4) gets r[0], r[1] = rows 2t, 2t + 1 of the
-// tile for A row q, and r[2], r[3] the same for A row q + 8 (streams 4..7).
+// One record (tile, group g) of the warp's share, added into acc (use = false: read but
+// not added).  A = the 16 weight rows (INT4 codes turned into exact fp16 integers, two
+// halves per mask and fp16 op), B = the activation planes (column 2m + j: stream m, hi or
+// lo).  Lane (r = lane / 4, t = lane % 4) holds acc[0], acc[1] = rows r of columns 2t, 2t + 1
+// (stream t, hi and lo), acc[2], acc[3] = row r + 8 of the same; acc[4..7] the same for
+// streams 4 + t.  The group's INT4 scales multiply each record's sums.
 template <int M, int FMT>
-__device__ __forceinline__ void mv_record(uint32_t rec, uint32_t planes, int pw, int g, float (&r)[4]) {
-  // Branch-free, so that the records a warp has in flight overlap: lanes whose A row does
-  // not exist (r >= 2M) read row 0 and zero it.
-  const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-  const bool alive = gid < 2 * M;
-  uint4 alo = lds_u4(planes + 4u * ((alive ? gid : 0) * pw + g * 16 + tq * 4));
-  if (M < 4) {
-    alo.x = alive ? alo.x : 0u;
-    alo.y = alive ? alo.y : 0u;
-    alo.z = alive ? alo.z : 0u;
-    alo.w = alive ? alo.w : 0u;
-  }
-  uint4 ahi = make_uint4(0u, 0u, 0u, 0u);
-  if (M > 4) ahi = lds_u4(planes + 4u * ((gid + 8) * pw + g * 16 + tq * 4));   // 2M = 16 rows
-  r[0] = r[1] = r[2] = r[3] = 0.f;
+__device__ __forceinline__ void mv_record(const unsigned char* rec, const uint32_t* blo, const uint32_t* bhi, int g,
+                                          bool use, float (&acc)[8]) {
+  const int lane = threadIdx.x & 31, gid = lane >> 2;
+  const uint4 b = *reinterpret_cast<const uint4*>(blo + g * 16);
+  uint4 b2 = make_uint4(0u, 0u, 0u, 0u);
+  if (M > 4) b2 = *reinterpret_cast<const uint4*>(bhi + g * 16);
+  uint32_t a[8];
+  float s0, s1;
   if (FMT == kInt4) {
-    const uint32_t w = lds_u32(rec + 4u * lane);
-    const float2 s = lds_f2(rec + 128u + 8u * tq);
-    mma16816(r, alo.x, ahi.x, alo.y, ahi.y, q_pair_a(w), q_pair_b(w));
-    mma16816(r, alo.z, ahi.z, alo.w, ahi.w, q_pair_a(w >> 8), q_pair_b(w >> 8));
-    r[0] *= s.x;
-    r[1] *= s.y;
-    r[2] *= s.x;
-    r[3] *= s.y;
+    const uint2 w = reinterpret_cast<const uint2*>(rec)[lane];
+    const float2 s = reinterpret_cast<const float2*>(rec + 256)[gid];
+    s0 = use ? s.x : 0.f;
+    s1 = use ? s.y : 0.f;
+    const uint32_t x8 = w.x >> 8, y8 = w.y >> 8;
+    a[0] = q_pair_a(w.x);
+    a[1] = q_pair_a(w.y);
+    a[2] = q_pair_b(w.x);
+    a[3] = q_pair_b(w.y);
+    a[4] = q_pair_a(x8);
+    a[5] = q_pair_a(y8);
+    a[6] = q_pair_b(x8);
+    a[7] = q_pair_b(y8);
   } else {
-    const uint4 b = lds_u4(rec + 16u * lane);
-    mma16816(r, alo.x, ahi.x, alo.y, ahi.y, b.x, b.y);
-    mma16816(r, alo.z, ahi.z, alo.w, ahi.w, b.z, b.w);
+    const uint4 x0 = reinterpret_cast<const uint4*>(rec)[2 * lane];
+    const uint4 x1 = reinterpret_cast<const uint4*>(rec)[2 * lane + 1];
+    s0 = s1 = use ? 1.f : 0.f;
+    a[0] = x0.x;
+    a[1] = x0.y;
+    a[2] = x0.z;
+    a[3] = x0.w;
+    a[4] = x1.x;
+    a[5] = x1.y;
+    a[6] = x1.z;
+    a[7] = x1.w;
+  }
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  mma16816(d, a[0], a[1], a[2], a[3], b.x, b.y);
+  mma16816(d, a[4], a[5], a[6], a[7], b.z, b.w);
+  acc[0] = fmaf(s0, d[0], acc[0]);
+  acc[1] = fmaf(s0, d[1], acc[1]);
+  acc[2] = fmaf(s1, d[2], acc[2]);
+  acc[3] = fmaf(s1, d[3], acc[3]);
+  if (M > 4) {
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    mma16816(e, a[0], a[1], a[2], a[3], b2.x, b2.y);
+    mma16816(e, a[4], a[5], a[6], a[7], b2.z, b2.w);
+    acc[4] = fmaf(s0, e[0], acc[4]);
+    acc[5] = fmaf(s0, e[1], acc[5]);
+    acc[6] = fmaf(s1, e[2], acc[6]);
+    acc[7] = fmaf(s1, e[3], acc[7]);
   }
 }
 
-// Adds a warp's sums for tile tl into its partial slots: hi and lo rows (lanes 4 apart)
-// first, then stream m = r / 2 (and m + 4) from the lanes with even r.
+// Adds a warp's sums for tile tl (hi + lo) into its partial slots [tile][warp][m][16].
 template <int M>
-__device__ __forceinline__ void flush_tile(float (&acc)[4], float* part, int tl) {
+__device__ __forceinline__ void flush_tile(float (&acc)[8], float* part, int tl) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gid = lane >> 2, tq = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 4);
-  if ((gid & 1) == 0) {
-    const int m = gid >> 1;
-    float* pp = part + (size_t)(tl * kWarps + warp) * M * 8;
-    if (m < M) {
-      pp[m * 8 + 2 * tq] += acc[0];
-      pp[m * 8 + 2 * tq + 1] += acc[1];
-    }
-    if (M > 4 && m + 4 < M) {
-      pp[(m + 4) * 8 + 2 * tq] += acc[2];
-      pp[(m + 4) * 8 + 2 * tq + 1] += acc[3];
-    }
+  float* pp = part + (size_t)(tl * kWarps + warp) * M * kTile;
+  if (tq < M) {
+    pp[tq * kTile + gid] += acc[0] + acc[1];
+    pp[tq * kTile + gid + 8] += acc[2] + acc[3];
+  }
+  if (M > 4 && tq + 4 < M) {
+    pp[(tq + 4) * kTile + gid] += acc[4] + acc[5];
+    pp[(tq + 4) * kTile + gid + 8] += acc[6] + acc[7];
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 }
 
 // Where a matrix phase's outputs go.  mode: 0 store, 1 residual (x += value, kept in the
@@ -559,131 +548,128 @@ struct OutSpec {
   int xr0;
 };
 
-// Consumer side of the ring: wait for a slot's bytes, hand it back when done.  Every
-// consumer thread waits (bounded) on its own; release() ORs the outcome over all of them
-// so that they either all carry on or all leave together (no thread is left waiting at
-// a named barrier for one that gave up).
-struct Consumer {
+__device__ __forceinline__ unsigned atom_add_acq_rel_shared(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+  return old;
+}
+
+// The weight ring.  Every thread consumes the slices in order (slice i in slot i % nslot);
+// a warp that is done with a slice counts itself out of the slot (acquire-release), and the
+// last of the eight warps refills the slot with slice i + nslot at once — no CTA barrier per
+// slot.  It refills only if its own wait saw the slice's bytes arrive (so no copy into the
+// slot is still in flight).  Waits are bounded; a thread whose wait ran out raises the
+// abort word and the CTA leaves at the end of the phase.
+struct Ring {
   const PersistArgs* a;
   Smem sm;
-  RingPos rp;           // next slot to consume
+  long long i = 0;       // next slice to consume
+  long long total = 0;   // slices of the launch
+  int E = 1;             // slices per step
   bool got = false;
-  // thread 0 only: the schedule cursor and the number of slices issued
-  Cursor cur;
-  long long issued = 0, consumed = 0;
-  __device__ void issue_next() {
-    const unsigned char* src;
-    uint32_t bytes;
-    if (!cur.next(*a, &src, &bytes)) return;
-    const int slot = (int)(issued % a->nslot);
-    mbar_expect_tx(&sm.full[slot], bytes);
-    bulk_g2s(sm.ring + (size_t)slot * kSlot, src, bytes, &sm.full[slot]);
-    ++issued;
+  __device__ void issue(long long j) {
+    if (j >= total) return;
+    const Slice sl = sm.tab[j % E];
+    const int slot = (int)(j % a->nslot);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(&sm.full[slot], sl.bytes);
+    bulk_g2s(sm.ring + (size_t)slot * kSlot, sl.src, sl.bytes, &sm.full[slot]);
+    sm.niss[slot] += 1u;
   }
   __device__ void start() {
     if (threadIdx.x == 0)
-      for (int i = 0; i < a->nslot; ++i) issue_next();
+      for (int k = 0; k < a->nslot; ++k) issue(k);
   }
-  // The slot's address (valid only if got: check it before reading).
+  // The slot of slice i (its bytes valid only if got).
   __device__ const unsigned char* acquire() {
-    got = mbar_wait(&sm.full[rp.slot], rp.phase, a->status);
+    const int slot = (int)(i % a->nslot);
+    got = mbar_wait(&sm.full[slot], (uint32_t)((i / a->nslot) & 1), a->status);
     if (!got) atomicExch(a->abort, 1u);
-    return sm.ring + (size_t)rp.slot * kSlot;
+    return sm.ring + (size_t)slot * kSlot;
   }
-  // All consumers are done with the slot: refill it with the slice nslot places ahead.
-  __device__ bool release() {
-    const bool failed = consumer_bar_or(!got);
-    if (failed) return false;
-    ++consumed;
-    // The named barrier above has every consumer's reads of the slot complete (their values
-    // are in registers) before thread 0 hands the slot to the next bulk copy.
-    if (threadIdx.x == 0) issue_next();
-    rp.next(a->nslot);
-    return true;
+  __device__ void release() {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+      const int slot = (int)(i % a->nslot);
+      const unsigned old = atom_add_acq_rel_shared(&sm.cnt[slot], 1u);
+      if (old % kWarps == kWarps - 1 && got) issue(i + a->nslot);
+    }
+    __syncwarp();
+    ++i;
   }
-  // Before leaving early: wait (bounded) for the copies still in flight.
+  // Before leaving early: wait (bounded) for the last copy issued into each slot.
   __device__ void drain() {
     if (threadIdx.x != 0) return;
-    RingPos q = rp;
-    for (long long i = consumed; i < issued; ++i) {
+    for (int k = 0; k < a->nslot; ++k) {
+      const unsigned n = sm.niss[k];
+      if (n == 0) continue;
       for (long long it = 0; it < kSpinLimit; ++it)
-        if (mbar_try_wait(&sm.full[q.slot], q.phase)) break;
-      q.next(a->nslot);
+        if (mbar_try_wait(&sm.full[k], (n - 1u) & 1u)) break;
     }
   }
 };
 
 // One matrix phase over the CTA's records [rbeg, rend) (whole tiles, K/32 records each),
-// slot by slot from the ring; the A planes hold the phase's input.  The warps split each
-// slot's records into eight contiguous runs; a run's sums go to the warp's partial slots at
-// each tile change; the CTA then adds the eight warps' partials in a fixed order, scales by
-// the input's 2^-e and applies the output mode.
+// slice by slice from the ring; the A planes hold the phase's input.  Each warp takes a
+// contiguous run of each slice's records, tile segment by tile segment (kUnroll records in
+// flight, branch-free); a segment's sums go to the warp's partial slots; the CTA then adds
+// the eight warps' partials in a fixed order, scales by the input's 2^-e and applies the
+// output mode.
 template <int M, int FMT>
-__device__ __forceinline__ bool mv_phase(Consumer& cs, const Region& rg, int K, int rbeg, int rend, const OutSpec& e,
+__device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, int K, int rbeg, int rend, const OutSpec& e,
                                          const float* inv_s) {
   constexpr int RB = FMT == kInt4 ? kRecInt4 : kRecF16;
   constexpr int PER = kSlot / RB;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int U = M > 4 ? kUnroll / 2 : kUnroll;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gid = lane >> 2, tq = lane & 3;
   const int KG = K >> 5;
   const int t0 = rbeg / KG, nt = (rend - rbeg) / KG;
   const int pw = (K >> 1) + 16;
-  const uint32_t planes_s = smem_u32(rg.planes);
-  for (int i = lane; i < nt * M * 8; i += 32) {
-    const int tl = i / (M * 8);
-    rg.part[(size_t)(tl * kWarps + warp) * M * 8 + (i - tl * M * 8)] = 0.f;
+  // this lane's B rows: plane row gid (the zero row past the streams) and, for 8 streams, gid + 8
+  const uint32_t* blo = (gid < 2 * M ? rg.planes + gid * pw : rg.zero) + tq * 4;
+  const uint32_t* bhi = rg.planes + (M > 4 ? (gid + 8) * pw : 0) + tq * 4;
+  for (int i = lane; i < nt * M * kTile; i += 32) {
+    const int tl = i / (M * kTile);
+    rg.part[(size_t)(tl * kWarps + warp) * M * kTile + (i - tl * M * kTile)] = 0.f;
   }
   __syncwarp();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int cur = -1;
+  bool ok = true;
   for (int p = rbeg; p < rend; p += PER) {
     const int n = min(PER, rend - p);
-    const uint32_t buf_s = smem_u32(cs.acquire());
-    if (cs.got) {
+    const unsigned char* buf = ring.acquire();
+    ok = ok && ring.got;
+    if (ring.got) {
       const int c0 = (n * warp) >> 3, c1 = (n * (warp + 1)) >> 3;
       const int r0 = p + c0 - rbeg;
       int tl = r0 / KG, g = r0 - tl * KG;
-      // U records at a time: their loads, conversions and MMAs are independent, so
-      // their latencies overlap; the sums then go into the accumulators in order.
-      constexpr int U = M > 4 ? kUnroll / 2 : kUnroll;
-      for (int i = c0; i < c1; i += U) {
-        float rr[U][4];
-        int gj = g;
+      int i = c0;
+      while (i < c1) {
+        const int s1 = min(c1, i + (KG - g));   // the run's records of tile tl
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (; i < s1; i += U) {
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-          // past the run's end: read the run's last record (in bounds); not accumulated
-          const int ij = min(i + j, c1 - 1);
-          mv_record<M, FMT>(buf_s + (uint32_t)(ij * RB), planes_s, pw, gj, rr[j]);
-          gj = gj + 1 == KG ? 0 : gj + 1;
-        }
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-          if (i + j < c1) {
-            if (tl != cur) {
-              if (cur >= 0) flush_tile<M>(acc, rg.part, cur);
-              cur = tl;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] += rr[j][k];
-            if (++g == KG) {
-              g = 0;
-              ++tl;
-            }
+          for (int j = 0; j < U; ++j) {
+            const int ij = min(i + j, s1 - 1);  // past the run's end: re-read its last record, not added
+            mv_record<M, FMT>(buf + (size_t)ij * RB, blo, bhi, g + (ij - i), i + j < s1, acc);
           }
+          g += U;
         }
+        flush_tile<M>(acc, rg.part, tl);
+        ++tl;
+        g = 0;
       }
     }
-    if (!cs.release()) return false;
+    ring.release();
   }
-  if (cur >= 0) flush_tile<M>(acc, rg.part, cur);
-  consumer_bar();
-  for (int o = threadIdx.x; o < nt * 8 * M; o += kThreads) {
-    const int tl = o / (8 * M), rem = o - tl * 8 * M, m = rem >> 3, cc = rem & 7;
-    const float* pp = rg.part + (size_t)tl * kWarps * M * 8 + m * 8 + cc;
+  if (consumer_bar_or(!ok)) return false;
+  for (int o = threadIdx.x; o < nt * kTile * M; o += kThreads) {
+    const int tl = o / (kTile * M), rem = o - tl * kTile * M, m = rem / kTile, rr = rem - m * kTile;
+    const float* pp = rg.part + (size_t)tl * kWarps * M * kTile + m * kTile + rr;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += pp[w * M * 8];
+    for (int w = 0; w < kWarps; ++w) v += pp[w * M * kTile];
     v *= inv_s[m];
-    const int nn = (t0 + tl) * 8 + cc;
+    const int nn = (t0 + tl) * kTile + rr;
     if (e.mode == 1) {
       float* xo = e.xown + m * kMaxOwn + (nn - e.xr0);
       v += *xo;
@@ -990,21 +976,30 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 }  // namespace
 
 template <int M, int FMT>
-__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers,
+__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, const Smem& sm, const PLayer* layers,
                                              const int* sched);
+
+// The CTA's units of each stage: sched[s] .. sched[5 + s] (records of matrix s < 4, LM head
+// rows for s = 4), whole tiles, contiguous and balanced over the CTAs.
+__device__ __forceinline__ int mat_KG(const PersistArgs& a, int s) { return mat_K(a, s) / 32; }
 
 template <int M, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) decode_persistent_kernel(const __grid_constant__ PersistArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  const Smem sm = carve(smem, a.nslot);
+  const Smem sm = carve(smem, a.nslot, a.sched_cap);
   __shared__ PLayer layers_s[kMaxLayers];
   __shared__ int sched_s[10];
+  const int kmax = max(max(a.d, a.H * 64), a.F);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < a.nslot; ++i) mbar_init(&sm.full[i], 1);
+    for (int i = 0; i < a.nslot; ++i) {
+      mbar_init(&sm.full[i], 1);
+      sm.cnt[i] = 0u;
+      sm.niss[i] = 0u;
+    }
     mbar_fence_init();
     const int c = blockIdx.x, G = gridDim.x;
     for (int s = 0; s < 4; ++s) {
-      const int nt = mat_N(a, s) / 8, KG = mat_K(a, s) / 32;
+      const int nt = mat_N(a, s) / kTile, KG = mat_KG(a, s);
       sched_s[s] = (nt * c / G) * KG;
       sched_s[5 + s] = (nt * (c + 1) / G) * KG;
     }
@@ -1013,18 +1008,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent_kernel(const __
   }
   for (int i = threadIdx.x; i < a.L * (int)(sizeof(PLayer) / 8); i += kThreads)
     reinterpret_cast<uint64_t*>(layers_s)[i] = reinterpret_cast<const uint64_t*>(a.layers)[i];
+  // the zero row (B columns of streams that do not exist); never written again
+  {
+    uint32_t* z = reinterpret_cast<uint32_t*>(sm.region + persist_main(M, a.d, a.H, a.F));
+    for (int i = threadIdx.x; i < kmax / 2 + 16; i += kThreads) z[i] = 0u;
+  }
   __syncthreads();
-  Consumer cs;
-  cs.cur.layers = layers_s;
-  cs.cur.sched = sched_s;
-  cs.a = &a;
-  cs.sm = sm;
-  cs.start();
-  if (!decode_steps<M, FMT>(a, cs, sm, layers_s, sched_s)) cs.drain();
+  // the slice table of one step (the same every step)
+  if (threadIdx.x == 0) {
+    const int rb = a.fmt == kInt4 ? kRecInt4 : kRecF16;
+    const int per = kSlot / rb, rpp = kSlot / (a.d * 4);
+    int E = 0;
+    bool fits = true;
+    for (int l = 0; l < a.L; ++l)
+      for (int s = 0; s < 4; ++s)
+        for (int p = sched_s[s]; p < sched_s[5 + s]; p += per) {
+          if (E < a.sched_cap)
+            sm.tab[E] = Slice{layers_s[l].w[s] + (size_t)p * rb, (uint32_t)(min(per, sched_s[5 + s] - p) * rb), 0u};
+          else fits = false;
+          ++E;
+        }
+    for (int p = sched_s[4]; p < sched_s[9]; p += rpp) {
+      if (E < a.sched_cap)
+        sm.tab[E] = Slice{reinterpret_cast<const unsigned char*>(a.lm_head) + (size_t)p * a.d * 4,
+                          (uint32_t)(min(rpp, sched_s[9] - p) * a.d * 4), 0u};
+      else fits = false;
+      ++E;
+    }
+    if (!fits || E == 0) {
+      flag_error(a.status, kErrShapeBit);
+      atomicExch(a.abort, 1u);
+      E = 0;
+    }
+    *sm.ntab = E;
+  }
+  __syncthreads();
+  Ring ring;
+  ring.a = &a;
+  ring.sm = sm;
+  ring.E = *sm.ntab;
+  if (ring.E == 0) return;
+  ring.total = (long long)a.n_steps * ring.E;
+  ring.start();
+  if (!decode_steps<M, FMT>(a, ring, sm, layers_s, sched_s)) ring.drain();
 }
 
 template <int M, int FMT>
-__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs, const Smem& sm, const PLayer* layers,
+__device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, const Smem& sm, const PLayer* layers,
                                              const int* sched) {
   __shared__ int ok_s;
   __shared__ unsigned ticket_s;
@@ -1044,13 +1074,14 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
   rg.xin = reinterpret_cast<float2*>(sm.region + plane_bytes(M, kmax));
   rg.gb = reinterpret_cast<float4*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax));
   rg.part = reinterpret_cast<float*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d));
+  rg.zero = reinterpret_cast<const uint32_t*>(sm.region + persist_main(M, d, H, F));
   float* scratch = reinterpret_cast<float*>(sm.region);
   Red red{sm.red, 0};
   unsigned epoch = 0;
   const int len0 = *a.dlen;
   // residual rows owned: the O and FC2 phases both have d rows and the same tiles
-  const int xr0 = sched[1] / (H * 2) * 8;
-  const int xr1 = sched[6] / (H * 2) * 8;
+  const int xr0 = sched[1] / (H * 2) * kTile;
+  const int xr1 = sched[6] / (H * 2) * kTile;
   const int units = B * Hk;
   int S = G / units;
   if (S < 1) S = 1;
@@ -1129,7 +1160,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
         e.ep = epA + ph;
         e.xown = xown;
         e.xr0 = xr0;
-        if (!mv_phase<M, FMT>(cs, rg, K, sched[mi], sched[5 + mi], e, inv_s)) return false;
+        if (!mv_phase<M, FMT>(ring, rg, K, sched[mi], sched[5 + mi], e, inv_s)) return false;
       }
     }
     // ---- LM head + argmax ------------------------------------------------------------
@@ -1152,12 +1183,14 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
       best[m] = -FLT_MAX;
       bi[m] = INT_MAX;
     }
+    bool lm_ok = true;
     {
       const int rb = d * 4, rpp = kSlot / rb;
       for (int p = sched[4]; p < sched[9]; p += rpp) {
         const int rows = min(rpp, sched[9] - p);
-        const unsigned char* buf = cs.acquire();
-        for (int r = warp; cs.got && r < rows; r += kWarps) {
+        const unsigned char* buf = ring.acquire();
+        lm_ok = lm_ok && ring.got;
+        for (int r = warp; ring.got && r < rows; r += kWarps) {
           const float4* w4 = reinterpret_cast<const float4*>(buf + (size_t)r * rb);
           float acc[M];
 #pragma unroll
@@ -1184,7 +1217,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
             }
           }
         }
-        if (!cs.release()) return false;
+        ring.release();
       }
     }
     if (lane == 0)
@@ -1192,7 +1225,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
         bval[warp][m] = best[m];
         bidx[warp][m] = bi[m];
       }
-    consumer_bar();
+    if (consumer_bar_or(!lm_ok)) return false;
     if (tid < M) {
       float bv = -FLT_MAX;
       int bx = INT_MAX;
@@ -1254,27 +1287,37 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Consumer& cs,
 }
 
 // ---------------------------------------------------------------------------------
-namespace {
-size_t persist_region(int M, int d, int H, int F) {
-  const int kmax = max(max(d, H * 64), F);
-  const size_t mv = plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d) + part_bytes(M);
-  const size_t att = align16(sizeof(float) * (size_t)kAttFloats);
-  const size_t lm = align16((size_t)M * d * 4);
-  size_t r = mv > att ? mv : att;
-  return r > lm ? r : lm;
+int persistent_sched_cap(int L, int d, int H, int Hk, int F, int V, int G, int fmt) {
+  const int rb = fmt == kInt4 ? kRecInt4 : kRecF16;
+  const int per = kSlot / rb;
+  const int Ns[4] = {(H + 2 * Hk) * 64, d, F, d};
+  const int Ks[4] = {d, H * 64, d, F};
+  long long per_layer = 0;
+  for (int s = 0; s < 4; ++s) {
+    const long long tmax = (Ns[s] / kTile + G - 1) / G;
+    per_layer += (tmax * (Ks[s] / 32) + per - 1) / per;
+  }
+  const long long rows = (V + G - 1) / G, rpp = kSlot / (d * 4);
+  const long long cap = (long long)L * per_layer + (rows + rpp - 1) / rpp;
+  return cap > (1 << 20) ? (1 << 20) : (int)cap;
 }
-}  // namespace
 
-int persistent_slots(int M, int d, int H, int F, size_t smem_optin) {
-  const size_t region = persist_region(M, d, H, F);
-  if (smem_optin < 1024 + region + 4 * (size_t)kSlot) return 0;
-  size_t n = (smem_optin - 1024 - region) / kSlot;
+static size_t region_bytes(int M, int d, int H, int F) {
+  const int kmax = max(max(d, H * 64), F);
+  return persist_main(M, d, H, F) + align16((size_t)kmax * 2 + 64);   // + the zero row
+}
+
+int persistent_slots(int M, int L, int d, int H, int Hk, int F, int V, int G, int fmt, size_t smem_optin) {
+  const size_t fixed = 1024 + tab_bytes(persistent_sched_cap(L, d, H, Hk, F, V, G, fmt)) + region_bytes(M, d, H, F);
+  if (smem_optin < fixed + 4 * (size_t)kSlot) return 0;
+  size_t n = (smem_optin - fixed) / kSlot;
   if (n > 16) n = 16;
   return (int)n;
 }
 
-size_t persistent_smem(int M, int d, int H, int F, int nslot) {
-  return 1024 + (size_t)nslot * kSlot + persist_region(M, d, H, F);
+size_t persistent_smem(int M, int L, int d, int H, int Hk, int F, int V, int G, int fmt, int nslot) {
+  return 1024 + tab_bytes(persistent_sched_cap(L, d, H, Hk, F, V, G, fmt)) + (size_t)nslot * kSlot +
+         region_bytes(M, d, H, F);
 }
 
 bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, const char** why) {
@@ -1286,7 +1329,8 @@ bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, cons
   if (G < 1) return no("no CTAs");
   const int Ns[3] = {(H + 2 * Hk) * 64, d, F};
   for (int N : Ns)
-    if (N % 8 != 0 || (N / 8 + G - 1) / G > kMaxTiles) return no("a matrix needs more than 8 tiles of 8 rows per CTA");
+    if (N % kTile != 0 || (N / kTile + G - 1) / G > kMaxTiles)
+      return no("a matrix needs more than 4 tiles of 16 rows per CTA");
   if (d % 64 != 0 || F % 64 != 0) return no("d_model and d_ff must be multiples of 64");
   if (d > 2 * kThreads * kPairBatch) return no("d_model above 4096");
   if ((size_t)d * 4 > (size_t)kSlot) return no("an LM head row does not fit a ring slot");

@@ -241,30 +241,30 @@ cudaError_t launch_rope_append(const Launch& L, const float* qkv, int B, int n, 
 
 // ---------------------------------------------------------------------------------
 // Tile-packed copies of the backbone matrices for the persistent decode kernel, whose
-// matrix-vector products run on warp-level tensor-core MMAs (m16n8k16, weights as the B
-// operand).  A record covers one tile of 8 rows and one group of 32 columns (k = 32g ..
-// 32g + 31); records are stored tile by tile, groups in order.  Lane l = 4 * r + t of a
-// warp needs, of row r of the tile, the columns 2t + {0, 1, 8, 9, 16, 17, 24, 25}:
-//   INT4 record (160 bytes): 32 words, word l holding those eight codes (u = q + 8) as
-//     nibbles, columns 2t, 2t+8, 2t+16, 2t+24 in bits 0-3, 4-7, 8-11, 12-15 and columns
-//     2t+1, 2t+9, 2t+17, 2t+25 in bits 16-19, 20-23, 24-27, 28-31 (so that one mask with
-//     0x000F000F or 0x00F000F0 yields a pair of them as two halves); then the 8 rows'
-//     fp32 scales of the group.
-//   FP16 record (512 bytes): 32 chunks of 16 bytes, chunk l holding those eight halves as
-//     pairs (2t, 2t+1), (2t+8, 2t+9), (2t+16, 2t+17), (2t+24, 2t+25).
+// matrix-vector products run on warp-level tensor-core MMAs (m16n8k16 with the weights as
+// the A operand).  A record covers one tile of 16 rows and one group of 32 columns (k =
+// 32g .. 32g + 31); records are stored tile by tile, groups in order.  Lane l = 4 r + t of a
+// warp needs, of rows r and r + 8 of the tile, the columns 2t + {0, 1, 8, 9, 16, 17, 24, 25}:
+//   INT4 record (320 bytes): 64 words, words 2l and 2l + 1 holding those eight codes
+//     (u = q + 8) of rows r and r + 8 as nibbles — columns 2t, 2t+8, 2t+16, 2t+24 in bits
+//     0-3, 4-7, 8-11, 12-15 and 2t+1, 2t+9, 2t+17, 2t+25 in bits 16-19, 20-23, 24-27, 28-31,
+//     so that one mask with 0x000F000F or 0x00F000F0 yields a pair of them as two halves;
+//     then the group's fp32 scales as pairs (row r, row r + 8), r = 0..7.
+//   FP16 record (1024 bytes): 32 chunks of 32 bytes, chunk l holding the pairs (r, 2t),
+//     (r + 8, 2t), (r, 2t + 8), (r + 8, 2t + 8), then the same at columns + 16.
 // ---------------------------------------------------------------------------------
 __global__ void repack_int4_tiles_kernel(const uint8_t* __restrict__ rows, int ldq, int K, long long records,
                                          uint32_t* __restrict__ out) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= records * 40) return;
-  const long long rec = i / 40;
-  const int l = (int)(i - rec * 40);
+  if (i >= records * 80) return;
+  const long long rec = i / 80;
+  const int w = (int)(i - rec * 80);
   const int KG = K / 32;
   const long long t = rec / KG;
   const int g = (int)(rec - t * KG);
-  if (l < 32) {
-    const int r = l >> 2, tq = l & 3;
-    const uint8_t* row = rows + (size_t)(t * 8 + r) * ldq;
+  if (w < 64) {
+    const int l = w >> 1, r = (l >> 2) + 8 * (w & 1), tq = l & 3;
+    const uint8_t* row = rows + (size_t)(t * 16 + r) * ldq;
     auto nib = [&](int k) -> uint32_t {
       const int kk = g * 32 + k;
       return (row[kk >> 1] >> (4 * (kk & 1))) & 15u;
@@ -273,8 +273,8 @@ __global__ void repack_int4_tiles_kernel(const uint8_t* __restrict__ rows, int l
     out[i] = nib(c) | nib(c + 8) << 4 | nib(c + 16) << 8 | nib(c + 24) << 12 | nib(c + 1) << 16 | nib(c + 9) << 20 |
              nib(c + 17) << 24 | nib(c + 25) << 28;
   } else {
-    const int r = l - 32;
-    const float* sc = reinterpret_cast<const float*>(rows + (size_t)(t * 8 + r) * ldq + K / 2);
+    const int r = ((w - 64) >> 1) + 8 * ((w - 64) & 1);
+    const float* sc = reinterpret_cast<const float*>(rows + (size_t)(t * 16 + r) * ldq + K / 2);
     out[i] = __float_as_uint(sc[g]);
   }
 }
@@ -282,28 +282,28 @@ __global__ void repack_int4_tiles_kernel(const uint8_t* __restrict__ rows, int l
 __global__ void repack_f16_tiles_kernel(const uint16_t* __restrict__ w, int K, long long records,
                                         uint32_t* __restrict__ out) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= records * 128) return;
-  const long long rec = i / 128;
-  const int j = (int)(i - rec * 128);
-  const int l = j >> 2, word = j & 3;
+  if (i >= records * 256) return;
+  const long long rec = i / 256;
+  const int j = (int)(i - rec * 256);
+  const int l = j >> 3, reg = j & 3, step = (j >> 2) & 1;
   const int KG = K / 32;
   const long long t = rec / KG;
   const int g = (int)(rec - t * KG);
-  const int r = l >> 2, tq = l & 3;
-  const uint16_t* row = w + (size_t)(t * 8 + r) * K + g * 32 + 2 * tq + 8 * word;
+  const int r = (l >> 2) + ((reg & 1) ? 8 : 0), tq = l & 3;
+  const uint16_t* row = w + (size_t)(t * 16 + r) * K + g * 32 + 2 * tq + ((reg & 2) ? 8 : 0) + 16 * step;
   out[i] = (uint32_t)row[0] | (uint32_t)row[1] << 16;
 }
 
 cudaError_t launch_repack_tiles(const WView& w, void* out, cudaStream_t s) {
-  if (w.N % 8 != 0 || w.K % 32 != 0) return cudaErrorInvalidValue;
-  const long long records = (long long)(w.N / 8) * (w.K / 32);
+  if (w.N % 16 != 0 || w.K % 32 != 0) return cudaErrorInvalidValue;
+  const long long records = (long long)(w.N / 16) * (w.K / 32);
   if (w.fmt == kInt4) {
     if (!w.interleaved()) return cudaErrorInvalidValue;
-    const long long n = records * 40;
+    const long long n = records * 80;
     repack_int4_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.q, w.ldq, w.K, records,
                                                                          static_cast<uint32_t*>(out));
   } else {
-    const long long n = records * 128;
+    const long long n = records * 256;
     repack_f16_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.h, w.K, records,
                                                                         static_cast<uint32_t*>(out));
   }
@@ -311,8 +311,8 @@ cudaError_t launch_repack_tiles(const WView& w, void* out, cudaStream_t s) {
 }
 
 size_t tile_packed_bytes(const WView& w) {
-  const size_t records = (size_t)(w.N / 8) * (w.K / 32);
-  return records * (w.fmt == kInt4 ? 160 : 512);
+  const size_t records = (size_t)(w.N / 16) * (w.K / 32);
+  return records * (w.fmt == kInt4 ? 320 : 1024);
 }
 
 }  // namespace ms

@@ -107,8 +107,8 @@ cudaError_t launch_lm_head(const Launch& L, const float* x, int ldx, int M, int 
                            int len_add, const LmHeadWork& w);
 int lm_head_grid(int V);
 
-// Tile-packed copy of a backbone matrix (records of 8 rows x 32 columns, laid out for the
-// persistent decode kernel's warp MMAs); N % 8 == 0, K % 32 == 0, INT4 rows interleaved.
+// Tile-packed copy of a backbone matrix (records of 16 rows x 32 columns, laid out for the
+// persistent decode kernel's warp MMAs); N % 16 == 0, K % 32 == 0, INT4 rows interleaved.
 cudaError_t launch_repack_tiles(const WView& w, void* out, cudaStream_t s);
 size_t tile_packed_bytes(const WView& w);
 

@@ -6,7 +6,7 @@
 namespace ms {
 
 // One layer as the persistent kernel sees it.  w[i]: tile-packed copy of matrix i (QKV, O,
-// FC1, FC2): records of 8 rows x 32 columns, tile by tile (see launch_repack_tiles).
+// FC1, FC2): records of 16 rows x 32 columns, tile by tile (see launch_repack_tiles).
 struct PLayer {
   const float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
   const uint8_t* w[4];
@@ -49,12 +49,15 @@ struct PersistArgs {
   int32_t* argmax_out;       // [B] last step's argmax, or null
   int n_steps;
   int nslot;
+  int sched_cap;             // capacity of the per-CTA slice table (entries)
 };
 
 cudaError_t init_attrs_persistent();
 // Ring slots that fit next to the kernel's other shared memory (0: the kernel does not fit).
-int persistent_slots(int M, int d, int H, int F, size_t smem_optin);
-size_t persistent_smem(int M, int d, int H, int F, int nslot);
+int persistent_slots(int M, int L, int d, int H, int Hk, int F, int V, int G, int fmt, size_t smem_optin);
+size_t persistent_smem(int M, int L, int d, int H, int Hk, int F, int V, int G, int fmt, int nslot);
+// Upper bound on a CTA's weight slices per decode step (the slice table's entries).
+int persistent_sched_cap(int L, int d, int H, int Hk, int F, int V, int G, int fmt);
 // Whether the model's shapes suit the kernel for M streams on G CTAs (tiles per CTA,
 // vector lengths); why gets a reason when not.
 bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, const char** why);

@@ -191,6 +191,7 @@ struct ms_cache {
   unsigned epoch_next = 0;               // first unused epoch of the stamped vectors
   int persist_grid = 0, persist_nslot = 0;
   size_t persist_smem = 0;
+  int persist_sched_cap = 0;
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
 };
@@ -340,6 +341,7 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.argmax_out = argmax;
   a.n_steps = n_steps;
   a.nslot = c->persist_nslot;
+  a.sched_cap = c->persist_sched_cap;
   return ms::launch_decode_persistent(a, c->B, c->persist_grid, c->persist_smem, st);
 }
 
@@ -545,14 +547,18 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
       const int fmt = g.weight_format == MS_W_FP16 ? ms::kFp16 : ms::kInt4;
       const size_t st_smem = ms::persistent_static_smem(batch, fmt);
       const int ns = st_smem < (size_t)optin
-                         ? ms::persistent_slots(batch, g.d_model, g.n_heads, g.d_ff, (size_t)optin - st_smem - 256)
+                         ? ms::persistent_slots(batch, g.n_layers, g.d_model, g.n_heads, g.n_kv_heads, g.d_ff, g.vocab,
+                                                nsm, fmt, (size_t)optin - st_smem - 256)
                          : 0;
       if (ns >= 4) {
-        const size_t sm_bytes = ms::persistent_smem(batch, g.d_model, g.n_heads, g.d_ff, ns);
+        const size_t sm_bytes = ms::persistent_smem(batch, g.n_layers, g.d_model, g.n_heads, g.n_kv_heads, g.d_ff,
+                                                    g.vocab, nsm, fmt, ns);
         if (ms::persistent_max_ctas(batch, fmt, sm_bytes) >= 1) {
           c->persist_grid = nsm;
           c->persist_nslot = ns;
           c->persist_smem = sm_bytes;
+          c->persist_sched_cap =
+              ms::persistent_sched_cap(g.n_layers, g.d_model, g.n_heads, g.n_kv_heads, g.d_ff, g.vocab, nsm, fmt);
           int s = nsm / (batch * g.n_kv_heads);
           if (s > 128) s = 128;
           if (s > c->splits) c->splits = s;
