@@ -60,8 +60,7 @@ constexpr int kAttSub = 64;
 constexpr int kAttMaxSplits = 128;
 constexpr int kMinPerSplit = 16;
 constexpr int kTile = 16;                 // weight rows per tile (the MMA's M)
-constexpr int kMaxTiles = 4;              // tiles of one matrix per CTA
-constexpr int kMaxOwn = kTile * kMaxTiles;  // residual rows a CTA owns
+constexpr int kMaxUnits = 4;              // work units (a tile's K range) of one matrix per CTA
 constexpr int kMaxLayers = 64;            // layer table kept in shared memory
 constexpr int kPairBatch = 8;             // element pairs a thread has in flight per round
 constexpr int kRecInt4 = 320;             // tile-packed record: 64 code words + 16 scales
@@ -163,8 +162,30 @@ __host__ __device__ __forceinline__ size_t plane_bytes(int M, int kmax) {
   return align16((size_t)2 * M * (2 * kmax + 64));
 }
 __host__ __device__ __forceinline__ size_t xin_bytes(int kmax) { return align16((size_t)kmax * 4); }
-__host__ __device__ __forceinline__ size_t part_bytes(int M) { return (size_t)kMaxTiles * kWarps * M * kTile * 4; }
+__host__ __device__ __forceinline__ size_t part_bytes(int M) { return (size_t)kMaxUnits * kWarps * M * kTile * 4; }
 __host__ __device__ __forceinline__ size_t gb_bytes(int d) { return align16((size_t)d * 8); }
+
+// Work units of a matrix: each 16-row tile's K range cut into S equal parts (S = 1, 2 or
+// 4), units spread evenly over the G CTAs.  S is the smallest that minimises the busiest
+// CTA's records, counting each extra part as 10 % more work (its consumers read one more
+// partial sum per element); at most kMaxUnits units per CTA.
+__host__ __device__ __forceinline__ int choose_split(int nt, int KG, int G) {
+  int best = 1;
+  long long best_cost = -1;
+  for (int S = 1; S <= 4; S *= 2) {
+    if (KG % S != 0) continue;
+    const long long units = ((long long)nt * S + G - 1) / G;
+    if (units > kMaxUnits) continue;
+    const long long cost = units * (KG / S) * (10 + (S - 1));
+    if (best_cost < 0 || cost < best_cost) {
+      best = S;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+// First record of unit u (tile u / S, part u % S) in the tile-packed matrix.
+__host__ __device__ __forceinline__ int unit_rec(int u, int S, int KG) { return (u / S) * KG + (KG * (u % S)) / S; }
 
 // Bytes of the region's aliased part: the matrix phases' planes, staging and partial sums,
 // the attention scratch, or the LM head's input, whichever is largest.  The zero row follows.
@@ -320,11 +341,16 @@ __device__ __forceinline__ int plane_word(int p) {
   return (p >> 4) * 16 + (q & 3) * 4 + (q >> 2);
 }
 
-// Source of a vector row: stamped words (wait for epoch ep) or plain floats.
+// Source of a phase's input row: S stamped slices (st + h * stride, h < S, added in order)
+// carrying epoch ep, or plain floats (pl, the token embedding); then, with res, the CTA's
+// copy of the residual row added to the sum (res := x), or GELU applied.
 struct VecSrc {
   const uint64_t* st;
+  long long stride;
   const float* pl;
   unsigned ep;
+  float2* res;   // residual pairs of this row (each thread's own pairs), or null
+  bool gelu;
 };
 
 // Loads one vector row of K elements, optionally LayerNorm'd (g != null), into shared
@@ -333,23 +359,25 @@ struct VecSrc {
 // values (and gamma, beta) are staged in shared memory, each thread reading back only the
 // pairs it wrote.  Returns false (this thread) on a failed wait; the caller ORs the outcome
 // over the CTA.
-template <bool PLANES>
+template <bool PLANES, int S>
 __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* g, const float* bt, float eps,
                                          uint32_t* phi, uint32_t* plo, float* inv, float* act, const Region& rg,
                                          Red& red, const PersistArgs& a) {
+  constexpr int PR = kPairBatch / S;   // pairs per round per thread
   const int tid = threadIdx.x, P = K >> 1;
   float2* xin = rg.xin;
   bool ok = true;
 #pragma unroll 1
-  for (int base = 0; base < P; base += kThreads * kPairBatch) {
+  for (int base = 0; base < P; base += kThreads * PR) {
     uint64_t w0[kPairBatch], w1[kPairBatch];
     const uint64_t* pp[kPairBatch];
     bool use[kPairBatch];
 #pragma unroll
     for (int j = 0; j < kPairBatch; ++j) {
-      const int p = base + tid + j * kThreads;
+      const int pj = j / S, hj = j % S;
+      const int p = base + tid + pj * kThreads;
       use[j] = p < P;
-      pp[j] = src.st + 2 * (use[j] ? p : 0);
+      pp[j] = src.st + hj * src.stride + 2 * (use[j] ? p : 0);
       w0[j] = w1[j] = 0;
       if (use[j]) {
         if (src.st) {
@@ -362,15 +390,35 @@ __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* 
       }
     }
     if (g)
-      for (int p = base + tid; p < min(P, base + kThreads * kPairBatch); p += kThreads) {
+      for (int p = base + tid; p < min(P, base + kThreads * PR); p += kThreads) {
         const float2 gv = reinterpret_cast<const float2*>(g)[p], bv = reinterpret_cast<const float2*>(bt)[p];
         rg.gb[p] = make_float4(gv.x, gv.y, bv.x, bv.y);
       }
     if (src.st && ok) ok = settle_pairs<kPairBatch>(w0, w1, pp, use, src.ep, a);
 #pragma unroll
-    for (int j = 0; j < kPairBatch; ++j) {
-      const int p = base + tid + j * kThreads;
-      if (use[j]) xin[p] = make_float2(__uint_as_float((unsigned)w0[j]), __uint_as_float((unsigned)w1[j]));
+    for (int pj = 0; pj < PR; ++pj) {
+      const int p = base + tid + pj * kThreads;
+      if (use[pj * S]) {
+        float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < S; ++h) {
+          v0 += __uint_as_float((unsigned)w0[pj * S + h]);
+          v1 += __uint_as_float((unsigned)w1[pj * S + h]);
+        }
+        if (src.res) {
+          if (!src.pl) {
+            const float2 r = src.res[p];
+            v0 = r.x + v0;
+            v1 = r.y + v1;
+          }
+          src.res[p] = make_float2(v0, v1);
+        }
+        if (src.gelu) {
+          v0 = gelu_ool(v0);
+          v1 = gelu_ool(v1);
+        }
+        xin[p] = make_float2(v0, v1);
+      }
     }
   }
   float mean = 0.f, rstd = 1.f, bound = 0.f;
@@ -537,15 +585,14 @@ __device__ __forceinline__ void flush_tile(float (&acc)[8], float* part, int tl)
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 }
 
-// Where a matrix phase's outputs go.  mode: 0 store, 1 residual (x += value, kept in the
-// CTA's own rows and published), 2 GELU.  Outputs are {value, epoch} words at out[m * ldo + n].
-struct OutSpec {
-  int mode;
+// A matrix phase's share: units [u0, u1) of the matrix's S-part split, i.e. records
+// [rbeg, rend); outputs (partial sums) go to slice (unit % S) of out, words
+// out[h * stride + m * N + n], with epoch ep.
+struct MvJob {
+  int K, N, S, u0, u1, rbeg, rend;
   uint64_t* out;
-  int ldo;
+  long long stride;
   unsigned ep;
-  float* xown;   // residual rows of this CTA, [M][kMaxOwn], first row xr0
-  int xr0;
 };
 
 __device__ __forceinline__ unsigned atom_add_acq_rel_shared(unsigned* p, unsigned v) {
@@ -609,75 +656,65 @@ struct Ring {
   }
 };
 
-// One matrix phase over the CTA's records [rbeg, rend) (whole tiles, K/32 records each),
-// slice by slice from the ring; the A planes hold the phase's input.  Each warp takes a
-// contiguous run of each slice's records, tile segment by tile segment (kUnroll records in
-// flight, branch-free); a segment's sums go to the warp's partial slots; the CTA then adds
-// the eight warps' partials in a fixed order, scales by the input's 2^-e and applies the
-// output mode.
+// One matrix phase over the CTA's records, slice by slice from the ring; the A planes hold
+// the phase's input.  Each warp takes a contiguous run of each slice's records, unit segment
+// by unit segment (kUnroll records in flight, branch-free); a segment's sums go to the
+// warp's partial slots; the CTA then adds the eight warps' partials in a fixed order, scales
+// by the input's 2^-e and publishes each unit's 16 rows as {value, epoch} words.
 template <int M, int FMT>
-__device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, int K, int rbeg, int rend, const OutSpec& e,
-                                         const float* inv_s) {
+__device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, const MvJob& jb, const float* inv_s) {
   constexpr int RB = FMT == kInt4 ? kRecInt4 : kRecF16;
   constexpr int PER = kSlot / RB;
   constexpr int U = M > 4 ? kUnroll / 2 : kUnroll;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gid = lane >> 2, tq = lane & 3;
-  const int KG = K >> 5;
-  const int t0 = rbeg / KG, nt = (rend - rbeg) / KG;
+  const int K = jb.K, S = jb.S, KG = K >> 5;
+  const int nu = jb.u1 - jb.u0;
   const int pw = (K >> 1) + 16;
   // this lane's B rows: plane row gid (the zero row past the streams) and, for 8 streams, gid + 8
   const uint32_t* blo = (gid < 2 * M ? rg.planes + gid * pw : rg.zero) + tq * 4;
   const uint32_t* bhi = rg.planes + (M > 4 ? (gid + 8) * pw : 0) + tq * 4;
-  for (int i = lane; i < nt * M * kTile; i += 32) {
-    const int tl = i / (M * kTile);
-    rg.part[(size_t)(tl * kWarps + warp) * M * kTile + (i - tl * M * kTile)] = 0.f;
+  for (int i = lane; i < nu * M * kTile; i += 32) {
+    const int ul = i / (M * kTile);
+    rg.part[(size_t)(ul * kWarps + warp) * M * kTile + (i - ul * M * kTile)] = 0.f;
   }
   __syncwarp();
   bool ok = true;
-  for (int p = rbeg; p < rend; p += PER) {
-    const int n = min(PER, rend - p);
+  for (int p = jb.rbeg; p < jb.rend; p += PER) {
+    const int n = min(PER, jb.rend - p);
     const unsigned char* buf = ring.acquire();
     ok = ok && ring.got;
     if (ring.got) {
       const int c0 = (n * warp) >> 3, c1 = (n * (warp + 1)) >> 3;
-      const int r0 = p + c0 - rbeg;
-      int tl = r0 / KG, g = r0 - tl * KG;
       int i = c0;
       while (i < c1) {
-        const int s1 = min(c1, i + (KG - g));   // the run's records of tile tl
+        const int r = p + i;                                 // record index in the matrix
+        const int t = r / KG, g = r - t * KG;
+        const int h = ((g + 1) * S - 1) / KG;                // part of the tile holding group g
+        const int rend_u = t * KG + (KG * (h + 1)) / S;       // the unit's end
+        const int s1 = min(c1, i + (rend_u - r));
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (; i < s1; i += U) {
+        for (int gi = g; i < s1; i += U, gi += U) {
 #pragma unroll
           for (int j = 0; j < U; ++j) {
-            const int ij = min(i + j, s1 - 1);  // past the run's end: re-read its last record, not added
-            mv_record<M, FMT>(buf + (size_t)ij * RB, blo, bhi, g + (ij - i), i + j < s1, acc);
+            const int ij = min(i + j, s1 - 1);  // past the segment's end: re-read its last record, not added
+            mv_record<M, FMT>(buf + (size_t)ij * RB, blo, bhi, gi + (ij - i), i + j < s1, acc);
           }
-          g += U;
         }
-        flush_tile<M>(acc, rg.part, tl);
-        ++tl;
-        g = 0;
+        i = s1;   // the next segment starts exactly where this one ends
+        flush_tile<M>(acc, rg.part, t * S + h - jb.u0);
       }
     }
     ring.release();
   }
   if (consumer_bar_or(!ok)) return false;
-  for (int o = threadIdx.x; o < nt * kTile * M; o += kThreads) {
-    const int tl = o / (kTile * M), rem = o - tl * kTile * M, m = rem / kTile, rr = rem - m * kTile;
-    const float* pp = rg.part + (size_t)tl * kWarps * M * kTile + m * kTile + rr;
+  for (int o = threadIdx.x; o < nu * kTile * M; o += kThreads) {
+    const int ul = o / (kTile * M), rem = o - ul * kTile * M, m = rem / kTile, rr = rem - m * kTile;
+    const float* pp = rg.part + (size_t)ul * kWarps * M * kTile + m * kTile + rr;
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) v += pp[w * M * kTile];
-    v *= inv_s[m];
-    const int nn = (t0 + tl) * kTile + rr;
-    if (e.mode == 1) {
-      float* xo = e.xown + m * kMaxOwn + (nn - e.xr0);
-      v += *xo;
-      *xo = v;
-    } else if (e.mode == 2) {
-      v = gelu_ool(v);
-    }
-    st_stamp(e.out + (size_t)m * e.ldo + nn, v, e.ep);
+    const int u = jb.u0 + ul, t = u / S, h = u - t * S;
+    st_stamp(jb.out + h * jb.stride + (size_t)m * jb.N + t * kTile + rr, v * inv_s[m], jb.ep);
   }
   consumer_bar();  // the region is reused by the next phase
   return true;
@@ -751,7 +788,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
   float* Ks = scratch + kAttKs;    // [64][65]
   float* Vs = scratch + kAttVs;    // [64][64]
   const int nq = (H + 2 * Hk) * 64;
-  const uint64_t* row = a.qkv_s + (size_t)b * nq;
+  const uint64_t* row = a.vs[0] + (size_t)b * nq;   // QKV is one slice
   const float* cs = a.cosv + (size_t)pos * 32;
   const float* sn = a.sinv + (size_t)pos * 32;
   const size_t head = ((size_t)b * Hk + g) * a.cap;
@@ -975,12 +1012,12 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 
 }  // namespace
 
+// The CTA's share of each stage: sched[s] .. sched[5 + s] = records of matrix s < 4 (units
+// sched[10 + s] .. sched[14 + s] of an sched[18 + s]-part split), LM head rows for s = 4.
 template <int M, int FMT>
 __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, const Smem& sm, const PLayer* layers,
                                              const int* sched);
 
-// The CTA's units of each stage: sched[s] .. sched[5 + s] (records of matrix s < 4, LM head
-// rows for s = 4), whole tiles, contiguous and balanced over the CTAs.
 __device__ __forceinline__ int mat_KG(const PersistArgs& a, int s) { return mat_K(a, s) / 32; }
 
 template <int M, int FMT>
@@ -988,7 +1025,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent_kernel(const __
   extern __shared__ __align__(1024) unsigned char smem[];
   const Smem sm = carve(smem, a.nslot, a.sched_cap);
   __shared__ PLayer layers_s[kMaxLayers];
-  __shared__ int sched_s[10];
+  __shared__ int sched_s[22];
   const int kmax = max(max(a.d, a.H * 64), a.F);
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.nslot; ++i) {
@@ -1000,8 +1037,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_persistent_kernel(const __
     const int c = blockIdx.x, G = gridDim.x;
     for (int s = 0; s < 4; ++s) {
       const int nt = mat_N(a, s) / kTile, KG = mat_KG(a, s);
-      sched_s[s] = (nt * c / G) * KG;
-      sched_s[5 + s] = (nt * (c + 1) / G) * KG;
+      // QKV stays whole per tile: the attention reads q, k and v as one slice
+      const int S = s == 0 ? 1 : choose_split(nt, KG, G);
+      const int U = nt * S, u0 = U * c / G, u1 = U * (c + 1) / G;
+      sched_s[s] = unit_rec(u0, S, KG);
+      sched_s[5 + s] = unit_rec(u1, S, KG);
+      sched_s[10 + s] = u0;
+      sched_s[14 + s] = u1;
+      sched_s[18 + s] = S;
     }
     sched_s[4] = a.V * c / G;
     sched_s[9] = a.V * (c + 1) / G;
@@ -1062,7 +1105,6 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
   __shared__ int bidx[8][8];
   __shared__ int tok_s[8];
   __shared__ float inv_s[8];
-  __shared__ float xown[8 * kMaxOwn];   // this CTA's residual rows (same rows in C and E)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = gridDim.x;
   const int d = a.d, H = a.H, Hk = a.Hk, F = a.F, V = a.V, B = M;
@@ -1075,30 +1117,34 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
   rg.gb = reinterpret_cast<float4*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax));
   rg.part = reinterpret_cast<float*>(sm.region + plane_bytes(M, kmax) + xin_bytes(kmax) + gb_bytes(d));
   rg.zero = reinterpret_cast<const uint32_t*>(sm.region + persist_main(M, d, H, F));
+  // the CTA's copy of the residual rows (each thread's own pairs), [M][d / 2] pairs
+  float2* xres = reinterpret_cast<float2*>(sm.region + persist_main(M, d, H, F) + align16((size_t)kmax * 2 + 64));
   float* scratch = reinterpret_cast<float*>(sm.region);
   Red red{sm.red, 0};
   unsigned epoch = 0;
   const int len0 = *a.dlen;
-  // residual rows owned: the O and FC2 phases both have d rows and the same tiles
-  const int xr0 = sched[1] / (H * 2) * kTile;
-  const int xr1 = sched[6] / (H * 2) * kTile;
   const int units = B * Hk;
   int S = G / units;
   if (S < 1) S = 1;
   if (S > a.att_splits) S = a.att_splits;
   const unsigned per_step = 5u * a.L;
 
-  // The phase input: row m of a vector (stamped words, or the token embedding) into A
-  // planes rows 2m, 2m + 1.
-  auto load_planes = [&](const uint64_t* st, const float* emb, int ld, int K, unsigned ep, const float* g,
-                         const float* bt) -> bool {
+  // The phase input: row m of a vector into A planes rows 2m, 2m + 1.  st: the S slices of
+  // the vector (stride between slices, ld between rows) or null for the token embedding;
+  // res: add and update the residual copy; gelu: GELU of the sum.
+  auto load_planes = [&](const uint64_t* st, long long stride, int S, int ld, int K, unsigned ep, const float* g,
+                         const float* bt, bool res, bool gelu) -> bool {
     bool ok = true;
     const int pw = (K >> 1) + 16;
 #pragma unroll 1
     for (int m = 0; m < M; ++m) {
-      const VecSrc src{st ? st + (size_t)m * ld : nullptr, emb ? emb + (size_t)tok_s[m] * d : nullptr, ep};
-      ok = load_row<true>(src, K, g, bt, a.eps, rg.planes + (2 * m) * pw, rg.planes + (2 * m + 1) * pw, &inv_s[m],
-                          nullptr, rg, red, a) && ok;
+      const VecSrc src{st ? st + (size_t)m * ld : nullptr, stride, st ? nullptr : a.tok_emb + (size_t)tok_s[m] * d, ep,
+                       res ? xres + (size_t)m * (d / 2) : nullptr, gelu};
+      uint32_t* phi = rg.planes + (2 * m) * pw;
+      uint32_t* plo = rg.planes + (2 * m + 1) * pw;
+      if (S == 1) ok = load_row<true, 1>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
+      else if (S == 2) ok = load_row<true, 2>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
+      else ok = load_row<true, 4>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
     }
     return !consumer_bar_or(!ok);
   };
@@ -1144,23 +1190,28 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
         }
         const int mi = ph == 0 ? 0 : ph - 1;   // matrix of the phase
         const int K = mat_K(a, mi);
-        const bool emb = ph == 0 && l == 0;    // layer 0 reads the token embedding
-        if (emb)
-          for (int m = 0; m < M; ++m)
-            for (int n = xr0 + tid; n < xr1; n += kThreads)
-              xown[m * kMaxOwn + n - xr0] = a.tok_emb[(size_t)tok_s[m] * d + n];
-        const uint64_t* src = emb ? nullptr : ph == 0 ? a.xe_s : ph == 2 ? a.o_s : ph == 3 ? a.xc_s : a.u_s;
+        // the input: the token embedding (layer 0), or the previous matrix's output slices;
+        // A and D add them to the residual copy, E applies GELU to FC1's sum
+        const bool emb = ph == 0 && l == 0;
+        const int pm = ph == 0 ? 3 : ph == 2 ? -1 : ph == 3 ? 1 : 2;   // producing matrix (-1: attention)
+        const uint64_t* src = emb ? nullptr : pm < 0 ? a.o_s : a.vs[pm];
+        const long long stride = pm < 0 ? 0 : a.vstride[pm];
+        const int S_in = (emb || pm < 0) ? 1 : sched[18 + pm];   // the embedding and o are single vectors
         const float* g = ph == 0 ? ly.ln1_g : ph == 3 ? ly.ln2_g : nullptr;
         const float* bt = ph == 0 ? ly.ln1_b : ph == 3 ? ly.ln2_b : nullptr;
-        if (!load_planes(src, emb ? a.tok_emb : nullptr, K, K, epA + ph - 1, g, bt)) return false;
-        OutSpec e;
-        e.mode = (ph == 2 || ph == 4) ? 1 : ph == 3 ? 2 : 0;
-        e.out = ph == 0 ? a.qkv_s : ph == 2 ? a.xc_s : ph == 3 ? a.u_s : a.xe_s;
-        e.ldo = ph == 0 ? nq : ph == 3 ? F : d;
-        e.ep = epA + ph;
-        e.xown = xown;
-        e.xr0 = xr0;
-        if (!mv_phase<M, FMT>(ring, rg, K, sched[mi], sched[5 + mi], e, inv_s)) return false;
+        if (!load_planes(src, stride, S_in, K, K, epA + ph - 1, g, bt, ph == 0 || ph == 3, ph == 4)) return false;
+        MvJob jb;
+        jb.K = K;
+        jb.N = mat_N(a, mi);
+        jb.S = sched[18 + mi];
+        jb.u0 = sched[10 + mi];
+        jb.u1 = sched[14 + mi];
+        jb.rbeg = sched[mi];
+        jb.rend = sched[5 + mi];
+        jb.out = a.vs[mi];
+        jb.stride = a.vstride[mi];
+        jb.ep = epA + ph;
+        if (!mv_phase<M, FMT>(ring, rg, jb, inv_s)) return false;
       }
     }
     // ---- LM head + argmax ------------------------------------------------------------
@@ -1169,9 +1220,18 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
       bool ok = true;
 #pragma unroll 1
       for (int m = 0; m < M; ++m) {
-        const VecSrc src{a.xe_s + (size_t)m * d, nullptr, ep0 + per_step - 1};
-        ok = load_row<false>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
-                             red, a) && ok;
+        const VecSrc src{a.vs[3] + (size_t)m * d, a.vstride[3], nullptr, ep0 + per_step - 1, xres + (size_t)m * (d / 2),
+                         false};
+        const int S3 = sched[18 + 3];
+        if (S3 == 1)
+          ok = load_row<false, 1>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+                                  red, a) && ok;
+        else if (S3 == 2)
+          ok = load_row<false, 2>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+                                  red, a) && ok;
+        else
+          ok = load_row<false, 4>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+                                  red, a) && ok;
       }
       if (consumer_bar_or(!ok)) return false;
     }
@@ -1294,8 +1354,10 @@ int persistent_sched_cap(int L, int d, int H, int Hk, int F, int V, int G, int f
   const int Ks[4] = {d, H * 64, d, F};
   long long per_layer = 0;
   for (int s = 0; s < 4; ++s) {
-    const long long tmax = (Ns[s] / kTile + G - 1) / G;
-    per_layer += (tmax * (Ks[s] / 32) + per - 1) / per;
+    const int nt = Ns[s] / kTile, KG = Ks[s] / 32;
+    const int S = s == 0 ? 1 : choose_split(nt, KG, G);
+    const long long umax = ((long long)nt * S + G - 1) / G;
+    per_layer += (umax * (KG / S) + per - 1) / per;
   }
   const long long rows = (V + G - 1) / G, rpp = kSlot / (d * 4);
   const long long cap = (long long)L * per_layer + (rows + rpp - 1) / rpp;
@@ -1304,7 +1366,8 @@ int persistent_sched_cap(int L, int d, int H, int Hk, int F, int V, int G, int f
 
 static size_t region_bytes(int M, int d, int H, int F) {
   const int kmax = max(max(d, H * 64), F);
-  return persist_main(M, d, H, F) + align16((size_t)kmax * 2 + 64);   // + the zero row
+  // + the zero row + the residual copy
+  return persist_main(M, d, H, F) + align16((size_t)kmax * 2 + 64) + align16((size_t)M * d * 4);
 }
 
 int persistent_slots(int M, int L, int d, int H, int Hk, int F, int V, int G, int fmt, size_t smem_optin) {
@@ -1327,10 +1390,14 @@ bool persistent_shapes_ok(int M, int d, int H, int Hk, int F, int V, int G, cons
   };
   if (M != 1 && M != 2 && M != 4 && M != 8) return no("batch must be 1, 2, 4 or 8");
   if (G < 1) return no("no CTAs");
-  const int Ns[3] = {(H + 2 * Hk) * 64, d, F};
-  for (int N : Ns)
-    if (N % kTile != 0 || (N / kTile + G - 1) / G > kMaxTiles)
-      return no("a matrix needs more than 4 tiles of 16 rows per CTA");
+  const int Ns[4] = {(H + 2 * Hk) * 64, d, F, d};
+  const int Ks[4] = {d, H * 64, d, F};
+  for (int s = 0; s < 4; ++s) {
+    const int nt = Ns[s] / kTile, KG = Ks[s] / 32;
+    const int S = s == 0 ? 1 : choose_split(nt, KG, G);
+    if (Ns[s] % kTile != 0 || Ks[s] % 32 != 0 || ((long long)nt * S + G - 1) / G > kMaxUnits)
+      return no("a matrix needs more than 4 work units per CTA");
+  }
   if (d % 64 != 0 || F % 64 != 0) return no("d_model and d_ff must be multiples of 64");
   if (d > 2 * kThreads * kPairBatch) return no("d_model above 4096");
   if ((size_t)d * 4 > (size_t)kSlot) return no("an LM head row does not fit a ring slot");

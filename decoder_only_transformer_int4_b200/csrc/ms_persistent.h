@@ -29,12 +29,12 @@ struct PersistArgs {
   int* dlen;                 // cache length (device)
   int32_t* hist;             // token history [cap][B]: argmax of position p at p * B + b
   unsigned* status;
-  // Activation vectors handed from phase to phase as {value, epoch} 64-bit words.
-  uint64_t* qkv_s;           // [B][(H + 2Hk) * 64]
-  uint64_t* o_s;             // [B][H * 64]
-  uint64_t* xc_s;            // residual after attention [B][d]
-  uint64_t* xe_s;            // residual after the FFN [B][d]
-  uint64_t* u_s;             // [B][d_ff]
+  // Activation vectors handed from phase to phase as {value, epoch} 64-bit words.  vs[i]:
+  // the outputs of matrix i (QKV, O, FC1, FC2) as up to 4 slices of [B][N_i] (each a
+  // partial sum over a K range), vstride[i] words apart.
+  uint64_t* vs[4];
+  long long vstride[4];
+  uint64_t* o_s;             // attention output [B][H * 64]
   unsigned epoch_base;       // epochs of this launch: epoch_base + 1 ...
   uint64_t* part_s;          // attention partials, stamped [B][Hk][att_splits][hpg][66]: m, l, o[64]
   int att_splits;

@@ -186,7 +186,9 @@ struct ms_cache {
   cudaEvent_t ev_in = nullptr, ev_out = nullptr;
   // persistent decode kernel
   unsigned* sync3 = nullptr;             // grid barrier count, completed epoch, abort word
-  uint64_t *qkv_s = nullptr, *o_s = nullptr, *xc_s = nullptr, *xe_s = nullptr, *u_s = nullptr, *part_s = nullptr;
+  uint64_t* vs[4] = {nullptr, nullptr, nullptr, nullptr};
+  long long vstride[4] = {0, 0, 0, 0};
+  uint64_t *o_s = nullptr, *part_s = nullptr;
   size_t stamp_bytes = 0;                // the five stamped vectors, contiguous
   unsigned epoch_next = 0;               // first unused epoch of the stamped vectors
   int persist_grid = 0, persist_nslot = 0;
@@ -294,7 +296,7 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   // before the 32-bit counter would wrap
   const unsigned long long need = (unsigned long long)n_steps * 5ull * (unsigned long long)g.n_layers + 2ull;
   if ((unsigned long long)c->epoch_next + need >= 0xFFFFFFF0ull) {
-    e = cudaMemsetAsync(c->qkv_s, 0, c->stamp_bytes, st);
+    e = cudaMemsetAsync(c->vs[0], 0, c->stamp_bytes, st);
     if (e != cudaSuccess) return e;
     c->epoch_next = 0;
   }
@@ -321,11 +323,11 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.dlen = c->dlen;
   a.hist = c->hist;
   a.status = c->status;
-  a.qkv_s = c->qkv_s;
+  for (int i = 0; i < 4; ++i) {
+    a.vs[i] = c->vs[i];
+    a.vstride[i] = c->vstride[i];
+  }
   a.o_s = c->o_s;
-  a.xc_s = c->xc_s;
-  a.xe_s = c->xe_s;
-  a.u_s = c->u_s;
   a.epoch_base = c->epoch_next;
   c->epoch_next += (unsigned)need;
   a.part_s = c->part_s;
@@ -583,18 +585,27 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->lm_counter = a.take<unsigned>(4);
     c->sync3 = a.take<unsigned>(4);
     {
+      // persistent kernel: the four matrices' output slices (up to 4 each), the attention
+      // output and the attention partials, all {value, epoch} words in one block
       const size_t n_qkv = (size_t)batch * (g.n_heads + 2 * g.n_kv_heads) * 64;
       const size_t n_o = (size_t)batch * g.n_heads * 64;
       const size_t n_x = (size_t)batch * g.d_model;
       const size_t n_u = (size_t)batch * g.d_ff;
       const size_t n_p = (size_t)batch * g.n_kv_heads * c->splits * hpg * 66;  // attention partials
-      c->qkv_s = a.take<uint64_t>(n_qkv + n_o + 2 * n_x + n_u + n_p);
-      c->o_s = c->qkv_s ? c->qkv_s + n_qkv : nullptr;
-      c->xc_s = c->o_s ? c->o_s + n_o : nullptr;
-      c->xe_s = c->xc_s ? c->xc_s + n_x : nullptr;
-      c->u_s = c->xe_s ? c->xe_s + n_x : nullptr;
-      c->part_s = c->u_s ? c->u_s + n_u : nullptr;
-      c->stamp_bytes = (n_qkv + n_o + 2 * n_x + n_u + n_p) * sizeof(uint64_t);
+      const size_t total = 4 * (n_qkv + n_x + n_u + n_x) + n_o + n_p;
+      c->vs[0] = a.take<uint64_t>(total);
+      c->vstride[0] = (long long)n_qkv;
+      c->vstride[1] = (long long)n_x;
+      c->vstride[2] = (long long)n_u;
+      c->vstride[3] = (long long)n_x;
+      if (c->vs[0]) {
+        c->vs[1] = c->vs[0] + 4 * n_qkv;
+        c->vs[2] = c->vs[1] + 4 * n_x;
+        c->vs[3] = c->vs[2] + 4 * n_u;
+        c->o_s = c->vs[3] + 4 * n_x;
+        c->part_s = c->o_s + n_o;
+      }
+      c->stamp_bytes = total * sizeof(uint64_t);
     }
     c->att_counters = a.take<unsigned>((size_t)batch * g.n_kv_heads);
     c->hist = a.take<int32_t>((size_t)capacity * batch);

@@ -233,6 +233,25 @@ def test_decode_paths_agree(batch):
         assert np.abs(a[:, b_] - ref).max() <= TOL
 
 
+@pytest.mark.parametrize("batch", [1, 2, 4])
+def test_persistent_runs_cross_tiles_and_split_units(batch):
+    """A shape whose FC1 has several 16-row tiles per CTA (so a warp's run of records
+    crosses tile boundaries) and whose O and FC2 are split into K-range parts: the
+    persistent kernel against the oracle and the one-kernel-per-operation path."""
+    sh = synth.Shape("cross", 2, 256, 4, 4, 4096, vocab=300)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    prefix = synth.make_prefix(sh, batch, prefix_len=40, seed=91)
+    start = synth.make_start_tokens(batch, vocab=300, seed=92)
+    forced = synth.make_token_sequence(6, batch, vocab=300, seed=93)
+    a, ca = _run_teacher_forced(gm, batch, 64, prefix, forced, start, path=1)
+    b, cb = _run_teacher_forced(gm, batch, 64, prefix, forced, start, path=2)
+    assert ca.decode_path == 1
+    assert np.abs(a - b).max() < 1e-4
+    for b_ in range(batch):
+        ref = om.teacher_forced(prefix[b_], [int(start[b_])] + list(forced[b_]))
+        assert np.abs(a[:, b_] - ref).max() <= TOL
+
+
 def test_persistent_path_unsupported_batch_is_rejected():
     sh = synth.Shape("tiny-u", 1, 256, 4, 4, 512, vocab=50)
     draw, om, gm = _build(sh)
