@@ -48,7 +48,7 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="override the workload's decode steps (short runs for profiling)")
-    ap.add_argument("--cpu-decode-steps", type=int, default=16,
+    ap.add_argument("--cpu-decode-steps", type=int, default=256,
                     help="decode steps in the oracle's timed sample")
     return ap.parse_args()
 
