@@ -211,6 +211,24 @@ def _oracle_sample(wl: synth.Workload, n_decode: int):
     return (n_decode + 1) / dt, dt, threads, sample, om, draw
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest x over all ranks of the job (the job takes as long as its slowest rank);
+    x itself without a process group or with one rank."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_step_per_rank: int, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank (one replica per GPU) generates the same tokens per
+    step; the time is the slowest rank's."""
+    return world * tokens_per_step_per_rank * steps / (total_ms / 1e3)
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -320,13 +338,9 @@ def run_ours(a):
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     tokens_per_step = B * (wl.decode_steps + 1)
-    value = world * tokens_per_step * a.steps / (total_ms / 1e3)
+    value = job_throughput(tokens_per_step, a.steps, world, total_ms)
     per_tok = [d / wl.decode_steps for d in dec_ms]
 
     wbytes, kv = _decode_bytes_per_token(wl)
