@@ -23,6 +23,11 @@
 // which issues 3 x 4 tcgen05.mma (K = 8 each) and commits them to the stage's mbarrier.  Two
 // operand stages: the conversion of block k+1 overlaps the MMAs of block k.  Every wait is
 // bounded; TMEM is freed on every path.
+//
+// Split-K: when the output tiles are too few to fill the GPU (batched decode: 8 to 32 tiles of
+// 128 weight rows), gridDim.z CTAs share a tile, each over a contiguous run of K blocks.  Each
+// writes its fp32 partial tile to a workspace; the last of them (a per-tile ticket) adds the
+// partials in a fixed order (z = 0, 1, ...) and applies the epilogue.
 #include "ms_device.cuh"
 #include "ms_launch.cuh"
 
@@ -44,6 +49,9 @@ struct TcArgs {
   float* y;
   int ldy;
   unsigned* status;
+  int splits;          // CTAs per output tile along K (gridDim.z)
+  float* part;         // partial tiles [splits][tiles][BN][128] (splits > 1)
+  unsigned* counters;  // per-tile tickets, zero between launches (splits > 1)
 };
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
@@ -184,14 +192,17 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   const uint32_t tmem_d = tmem_base_s;
   pdl_wait();
 
-  const int nk = a.K / TK;
+  const int nk_all = a.K / TK;
+  const int z = blockIdx.z;
+  const int kb0 = nk_all * z / a.splits, kb1 = nk_all * (z + 1) / a.splits;
+  const int nk = kb1 - kb0;   // this CTA's K blocks: kb0 + 0 .. kb0 + nk - 1
   const uint32_t idesc = idesc_tf32(BN);
   uint32_t phase[2] = {0u, 0u};
   bool ok = true;
   // prologue: stage the first kStages - 1 blocks
 #pragma unroll
   for (int i = 0; i < kStages - 1; ++i) {
-    if (i < nk) stage_block<BN, FMT>(a, raw0 + i * LY::kRawStage, n0, m0, i);
+    if (i < nk) stage_block<BN, FMT>(a, raw0 + i * LY::kRawStage, n0, m0, kb0 + i);
     cp_async_commit();
   }
   for (int kb = 0; kb < nk; ++kb) {
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
     unsigned char* st = base + s * LY::kOpStage;
     // keep the copy engine kStages - 1 blocks ahead
     if (kb + kStages - 1 < nk)
-      stage_block<BN, FMT>(a, raw0 + ((kb + kStages - 1) % kStages) * LY::kRawStage, n0, m0, kb + kStages - 1);
+      stage_block<BN, FMT>(a, raw0 + ((kb + kStages - 1) % kStages) * LY::kRawStage, n0, m0, kb0 + kb + kStages - 1);
     cp_async_commit();
     cp_async_wait<kStages - 1>();  // this thread's copies of block kb have landed
     // the MMAs that read this operand stage two blocks ago must be done before it is rewritten
@@ -286,7 +297,49 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   if (__syncthreads_or(!ok)) fail_s = 1;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   pdl_trigger();
-  if (!fail_s) {
+  const int tile = blockIdx.y * gridDim.x + blockIdx.x, ntiles = gridDim.x * gridDim.y;
+  __shared__ unsigned last_s;
+  if (a.splits > 1) {
+    // ---- split-K: this CTA's partial tile to the workspace, then the last CTA of the tile
+    // adds all partials in z order and applies the epilogue.  A CTA whose waits failed still
+    // takes its ticket, so the counter returns to zero (the status word has the timeout bit).
+    const int q = warp & 3, hh = warp >> 2;
+    constexpr int kHalf = BN / 2;
+    float* wp = a.part + ((size_t)z * ntiles + tile) * BN * TM;
+#pragma unroll
+    for (int c0 = 0; c0 < (fail_s ? 0 : kHalf); c0 += 8) {
+      uint32_t r[8];
+      const int col = hh * kHalf + c0;
+      const uint32_t taddr = tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)col;
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                   : "r"(taddr)
+                   : "memory");
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wp[(size_t)(col + j) * TM + q * 32 + lane] = __uint_as_float(r[j]);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = atomicAdd(&a.counters[tile], 1u) == (unsigned)(a.splits - 1) ? 1u : 0u;
+    __syncthreads();
+    if (last_s) {
+      __threadfence();
+      for (int i = tid; i < BN * TM; i += 256) {
+        const int col = i / TM, row = i - col * TM;
+        const int n = n0 + row, m = m0 + col;
+        float v = 0.f;
+        for (int zz = 0; zz < a.splits; ++zz) v += __ldcg(a.part + ((size_t)zz * ntiles + tile) * BN * TM + i);
+        if (n < a.N && m < a.M) {
+          float* yp = a.y + (size_t)m * a.ldy + n;
+          if (EPI == kAdd) v += *yp;
+          else if (EPI == kGelu) v = gelu_erf(v);
+          *yp = v;
+        }
+      }
+      if (tid == 0) a.counters[tile] = 0u;
+    }
+  } else if (!fail_s) {
     // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (weight rows); warps 0-3 take
     // the first half of the BN columns, warps 4-7 the second ----
     const int q = warp & 3, hh = warp >> 2;
@@ -325,8 +378,24 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
 
 namespace {
 template <int BN, int FMT>
-cudaError_t tc_go(const Launch& L, const TcArgs& a, int epi) {
-  const dim3 grid((a.N + TM - 1) / TM, (a.M + BN - 1) / BN);
+cudaError_t tc_go(const Launch& L, TcArgs a, int epi, const GemmWork* gw) {
+  const int tiles = ((a.N + TM - 1) / TM) * ((a.M + BN - 1) / BN);
+  // split K when the tiles leave SMs idle: as many parts as keep the grid to one wave (one
+  // CTA per SM), at least 2 K blocks each
+  a.splits = 1;
+  if (gw && gw->ws && 2 * tiles <= gw->sms) {
+    int s = gw->sms / tiles;
+    const int nk = a.K / TK;
+    if (s > nk / 2) s = nk / 2;
+    if (s > 16) s = 16;
+    while (s > 1 && ((size_t)s * tiles * BN * TM > gw->ws_floats || tiles > gw->max_tiles)) --s;
+    if (s > 1) {
+      a.splits = s;
+      a.part = gw->ws;
+      a.counters = gw->counters;
+    }
+  }
+  const dim3 grid((a.N + TM - 1) / TM, (a.M + BN - 1) / BN, a.splits);
   const size_t smem = TcLayout<BN, FMT>::kBytes;
   Launch L2 = L;
   L2.pdl = false;  // TMEM is allocated at kernel start: keep launches stream-ordered
@@ -357,7 +426,7 @@ cudaError_t init_attrs_gemm_tc() {
 }
 
 cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y, int ldy,
-                           int epi) {
+                           int epi, const GemmWork* gw) {
   if (M <= 0) return cudaSuccess;
   if (w.K % TK != 0 || ldx % 4 != 0) return cudaErrorInvalidValue;
   TcArgs a;
@@ -374,10 +443,13 @@ cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int 
   a.y = y;
   a.ldy = ldy;
   a.status = L.status;
+  a.splits = 1;
+  a.part = nullptr;
+  a.counters = nullptr;
   const bool h = w.fmt == kFp16;
-  if (M <= 16) return h ? tc_go<16, kFp16>(L, a, epi) : tc_go<16, kInt4>(L, a, epi);
-  if (M <= 32) return h ? tc_go<32, kFp16>(L, a, epi) : tc_go<32, kInt4>(L, a, epi);
-  return h ? tc_go<64, kFp16>(L, a, epi) : tc_go<64, kInt4>(L, a, epi);
+  if (M <= 16) return h ? tc_go<16, kFp16>(L, a, epi, gw) : tc_go<16, kInt4>(L, a, epi, gw);
+  if (M <= 32) return h ? tc_go<32, kFp16>(L, a, epi, gw) : tc_go<32, kInt4>(L, a, epi, gw);
+  return h ? tc_go<64, kFp16>(L, a, epi, gw) : tc_go<64, kInt4>(L, a, epi, gw);
 }
 
 }  // namespace ms

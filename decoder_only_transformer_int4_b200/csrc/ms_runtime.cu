@@ -194,6 +194,10 @@ struct ms_cache {
   int persist_grid = 0, persist_nslot = 0;
   size_t persist_smem = 0;
   int persist_sched_cap = 0;
+  float* gemm_ws = nullptr;          // split-K partial tiles of the tcgen05 GEMM
+  size_t gemm_ws_floats = 0;
+  unsigned* gemm_ctr = nullptr;      // its per-tile tickets (zero between launches)
+  int nsm = 148;                     // SMs of the device
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
 };
@@ -210,6 +214,7 @@ ms::Launch launch_of(ms_cache* c, cudaStream_t s, bool pdl) { return ms::Launch{
 // Prefill of n = P + S rows per stream.  Rows of stream b are b * n + i.
 cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, const float* prefix, int P,
                         float* logits, int32_t* argmax, cudaStream_t st) {
+  const ms::GemmWork gw{c->gemm_ws, c->gemm_ws_floats, c->gemm_ctr, 256, c->nsm};
   const ms_config& g = m->cfg;
   const int n = P + S, B = c->B, R = B * n, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads;
   const int nq = (H + 2 * Hk) * 64;
@@ -220,13 +225,13 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
     float* kc = c->k + l * layer_stride(c);
     float* vc = c->v + l * layer_stride(c);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore, &gw);
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore, &gw);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu, &gw);
+    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore, &gw);
   }
   if (e == cudaSuccess)
     e = ms::launch_skipln(L, c->x, g.n_layers > 0 ? c->y : nullptr, m->ln_f_g, m->ln_f_b, g.ln_eps, R, d, c->h);
@@ -241,6 +246,7 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
 // the cache's token history (the greedy loop).
 cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* logits, int32_t* argmax,
                        cudaStream_t st, bool first_pdl) {
+  const ms::GemmWork gw{c->gemm_ws, c->gemm_ws_floats, c->gemm_ctr, 256, c->nsm};
   const ms_config& g = m->cfg;
   const int B = c->B, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads, F = g.d_ff;
   const int nq = (H + 2 * Hk) * 64;
@@ -258,7 +264,7 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
       e = ms::launch_gemv(L, ly.w[0], c->x, d, B, ly.ln1_g, ly.ln1_b, g.ln_eps, c->qkv, nq, ms::kStore);
     } else {
       e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore, &gw);
     }
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o);
@@ -267,10 +273,10 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[3], c->u, F, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
     } else {
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd, &gw);
       if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu, &gw);
+      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd, &gw);
     }
   }
   ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
@@ -536,6 +542,8 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
   c->cap = capacity;
   c->splits = ms::attn_decode_splits(batch, g.n_kv_heads, capacity);
   c->rows_cap = (size_t)batch * capacity;
+  cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, m->device);
+  if (c->nsm < 1) c->nsm = 1;
   {
     // persistent decode kernel: one CTA per SM if its shared memory fits
     int dev = m->device, nsm = 0, optin = 0, coop = 0;
@@ -620,6 +628,10 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->o = a.take<float>(R * g.n_heads * 64);
     c->u = a.take<float>(R * g.d_ff);
     c->logits = a.take<float>((size_t)batch * g.vocab);
+    // split-K workspace of the tcgen05 GEMM: about one partial tile per SM, twice over
+    c->gemm_ws_floats = (size_t)2 * 160 * 128 * 64;
+    c->gemm_ws = a.take<float>(c->gemm_ws_floats);
+    c->gemm_ctr = a.take<unsigned>(256);
     if (pass == 0) {
       a.size = round_up(a.used, 256);
       cudaError_t e = cudaMalloc(&a.base, a.size);
