@@ -25,9 +25,12 @@
 // bounded; TMEM is freed on every path.
 //
 // Split-K: when the output tiles are too few to fill the GPU (batched decode: 8 to 32 tiles of
-// 128 weight rows), gridDim.z CTAs share a tile, each over a contiguous run of K blocks.  Each
-// writes its fp32 partial tile to a workspace; the last of them (a per-tile ticket) adds the
-// partials in a fixed order (z = 0, 1, ...) and applies the epilogue.
+// 128 weight rows), the S <= 8 CTAs of a tile form a thread-block cluster (1, 1, S), each over
+// a contiguous run of K blocks.  Each leaves its fp32 partial tile in its own shared memory;
+// after a cluster barrier every CTA adds, for its 1/S of the tile, the S partials in rank
+// order by reading its peers' shared memory (distributed shared memory), and applies the
+// epilogue; a second cluster barrier keeps each CTA's shared memory alive until its peers
+// are done reading it.  Every CTA of the cluster passes both barriers on every path.
 #include "ms_device.cuh"
 #include "ms_launch.cuh"
 
@@ -49,10 +52,24 @@ struct TcArgs {
   float* y;
   int ldy;
   unsigned* status;
-  int splits;          // CTAs per output tile along K (gridDim.z)
-  float* part;         // partial tiles [splits][tiles][BN][128] (splits > 1)
-  unsigned* counters;  // per-tile tickets, zero between launches (splits > 1)
+  int splits;          // CTAs per output tile along K (gridDim.z = the cluster's size)
 };
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ float ld_peer(uint32_t local_saddr, uint32_t rank) {
+  uint32_t ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_saddr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   // K-major, 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (SBO),
@@ -193,7 +210,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   pdl_wait();
 
   const int nk_all = a.K / TK;
-  const int z = blockIdx.z;
+  const int z = a.splits > 1 ? (int)cluster_rank() : 0;   // this CTA's K slice
   const int kb0 = nk_all * z / a.splits, kb1 = nk_all * (z + 1) / a.splits;
   const int nk = kb1 - kb0;   // this CTA's K blocks: kb0 + 0 .. kb0 + nk - 1
   const uint32_t idesc = idesc_tf32(BN);
@@ -297,15 +314,13 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   if (__syncthreads_or(!ok)) fail_s = 1;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   pdl_trigger();
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x, ntiles = gridDim.x * gridDim.y;
-  __shared__ unsigned last_s;
   if (a.splits > 1) {
-    // ---- split-K: this CTA's partial tile to the workspace, then the last CTA of the tile
-    // adds all partials in z order and applies the epilogue.  A CTA whose waits failed still
-    // takes its ticket, so the counter returns to zero (the status word has the timeout bit).
+    // ---- split-K: partial tile [col][row] into this CTA's shared memory (operand stage 0,
+    // free now that every MMA has completed), then this CTA's 1/S of the tile summed over the
+    // cluster in rank order ----
     const int q = warp & 3, hh = warp >> 2;
     constexpr int kHalf = BN / 2;
-    float* wp = a.part + ((size_t)z * ntiles + tile) * BN * TM;
+    float* P = reinterpret_cast<float*>(base);
 #pragma unroll
     for (int c0 = 0; c0 < (fail_s ? 0 : kHalf); c0 += 8) {
       uint32_t r[8];
@@ -317,28 +332,30 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
                    : "memory");
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int j = 0; j < 8; ++j) wp[(size_t)(col + j) * TM + q * 32 + lane] = __uint_as_float(r[j]);
+      for (int j = 0; j < 8; ++j) P[(col + j) * TM + q * 32 + lane] = __uint_as_float(r[j]);
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = atomicAdd(&a.counters[tile], 1u) == (unsigned)(a.splits - 1) ? 1u : 0u;
-    __syncthreads();
-    if (last_s) {
-      __threadfence();
-      for (int i = tid; i < BN * TM; i += 256) {
-        const int col = i / TM, row = i - col * TM;
-        const int n = n0 + row, m = m0 + col;
-        float v = 0.f;
-        for (int zz = 0; zz < a.splits; ++zz) v += __ldcg(a.part + ((size_t)zz * ntiles + tile) * BN * TM + i);
-        if (n < a.N && m < a.M) {
-          float* yp = a.y + (size_t)m * a.ldy + n;
-          if (EPI == kAdd) v += *yp;
-          else if (EPI == kGelu) v = gelu_erf(v);
-          *yp = v;
-        }
+    cluster_sync_all();
+    const int S = a.splits, E = BN * TM;
+    const int e0 = E * z / S, e1 = E * (z + 1) / S;
+    const uint32_t pbase = smem_u32(P);
+    for (int e = e0 + tid; e < e1; e += 256) {
+      float part[8];
+#pragma unroll
+      for (int zz = 0; zz < 8; ++zz) part[zz] = zz < S ? ld_peer(pbase + 4u * (uint32_t)e, (uint32_t)zz) : 0.f;
+      float v = 0.f;
+#pragma unroll
+      for (int zz = 0; zz < 8; ++zz)
+        if (zz < S) v += part[zz];
+      const int col = e / TM, row = e - col * TM;
+      const int n = n0 + row, m = m0 + col;
+      if (!fail_s && n < a.N && m < a.M) {
+        float* yp = a.y + (size_t)m * a.ldy + n;
+        if (EPI == kAdd) v += *yp;
+        else if (EPI == kGelu) v = gelu_erf(v);
+        *yp = v;
       }
-      if (tid == 0) a.counters[tile] = 0u;
     }
+    cluster_sync_all();   // the peers have read this CTA's partial
   } else if (!fail_s) {
     // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (weight rows); warps 0-3 take
     // the first half of the BN columns, warps 4-7 the second ----
@@ -380,28 +397,37 @@ namespace {
 template <int BN, int FMT>
 cudaError_t tc_go(const Launch& L, TcArgs a, int epi, const GemmWork* gw) {
   const int tiles = ((a.N + TM - 1) / TM) * ((a.M + BN - 1) / BN);
-  // split K when the tiles leave SMs idle: as many parts as keep the grid to one wave (one
-  // CTA per SM), at least 2 K blocks each
+  // split K when the tiles leave SMs idle: as many parts (<= 8, a portable cluster) as keep
+  // the grid to one wave (one CTA per SM), at least 2 K blocks each
   a.splits = 1;
-  if (gw && gw->ws && 2 * tiles <= gw->sms) {
+  if (gw && 2 * tiles <= gw->sms) {
     int s = gw->sms / tiles;
     const int nk = a.K / TK;
     if (s > nk / 2) s = nk / 2;
-    if (s > 16) s = 16;
-    while (s > 1 && ((size_t)s * tiles * BN * TM > gw->ws_floats || tiles > gw->max_tiles)) --s;
-    if (s > 1) {
-      a.splits = s;
-      a.part = gw->ws;
-      a.counters = gw->counters;
-    }
+    if (s > 8) s = 8;
+    if (s > 1) a.splits = s;
   }
   const dim3 grid((a.N + TM - 1) / TM, (a.M + BN - 1) / BN, a.splits);
   const size_t smem = TcLayout<BN, FMT>::kBytes;
-  Launch L2 = L;
-  L2.pdl = false;  // TMEM is allocated at kernel start: keep launches stream-ordered
-  if (epi == kAdd) return launch_k(L2, gemm_tc_kernel<BN, FMT, kAdd>, grid, dim3(256), smem, a);
-  if (epi == kGelu) return launch_k(L2, gemm_tc_kernel<BN, FMT, kGelu>, grid, dim3(256), smem, a);
-  return launch_k(L2, gemm_tc_kernel<BN, FMT, kStore>, grid, dim3(256), smem, a);
+  void (*k)(TcArgs) = epi == kAdd    ? gemm_tc_kernel<BN, FMT, kAdd>
+                      : epi == kGelu ? gemm_tc_kernel<BN, FMT, kGelu>
+                                     : gemm_tc_kernel<BN, FMT, kStore>;
+  // TMEM is allocated at kernel start: launches stay stream-ordered (no PDL)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)a.splits;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.splits > 1 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, a);
+  if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
+  return e;
 }
 
 template <int BN>
@@ -444,8 +470,6 @@ cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int 
   a.ldy = ldy;
   a.status = L.status;
   a.splits = 1;
-  a.part = nullptr;
-  a.counters = nullptr;
   const bool h = w.fmt == kFp16;
   if (M <= 16) return h ? tc_go<16, kFp16>(L, a, epi, gw) : tc_go<16, kInt4>(L, a, epi, gw);
   if (M <= 32) return h ? tc_go<32, kFp16>(L, a, epi, gw) : tc_go<32, kInt4>(L, a, epi, gw);

@@ -74,13 +74,9 @@ cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx
 bool gemv_fits(const WView& w, int M);
 
 // General-M path on the tensor cores (tcgen05, 3xTF32): prefill and batched decode.  With
-// gw (a workspace of the caller's), K is split over several CTAs per output tile when the
-// tiles alone would leave SMs idle.
+// gw, K is split over a cluster of CTAs per output tile when the tiles alone would leave SMs
+// idle.
 struct GemmWork {
-  float* ws;           // partial tiles
-  size_t ws_floats;
-  unsigned* counters;  // per-tile tickets, zero-initialised, max_tiles of them
-  int max_tiles;
   int sms;             // SMs of the device
 };
 cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y,

@@ -194,9 +194,6 @@ struct ms_cache {
   int persist_grid = 0, persist_nslot = 0;
   size_t persist_smem = 0;
   int persist_sched_cap = 0;
-  float* gemm_ws = nullptr;          // split-K partial tiles of the tcgen05 GEMM
-  size_t gemm_ws_floats = 0;
-  unsigned* gemm_ctr = nullptr;      // its per-tile tickets (zero between launches)
   int nsm = 148;                     // SMs of the device
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
@@ -214,7 +211,7 @@ ms::Launch launch_of(ms_cache* c, cudaStream_t s, bool pdl) { return ms::Launch{
 // Prefill of n = P + S rows per stream.  Rows of stream b are b * n + i.
 cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, const float* prefix, int P,
                         float* logits, int32_t* argmax, cudaStream_t st) {
-  const ms::GemmWork gw{c->gemm_ws, c->gemm_ws_floats, c->gemm_ctr, 256, c->nsm};
+  const ms::GemmWork gw{c->nsm};
   const ms_config& g = m->cfg;
   const int n = P + S, B = c->B, R = B * n, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads;
   const int nq = (H + 2 * Hk) * 64;
@@ -246,7 +243,7 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
 // the cache's token history (the greedy loop).
 cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* logits, int32_t* argmax,
                        cudaStream_t st, bool first_pdl) {
-  const ms::GemmWork gw{c->gemm_ws, c->gemm_ws_floats, c->gemm_ctr, 256, c->nsm};
+  const ms::GemmWork gw{c->nsm};
   const ms_config& g = m->cfg;
   const int B = c->B, d = g.d_model, H = g.n_heads, Hk = g.n_kv_heads, F = g.d_ff;
   const int nq = (H + 2 * Hk) * 64;
@@ -628,10 +625,6 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->o = a.take<float>(R * g.n_heads * 64);
     c->u = a.take<float>(R * g.d_ff);
     c->logits = a.take<float>((size_t)batch * g.vocab);
-    // split-K workspace of the tcgen05 GEMM: about one partial tile per SM, twice over
-    c->gemm_ws_floats = (size_t)2 * 160 * 128 * 64;
-    c->gemm_ws = a.take<float>(c->gemm_ws_floats);
-    c->gemm_ctr = a.take<unsigned>(256);
     if (pass == 0) {
       a.size = round_up(a.used, 256);
       cudaError_t e = cudaMalloc(&a.base, a.size);
