@@ -74,6 +74,8 @@ _PROTOS = {
     "ms_cache_kernel_launches": (ctypes.c_uint64, [_P]),
     "ms_cache_set_decode_path": (_I, [_P, _I]),
     "ms_cache_decode_path": (_I, [_P]),
+    "ms_cache_set_guidance": (_I, [_P, ctypes.c_float]),
+    "ms_cache_guidance": (ctypes.c_float, [_P]),
     "ms_cache_destroy": (_I, [_P]),
     "ms_cache_kv_bytes": (ctypes.c_size_t, [ctypes.POINTER(Config), _I, _I]),
     "ms_prefill": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _P]),
@@ -285,6 +287,15 @@ class Cache:
         return int(_lib.ms_cache_kernel_launches(self._h))
 
     PATH_AUTO, PATH_PERSISTENT, PATH_PER_OP = 0, 1, 2
+
+    def set_guidance(self, scale: float):
+        """Classifier-free guidance over stream pairs (2p, 2p+1) = (conditional,
+        unconditional): both take the argmax of u + scale (k - u); 0 turns it off."""
+        _check(_lib.ms_cache_set_guidance(self._h, ctypes.c_float(scale)), "ms_cache_set_guidance")
+
+    @property
+    def guidance(self) -> float:
+        return float(_lib.ms_cache_guidance(self._h))
 
     def set_decode_path(self, path: int):
         """0 automatic, 1 persistent decode kernel, 2 one kernel per operation."""

@@ -1267,12 +1267,22 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
             }
           }
           const int v = p + r;
+          float sv[M];
 #pragma unroll
           for (int m = 0; m < M; ++m) {
-            const float s = warp_sum(acc[m]);
-            if (lane == 0 && a.logits) a.logits[(size_t)m * V + v] = s;
-            if (better(s, v, best[m], bi[m])) {
-              best[m] = s;
+            sv[m] = warp_sum(acc[m]);
+            if (lane == 0 && a.logits) a.logits[(size_t)m * V + v] = sv[m];
+          }
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            // classifier-free guidance: both streams of a pair choose by u + scale (k - u)
+            float gv = sv[m];
+            if (M >= 2 && a.guidance != 0.f) {
+              const int c2 = m & ~1;
+              gv = sv[c2 + 1] + a.guidance * (sv[c2] - sv[c2 + 1]);
+            }
+            if (better(gv, v, best[m], bi[m])) {
+              best[m] = gv;
               bi[m] = v;
             }
           }

@@ -333,6 +333,7 @@ struct LmArgs {
   int* part_idx;
   unsigned* counter;
   unsigned* status;
+  float guidance;   // 0: argmax per row; else rows (2p, 2p+1) = (conditional, unconditional) pairs
 };
 
 int lm_rpc(int V) { return (V + kTargetCtas - 1) / kTargetCtas; }
@@ -440,12 +441,22 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
         }
       }
       const int v = v0 + r;
+      float sv[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) {
-        const float s = warp_sum(acc[m]);
-        if (lane == 0 && a.logits) a.logits[(size_t)(a.m_base + m) * a.V + v] = s;
-        if (better(s, v, best[m], bi[m])) {
-          best[m] = s;
+        sv[m] = warp_sum(acc[m]);
+        if (lane == 0 && a.logits) a.logits[(size_t)(a.m_base + m) * a.V + v] = sv[m];
+      }
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        // classifier-free guidance: both rows of a pair choose by u + scale (k - u)
+        float g = sv[m];
+        if (M >= 2 && a.guidance != 0.f) {
+          const int c = m & ~1;
+          g = sv[c + 1] + a.guidance * (sv[c] - sv[c + 1]);
+        }
+        if (better(g, v, best[m], bi[m])) {
+          best[m] = g;
           bi[m] = v;
         }
       }
@@ -519,8 +530,10 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
 
 cudaError_t launch_lm_head(const Launch& L, const float* x, int ldx, int M, int d, const float* ln_g,
                            const float* ln_b, float eps, const float* W, int V, float* logits, int32_t* argmax,
-                           int32_t* hist, int hist_B, int hist_off, int* dlen, int len_add, const LmHeadWork& w) {
+                           int32_t* hist, int hist_B, int hist_off, int* dlen, int len_add, const LmHeadWork& w,
+                           float guidance) {
   if (M < 1 || M > 64 || d % 128 != 0) return cudaErrorInvalidValue;
+  if (guidance != 0.f && M % 2 != 0) return cudaErrorInvalidValue;
   LmArgs a;
   a.x = x;
   a.ldx = ldx;
@@ -541,14 +554,17 @@ cudaError_t launch_lm_head(const Launch& L, const float* x, int ldx, int M, int 
   a.part_idx = w.part_idx;
   a.counter = w.counter;
   a.status = L.status;
+  a.guidance = guidance;
   const int grid = (V + a.rpc - 1) / a.rpc;
   cudaError_t e = cudaSuccess;
-  for (int mb = 0; mb < M && e == cudaSuccess; mb += kLmMaxChunk) {
-    const int mc = M - mb < kLmMaxChunk ? M - mb : kLmMaxChunk;
-    const int mp = mc <= 1 ? 1 : mc <= 2 ? 2 : mc <= 4 ? 4 : 8;
+  // chunks of 8, 4, 2 (then 1) rows: the rows of a guidance pair stay in one launch
+  for (int mb = 0, mc = 0; mb < M && e == cudaSuccess; mb += mc) {
+    const int rest = M - mb;
+    mc = rest >= kLmMaxChunk ? kLmMaxChunk : rest >= 4 ? 4 : rest >= 2 ? 2 : 1;
+    const int mp = mc;
     a.m_base = mb;
     a.M = mc;
-    a.len_add = (mb + kLmMaxChunk >= M) ? len_add : 0;
+    a.len_add = (mb + mc >= M) ? len_add : 0;
     const size_t smem = 16 + (size_t)a.rpc * d * 4 + (size_t)mp * d * 4 + 64 * 4 + kLmWarps * mp * 8;
     Launch Lc = L;
     if (mb > 0) Lc.pdl = true;

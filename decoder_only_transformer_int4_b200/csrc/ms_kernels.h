@@ -106,10 +106,12 @@ struct LmHeadWork {
   int* part_idx;      // [grid][64]
   unsigned* counter;  // one word, zero between launches
 };
+// guidance != 0 (M even): rows (2p, 2p+1) are (conditional, unconditional) pairs and both
+// take the argmax of u + guidance (k - u); logits stay per row.
 cudaError_t launch_lm_head(const Launch& L, const float* x, int ldx, int M, int d, const float* ln_g,
                            const float* ln_b, float eps, const float* W, int V, float* logits,
                            int32_t* argmax, int32_t* hist, int hist_B, int hist_off, int* dlen,
-                           int len_add, const LmHeadWork& w);
+                           int len_add, const LmHeadWork& w, float guidance = 0.f);
 int lm_head_grid(int V);
 
 // Tile-packed copy of a backbone matrix (records of 16 rows x 32 columns, laid out for the

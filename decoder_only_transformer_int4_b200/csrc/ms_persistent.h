@@ -50,6 +50,7 @@ struct PersistArgs {
   int n_steps;
   int nslot;
   int sched_cap;             // capacity of the per-CTA slice table (entries)
+  float guidance;            // 0, or classifier-free guidance over stream pairs (2p, 2p+1)
 };
 
 cudaError_t init_attrs_persistent();

@@ -194,6 +194,7 @@ struct ms_cache {
   int persist_grid = 0, persist_nslot = 0;
   size_t persist_smem = 0;
   int persist_sched_cap = 0;
+  float guidance = 0.f;              // classifier-free guidance scale (0: off)
   int nsm = 148;                     // SMs of the device
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
@@ -235,7 +236,7 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
   ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
   if (e == cudaSuccess)
     e = ms::launch_lm_head(L, c->h + (size_t)(n - 1) * d, n * d, B, d, nullptr, nullptr, g.ln_eps, m->lm_head, g.vocab,
-                           logits, argmax, c->hist, B, n - 1, c->dlen, n, w);
+                           logits, argmax, c->hist, B, n - 1, c->dlen, n, w, c->guidance);
   return e;
 }
 
@@ -279,7 +280,7 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
   ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
   if (e == cudaSuccess)
     e = ms::launch_lm_head(L, c->x, d, B, d, m->ln_f_g, m->ln_f_b, g.ln_eps, m->lm_head, g.vocab, logits, argmax,
-                           c->hist, B, 0, c->dlen, 1, w);
+                           c->hist, B, 0, c->dlen, 1, w, c->guidance);
   return e;
 }
 
@@ -347,6 +348,7 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.n_steps = n_steps;
   a.nslot = c->persist_nslot;
   a.sched_cap = c->persist_sched_cap;
+  a.guidance = c->guidance;
   return ms::launch_decode_persistent(a, c->B, c->persist_grid, c->persist_smem, st);
 }
 
@@ -702,6 +704,17 @@ ms_status ms_cache_set_decode_path(ms_cache* c, int path) {
   c->path_request = path;
   return MS_OK;
 }
+
+ms_status ms_cache_set_guidance(ms_cache* c, float scale) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_guidance: null cache");
+  if (!std::isfinite(scale)) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_guidance: scale must be finite");
+  if (scale != 0.f && c->B % 2 != 0)
+    return fail(MS_ERR_SHAPE, "ms_cache_set_guidance: guidance pairs streams (2p, 2p+1); batch %d is odd", c->B);
+  c->guidance = scale;
+  return MS_OK;
+}
+
+float ms_cache_guidance(const ms_cache* c) { return c ? c->guidance : 0.f; }
 
 int ms_cache_decode_path(const ms_cache* c) {
   if (!c) return -1;

@@ -171,6 +171,20 @@ ms_status ms_cache_set_decode_path(ms_cache* cache, int path);
  * operation; -1 on NULL. */
 int ms_cache_decode_path(const ms_cache* cache);
 
+/* Classifier-free guidance ("MuScriptor — small (≈100M)" model card, Model description:
+ * generation with classifier-free guidance; the pages give no formula, this library reads it
+ * as the usual u + scale (k - u)).  With scale != 0 the streams of the cache form pairs
+ * (2p, 2p + 1) = (conditional, unconditional): every greedy choice — the argmax returned by
+ * ms_prefill / ms_decode_step, recorded in the token history and fed back by ms_generate —
+ * takes, for both streams of a pair, the lowest index maximising
+ *     u[v] + scale * (k[v] - u[v]),  k = conditional logits, u = unconditional logits,
+ * in fp32.  The logits returned stay each stream's own.  scale = 0 (the default) turns it
+ * off.  MS_ERR_SHAPE for a non-zero scale on an odd batch, MS_ERR_INVALID_ARG for a
+ * non-finite scale.  Host state only; applies to the next call. */
+ms_status ms_cache_set_guidance(ms_cache* cache, float scale);
+/* The current guidance scale (0 when off or on NULL). */
+float ms_cache_guidance(const ms_cache* cache);
+
 /* ---- cache transfer (host pointers, synchronous) --------------------------------------
  * Export in the pages' layout [L][batch][T][Hk][64] (T = current length);
  * import T positions in the same layout and set the length to T. */

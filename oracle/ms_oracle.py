@@ -181,6 +181,18 @@ def argmax_lowest(logits: np.ndarray) -> np.ndarray:
     return np.argmax(np.asarray(logits), axis=-1)
 
 
+def guided(logits_cond: np.ndarray, logits_uncond: np.ndarray, scale: float) -> np.ndarray:
+    """Classifier-free guidance of one (conditional, unconditional) pair of logit vectors.
+
+    "MuScriptor — small (≈100M)" model card, Model description: greedy decoding with optional
+    classifier-free guidance.  The pages give no formula; the reading used is the usual
+    u + scale * (k - u), k the conditional and u the unconditional logits (scale 1: the
+    conditional stream alone; scale 0: the unconditional one).
+    """
+    u = np.asarray(logits_uncond, np.float64)
+    return u + scale * (np.asarray(logits_cond, np.float64) - u)
+
+
 def top2_margin(logits: np.ndarray) -> np.ndarray:
     """Largest minus second-largest logit (over the last axis)."""
     part = np.sort(np.asarray(logits, np.float64), axis=-1)
@@ -323,6 +335,25 @@ class OracleModel:
             logits.append(self.decode_step(cache, toks[-1]))
             toks.append(int(argmax_lowest(logits[-1])))
         return np.array(toks, np.int64), np.stack(logits)
+
+    def greedy_guided(self, prefix_cond, prefix_uncond, start_cond: int, start_uncond: int, n_steps: int,
+                      scale: float, capacity: int):
+        """Greedy decoding of a (conditional, unconditional) pair with classifier-free
+        guidance: both streams are prefilled with their own prefix and start token, then every
+        step both receive the argmax of ``guided(k, u, scale)``.
+
+        Returns (tokens int64 [n_steps + 1], logits_cond [n_steps + 1, V], logits_uncond
+        [n_steps + 1, V]); row 0 is the prefills' output.
+        """
+        cc, cu = self.new_cache(capacity), self.new_cache(capacity)
+        lc = [self.prefill(cc, prefix_cond, [start_cond])]
+        lu = [self.prefill(cu, prefix_uncond, [start_uncond])]
+        toks = [int(argmax_lowest(guided(lc[-1], lu[-1], scale)))]
+        for _ in range(n_steps):
+            lc.append(self.decode_step(cc, toks[-1]))
+            lu.append(self.decode_step(cu, toks[-1]))
+            toks.append(int(argmax_lowest(guided(lc[-1], lu[-1], scale))))
+        return np.array(toks, np.int64), np.stack(lc), np.stack(lu)
 
     def teacher_forced(self, prefix, tokens: Sequence[int]) -> np.ndarray:
         """Logits after the prefill and after every forced token: [len(tokens), V].

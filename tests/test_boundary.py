@@ -79,3 +79,9 @@ def test_calls_reject_null_handles_and_bad_sizes_on_the_host():
     assert L.ms_op_skip_layernorm(p, None, p, p, 1e-5, 4, 100, p, None) == ms.MS_ERR_SHAPE
     assert L.ms_op_lm_head_argmax(p, 256, 65, 256, None, None, 1e-5, p, 10, p, p, None) == ms.MS_ERR_SHAPE
     assert ms.last_error()
+
+
+def test_guidance_rejects_null_cache():
+    import ctypes
+    assert ms._lib.ms_cache_set_guidance(None, ctypes.c_float(2.0)) == ms.MS_ERR_INVALID_ARG
+    assert ms._lib.ms_cache_guidance(None) == 0.0

@@ -252,6 +252,41 @@ def test_persistent_runs_cross_tiles_and_split_units(batch):
         assert np.abs(a[:, b_] - ref).max() <= TOL
 
 
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("batch", [2, 4])
+def test_classifier_free_guidance_pairs(path, batch):
+    """Streams (2p, 2p+1) = (conditional, unconditional) with guidance scale 2: both take the
+    argmax of u + 2 (k - u); tokens against the oracle's guided greedy driver (margin rule on
+    the guided logits), the two streams of a pair identical, on both decode paths."""
+    sh = synth.Shape("tiny-cfg", 2, 256, 4, 2, 512, vocab=300)
+    draw, om, gm = _build(sh, ln_random=True, std=0.05)
+    n, scale = 16, 2.0
+    prefix = synth.make_prefix(sh, batch, prefix_len=40, seed=101)
+    start = synth.make_start_tokens(batch, vocab=300, seed=102)
+    cache = ms.Cache(gm, batch, 64)
+    cache.set_decode_path(path)
+    cache.set_guidance(scale)
+    assert cache.guidance == scale
+    _, am = cache.prefill(_dev(start.reshape(batch, 1).astype(np.int64)), _dev(prefix))
+    toks, _ = cache.generate(n)
+    assert cache.device_status() == ms.MS_OK
+    got = np.concatenate([am.cpu().numpy()[None, :], toks.cpu().numpy()], axis=0)   # [n + 1, B]
+    for p in range(batch // 2):
+        assert np.array_equal(got[:, 2 * p], got[:, 2 * p + 1])
+        ref, lc, lu = om.greedy_guided(prefix[2 * p], prefix[2 * p + 1], int(start[2 * p]), int(start[2 * p + 1]), n,
+                                       scale, capacity=64)
+        _greedy_agree(list(got[:, 2 * p]), list(ref), O.guided(lc, lu, scale))
+
+
+def test_guidance_needs_an_even_batch():
+    sh = synth.Shape("tiny-u", 1, 256, 4, 4, 512, vocab=50)
+    draw, om, gm = _build(sh)
+    c = ms.Cache(gm, 3, 16)
+    with pytest.raises(ms.MsError):
+        c.set_guidance(1.5)
+    c.set_guidance(0.0)   # off is always allowed
+
+
 def test_persistent_path_unsupported_batch_is_rejected():
     sh = synth.Shape("tiny-u", 1, 256, 4, 4, 512, vocab=50)
     draw, om, gm = _build(sh)

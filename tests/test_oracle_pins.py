@@ -450,3 +450,43 @@ def test_planted_mistakes_are_caught(monkeypatch, name, patch):
     monkeypatch.setattr(O, attr, fn)
     got, _ = m.forward_full(prefix, toks)
     assert not np.allclose(got, want, rtol=0, atol=1e-6), name
+
+
+# ---------------------------------------------------------------------------
+# Classifier-free guidance ("MuScriptor — small (≈100M)" model card, Model description;
+# reading u + scale (k - u))
+# ---------------------------------------------------------------------------
+
+def test_guidance_combination_by_hand():
+    # u = [0, 1], k = [2, 0]: scale 3 gives [6, -2] (picks 0, where u alone picks 1)
+    g = O.guided(np.array([2.0, 0.0]), np.array([0.0, 1.0]), 3.0)
+    assert np.array_equal(g, np.array([6.0, -2.0]))
+    assert int(O.argmax_lowest(g)) == 0 and int(O.argmax_lowest(np.array([0.0, 1.0]))) == 1
+
+
+def test_guided_greedy_reduces_to_each_stream():
+    """Scale 1 follows the conditional stream alone, scale 0 the unconditional one: the
+    guided driver then equals the plain greedy driver on that stream."""
+    sh = synth.tiny_shape()
+    om = O.OracleModel(synth.make_weights(sh, seed=0, std=0.05), "int4")
+    pc = synth.make_prefix(sh, 1, prefix_len=6, seed=11)[0]
+    pu = synth.make_prefix(sh, 1, prefix_len=6, seed=12)[0]
+    for scale, (prefix, start) in ((1.0, (pc, 5)), (0.0, (pu, 9))):
+        toks, lc, lu = om.greedy_guided(pc, pu, 5, 9, 6, scale, capacity=16)
+        ref_toks, ref_lg = om.greedy(prefix, start, 6, capacity=16)
+        assert np.array_equal(toks, ref_toks)
+        assert np.array_equal(lc if scale == 1.0 else lu, ref_lg)
+
+
+def test_guided_greedy_feeds_both_streams_the_same_token():
+    sh = synth.tiny_shape()
+    om = O.OracleModel(synth.make_weights(sh, seed=0, std=0.05), "int4")
+    pc = synth.make_prefix(sh, 1, prefix_len=6, seed=11)[0]
+    pu = synth.make_prefix(sh, 1, prefix_len=6, seed=12)[0]
+    toks, lc, lu = om.greedy_guided(pc, pu, 5, 9, 5, 2.0, capacity=16)
+    # each stream's logits are its own teacher-forced outputs on the shared tokens
+    tf_c = om.teacher_forced(pc, [5] + list(toks[:-1]))
+    tf_u = om.teacher_forced(pu, [9] + list(toks[:-1]))
+    assert np.abs(lc - tf_c).max() < 1e-9 and np.abs(lu - tf_u).max() < 1e-9
+    for i in range(len(toks)):
+        assert toks[i] == int(np.argmax(lu[i] + 2.0 * (lc[i] - lu[i])))
