@@ -23,7 +23,7 @@ namespace {
 constexpr int kDecThreads = 128;
 constexpr int kDecSub = 64;        // positions staged in shared memory at a time
 constexpr int kMinPerSplit = 16;   // smallest run of positions worth a CTA
-constexpr int kDecTargetCtas = 2 * 148;
+constexpr int kDecTargetCtas = 6 * 148;   // several resident CTAs per SM overlap their K/V loads
 constexpr int kMaxSplits = 128;    // partials one (stream, kv head) may have
 
 struct AttnDecArgs {
