@@ -1,48 +1,49 @@
 // Persistent decode kernel: greedy decode steps of the whole decoder (all layers, LM head,
 // argmax, token feedback) in one cooperative launch, one CTA per SM.
 //
-// Why: at a few streams the decoder step is a chain of ~5 dependent matrix-vector phases
-// per layer, each moving only a few MB; separate kernel launches pay a launch and drain per
-// phase, and even a grid barrier costs ~2 us on 148 SMs.  Here the weight bytes — which
-// never depend on the previous phase — stream continuously: each CTA walks its whole weight
-// schedule (every slice of every layer of every step) with bulk copies into a shared-memory
-// ring; the slot the eight warps have just finished with is refilled at once with the slice
-// nslot places ahead, so the copies run ahead of use across phase, layer and step
-// boundaries.  And the hand-off between phases needs no barrier: every activation
-// vector a phase produces (qkv, o, x, u, attention partials) is written as 64-bit words
-// {value, epoch}, each element stored once, and the consumer polls the words it needs —
-// all of them in flight at once — until they carry the current epoch: the wait and the read
-// are one round trip.  One grid barrier per step (after the LM head) orders the rest (cache
-// append, token history).
+// Why: at a few streams the decoder step is a chain of ~6 dependent phases per layer, each
+// moving only a few MB; separate kernel launches pay a launch and drain per phase, and even a
+// grid barrier costs ~2 us on 148 SMs.  Here the weight bytes — which never depend on the
+// previous phase — stream continuously: each CTA builds the table of its weight slices for
+// one step (its records of every matrix of every layer, then its LM head rows) and copies
+// them with cp.async.bulk into a ring of shared-memory slots, nslot slices ahead of use
+// across phase, layer and step boundaries; the last warp to finish a slot refills it, with no
+// CTA barrier per slot.  The hand-off between phases needs no barrier either: every vector a
+// phase produces (QKV, O, FC1 and FC2 outputs, attention output and partials) is written once
+// as 64-bit words {value, epoch}; the consumer loads all the words it needs at once and
+// re-reads only the stale ones, all together — the wait and the read are one L2 round trip.
+// One grid barrier per step (after the LM head) orders the rest (cache append, token
+// history).
 //
 // Phases of one step (token position pos, T = pos + 1 keys):
-//   A  LN1 of x, QKV rows (raw q, k, v)                                 -> qkv
+//   A  x += FC2 parts of the previous layer (or x = the token embedding), LN1, QKV rows
 //   B  attention unit (stream, kv head, split): RoPE of q (and of the new k, which the
-//      last split appends to the cache with v), scores over its run of positions, partial
-//      (m, l, o); one CTA per head then merges the splits' partials     -> o
-//   C  O rows, residual                                                  x += o Wo^T -> xc
-//   D  LN2 of x, FC1 rows, GELU                                          -> u
-//   E  FC2 rows, residual                                                x += u W2^T -> xe
-// The residual rows a CTA owns (the same rows in C and E) stay in its shared memory; the
-// other CTAs read them from the stamped copies.
-//   after the last layer: LN_f of x, LM head rows, per-CTA argmax, last CTA picks the token,
-//   records it in the token history and advances the cache length.
+//      split holding pos appends to the cache with v), scores over its run of positions,
+//      partial (m, l, o); one CTA per head then merges the splits' partials  -> o
+//   C  O rows
+//   D  x += O parts, LN2, FC1 rows (GELU applied by the consumer when FC1 is split)
+//   E  GELU of the FC1 parts' sum, FC2 rows
+// Every CTA keeps its own copy of the residual rows x (each thread its own elements) and
+// adds the published partial sums itself, so no CTA owns output rows.
+//   after the last layer: x, LN_f, LM head rows, per-CTA argmax (guided for stream pairs
+//   when classifier-free guidance is on), the last CTA picks the token, records it in the
+//   token history and advances the cache length.
 //
-// Matrix-vector products.  A CTA owns whole tiles of 8 weight rows; the tile-packed weights
-// (records of 8 rows x 32 columns, one group of INT4 scales each) stream through the ring,
-// and the eight warps split each slot's records evenly.  Per record a warp runs two
-// m16n8k16 tensor-core MMAs with the weights as B (8 rows = the 8 columns n; INT4 codes
-// turned into exact fp16 integers with one mask and one fp16 op per pair) and the
-// activation as A: the fp32 vector, scaled by a power of two so that its largest element is
-// below 2^14, is written once per phase as an fp16 pair hi + lo (hi = fp16(x), lo =
-// fp16(x - hi)), i.e. 22 significant bits, in rows 2m and 2m + 1 of A for stream m.  The
-// products are exact and accumulate in fp32; the group's scale multiplies each record's
-// result in fp32, as in the plain dequantised product.  This replaces ~5.6 instructions per
-// weight of a CUDA-core dot product by ~2.
+// Matrix-vector products.  The weights are a tile-packed copy of each matrix: records of 16
+// rows x 32 columns (one quantisation group), each lane's MMA fragment words adjacent.  Each
+// tile's K range is cut into S = 1, 2 or 4 work units, spread evenly over the CTAs; the eight
+// warps split each slice's records.  Per record a warp runs two m16n8k16 tensor-core MMAs
+// with the 16 weight rows as A (INT4 codes turned into exact fp16 integers with one mask and
+// one fp16 op per pair) and the activations as B: the fp32 input vector, scaled by a power of
+// two so that its largest element is below 2^14, is written once per phase as an fp16 pair
+// hi + lo (hi = fp16(x), lo = fp16(x - hi): 22 significant bits), columns 2m and 2m + 1 for
+// stream m.  The products are exact, the sums fp32, and each record's result is multiplied
+// by its group's fp32 scales.
 //
-// Every wait is bounded: the grid barrier's spin, the stamp polls and the ring's mbarrier
-// waits give up after a limit, set the status word's timeout bit and an abort word that
-// makes every CTA leave; a CTA that leaves first waits (bounded) for its copies in flight.
+// Every wait is bounded: the grid barrier's spin, the stamped-word settles and the ring's
+// mbarrier waits give up after a limit, set the status word's timeout bit and an abort word
+// that makes every CTA leave; a CTA that leaves first waits (bounded) for its copies in
+// flight.
 #include <float.h>
 #include <limits.h>
 #include "ms_device.cuh"
