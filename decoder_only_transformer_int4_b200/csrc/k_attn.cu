@@ -88,18 +88,36 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
   const float* kb = a.kc + head * 64;
   const float* vb = a.vc + head * 64;
 
+  // K/V of the next run of positions are loaded into registers while the current run is
+  // computed (each thread: float4 i = tid + 128 j of the run, j < 8)
+  constexpr int kPf = kDecSub * 16 / kDecThreads;
+  float4 pk[kPf], pv[kPf];
+  auto fetch = [&](int c0, int cn) {
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) {
+      const int i = tid + j * kDecThreads, p = i >> 4, f = i & 15;
+      if (p < cn) {
+        pk[j] = reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64)[f];
+        pv[j] = reinterpret_cast<const float4*>(vb + (size_t)(c0 + p) * 64)[f];
+      }
+    }
+  };
+  if (t0 < t1) fetch(t0, min(kDecSub, t1 - t0));
   for (int c0 = t0; c0 < t1; c0 += kDecSub) {
     const int cn = min(kDecSub, t1 - c0);
     __syncthreads();
-    for (int i = tid; i < cn * 16; i += kDecThreads) {
-      const int p = i >> 4, f = i & 15;
-      const float4 kv = reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64)[f];
-      Ks[p][4 * f + 0] = kv.x;
-      Ks[p][4 * f + 1] = kv.y;
-      Ks[p][4 * f + 2] = kv.z;
-      Ks[p][4 * f + 3] = kv.w;
-      reinterpret_cast<float4*>(&Vs[p][0])[f] = reinterpret_cast<const float4*>(vb + (size_t)(c0 + p) * 64)[f];
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) {
+      const int i = tid + j * kDecThreads, p = i >> 4, f = i & 15;
+      if (p < cn) {
+        Ks[p][4 * f + 0] = pk[j].x;
+        Ks[p][4 * f + 1] = pk[j].y;
+        Ks[p][4 * f + 2] = pk[j].z;
+        Ks[p][4 * f + 3] = pk[j].w;
+        reinterpret_cast<float4*>(&Vs[p][0])[f] = pv[j];
+      }
     }
+    if (c0 + kDecSub < t1) fetch(c0 + kDecSub, min(kDecSub, t1 - c0 - kDecSub));
     __syncthreads();
     for (int i = tid; i < HPG * kDecSub; i += kDecThreads) {
       const int h = i / kDecSub, p = i - h * kDecSub;
