@@ -1,6 +1,6 @@
 """Decoder-level parity through the C ABI against the oracle.
 
-Acceptance, from the benchmark spec of parity: teacher-forced logits within max-abs 2e-3
+Acceptance: teacher-forced logits within max-abs 2e-3 of the fp64 oracle
 at every compared step; greedy tokens equal wherever the oracle's top-2 logit margin is
 above 1e-2 (after the first step below that margin the greedy runs may legitimately part,
 so the comparison stops there and the teacher-forced check carries on).  Teacher forcing
