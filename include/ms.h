@@ -164,8 +164,10 @@ ms_status ms_generate(ms_model* model, ms_cache* cache, int n_steps, int32_t* ou
 /* Decode path for ms_decode_step and ms_generate on this cache: 0 = automatic (the
  * persistent kernel when it fits, else one kernel per operation), 1 = the persistent
  * kernel (MS_ERR_UNSUPPORTED when it does not fit: batch not 1, 2, 4 or 8, or its shared
- * memory does not fit), 2 = one kernel per operation.  Both paths compute the same
- * arithmetic; the choice only changes how the work is launched.  Host state only. */
+ * memory does not fit), 2 = one kernel per operation.  Both compute the same decoder and
+ * differ only in rounding: the persistent kernel's matrix products take each activation
+ * as an exact fp16 pair hi + lo (22 significant bits, products exact, sums fp32), the
+ * other path multiplies in fp32; their logits agree to about 1e-4.  Host state only. */
 ms_status ms_cache_set_decode_path(ms_cache* cache, int path);
 /* The path the next decode call will take: 1 persistent kernel, 2 one kernel per
  * operation; -1 on NULL. */
