@@ -156,8 +156,10 @@ ms_status ms_decode_step(ms_model* model, ms_cache* cache, const int32_t* tokens
 /* Greedy loop: n_steps decode steps, each feeding the previous argmax back (the first
  * step takes the argmax of the last prefill or decode call on this cache).  out_tokens:
  * device int32 [n_steps][batch] receives every step's argmax; logits: device fp32
- * [batch][vocab] receives the last step's logits, or NULL.  Runs from a CUDA graph of
- * one step that is captured on first use and replayed; no host synchronisation. */
+ * [batch][vocab] receives the last step's logits, or NULL.  On the persistent path it
+ * runs up to 128 steps per kernel launch (the argmax feeds the next step on the device);
+ * on the per-operation path it replays a CUDA graph of one step, captured on first use.
+ * No host synchronisation either way. */
 ms_status ms_generate(ms_model* model, ms_cache* cache, int n_steps, int32_t* out_tokens,
                       float* logits, void* stream);
 
