@@ -20,8 +20,9 @@
 // (nibbles and scale of 128 weight rows, BN activation rows) three blocks ahead; 256 threads
 // dequantise and split it into the four operand tiles in the canonical K-major
 // 128-byte-swizzled layout; a proxy fence and a CTA barrier hand them to the elected thread,
-// which issues 3 x 4 tcgen05.mma (K = 8 each) and commits them to the stage's mbarrier.  Two
-// operand stages: the conversion of block k+1 overlaps the MMAs of block k.  Every wait is
+// which issues 3 x 4 tcgen05.mma (K = 8 each) and commits them to the stage's mbarrier.  Three
+// operand stages (two for 16-wide tiles): the conversion of block k+1 overlaps the MMAs of
+// blocks k and k-1.  Every wait is
 // bounded; TMEM is freed on every path.
 //
 // Split-K: when the output tiles are too few to fill the GPU (batched decode: 8 to 32 tiles of
@@ -118,6 +119,10 @@ __device__ __forceinline__ void split4(const float4 v, float4& big, float4& smal
 // bytes and one scale per row, or 64 half bytes; activations: 128 bytes per row); 256
 // threads then convert a staged block into the MMA operand tiles.
 constexpr int kStages = 4;
+// Operand stages: block k's conversion waits for the MMAs of block k - NS.  Three for wide
+// tiles; two for BN = 16, whose smaller CTAs then fit two to an SM.
+template <int BN>
+constexpr int op_stages() { return BN >= 32 ? 3 : 2; }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
@@ -141,7 +146,7 @@ struct TcLayout {
   static constexpr int kRawS = FMT == kInt4 ? TM * 4 : 0;          // staged scales
   static constexpr int kRawX = BN * TK * 4;                        // staged activations
   static constexpr int kRawStage = kRawW + kRawS + kRawX;
-  static constexpr size_t kBytes = 1024 + 2 * (size_t)kOpStage + (size_t)kStages * kRawStage;
+  static constexpr size_t kBytes = 1024 + op_stages<BN>() * (size_t)kOpStage + (size_t)kStages * kRawStage;
 };
 
 template <int BN, int FMT>
@@ -174,19 +179,20 @@ __device__ __forceinline__ void stage_block(const TcArgs& a, unsigned char* raw,
   }
 }
 
-// Stage layout (dynamic shared memory, 1024-byte aligned): two operand stages (A_big,
+// Stage layout (dynamic shared memory, 1024-byte aligned): kOpStages operand stages (A_big,
 // A_small for 128 weight rows, B_big, B_small for BN activation rows), then kStages raw
 // staging slots.
 template <int BN, int FMT, int EPI>
 __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   using LY = TcLayout<BN, FMT>;
+  constexpr int kOpStages = op_stages<BN>();
   extern __shared__ __align__(1024) unsigned char dsm[];
-  __shared__ uint64_t bars[2];
+  __shared__ uint64_t bars[kOpStages];
   __shared__ uint32_t tmem_base_s;
   __shared__ int fail_s;
   constexpr int kCols = BN < 32 ? 32 : BN;
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
-  unsigned char* raw0 = base + 2 * LY::kOpStage;
+  unsigned char* raw0 = base + kOpStages * LY::kOpStage;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * TM;   // weight rows
   const int m0 = blockIdx.y * BN;   // activation rows
@@ -198,8 +204,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < kOpStages; ++i) mbar_init(&bars[i], 1);
     mbar_fence_init();
     fail_s = 0;
   }
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   const int kb0 = nk_all * z / a.splits, kb1 = nk_all * (z + 1) / a.splits;
   const int nk = kb1 - kb0;   // this CTA's K blocks: kb0 + 0 .. kb0 + nk - 1
   const uint32_t idesc = idesc_tf32(BN);
-  uint32_t phase[2] = {0u, 0u};
+  uint32_t phases = 0u;   // bit s: the parity of operand stage s's next MMA completion
   bool ok = true;
   // prologue: stage the first kStages - 1 blocks
 #pragma unroll
@@ -223,17 +228,18 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
     cp_async_commit();
   }
   for (int kb = 0; kb < nk; ++kb) {
-    const int s = kb & 1;
+    const int s = kb % kOpStages;
     unsigned char* st = base + s * LY::kOpStage;
     // keep the copy engine kStages - 1 blocks ahead
     if (kb + kStages - 1 < nk)
       stage_block<BN, FMT>(a, raw0 + ((kb + kStages - 1) % kStages) * LY::kRawStage, n0, m0, kb0 + kb + kStages - 1);
     cp_async_commit();
     cp_async_wait<kStages - 1>();  // this thread's copies of block kb have landed
-    // the MMAs that read this operand stage two blocks ago must be done before it is rewritten
-    if (kb >= 2) {
-      if (!mbar_wait(&bars[s], phase[s], a.status)) ok = false;
-      phase[s] ^= 1u;
+    // the MMAs that read this operand stage kOpStages blocks ago must be done before it is
+    // rewritten
+    if (kb >= kOpStages) {
+      if (!mbar_wait(&bars[s], (phases >> s) & 1u, a.status)) ok = false;
+      phases ^= 1u << s;
     }
     if (__syncthreads_or(!ok)) break;  // also: every thread's copies of block kb are visible
     const unsigned char* raw = raw0 + (kb % kStages) * LY::kRawStage;
@@ -307,9 +313,9 @@ __global__ void __launch_bounds__(256, 1) gemm_tc_kernel(TcArgs a) {
   // wait for the MMAs still outstanding: the latest commit of each stage in use.  Also on
   // the failure path (bounded), so that TMEM is never freed under a running MMA.
   {
-    const int used = nk < 2 ? nk : 2;
+    const int used = nk < kOpStages ? nk : kOpStages;
     for (int s = 0; s < used; ++s)
-      if (!mbar_wait(&bars[s], phase[s], a.status)) ok = false;
+      if (!mbar_wait(&bars[s], (phases >> s) & 1u, a.status)) ok = false;
   }
   if (__syncthreads_or(!ok)) fail_s = 1;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
