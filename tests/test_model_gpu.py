@@ -338,3 +338,11 @@ def test_full_c2_small():
 def test_full_c3_medium_gqa():
     tok = _full_config("c3", 24, 40)
     assert tok.shape == (1, 2001)
+
+
+@pytest.mark.slow
+def test_full_c4_medium_64_streams():
+    # 64 independent streams through the batched path (tcgen05 GEMMs, split-K attention);
+    # streams 0 and 1 are checked against the oracle.
+    tok = _full_config("c4", 16, 16)
+    assert tok.shape == (64, 513)
