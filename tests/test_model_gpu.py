@@ -346,3 +346,28 @@ def test_full_c4_medium_64_streams():
     # streams 0 and 1 are checked against the oracle.
     tok = _full_config("c4", 16, 16)
     assert tok.shape == (64, 513)
+
+
+@pytest.mark.slow
+def test_full_c5_large():
+    # Large model, batch 1, at full size.  One oracle run (prefill + greedy) serves both
+    # checks: the GPU is teacher-forced on the oracle's own greedy tokens, and the GPU's
+    # greedy run over the whole decode length is compared under the margin rule.
+    wl = synth.WORKLOADS["c5"]
+    sh = wl.shape
+    _, om, gm = _build(sh, fmt=wl.weight_format)
+    prefix = synth.make_prefix(sh, 1, seed=1)
+    start = synth.make_start_tokens(1, seed=2)
+    steps = 6
+    ora_tok, ora_lg = om.greedy(prefix[0], int(start[0]), steps, capacity=wl.capacity)
+    forced = np.asarray(ora_tok[:steps], np.int64).reshape(1, steps)
+    got, _ = _run_teacher_forced(gm, 1, wl.capacity, prefix, forced, start)
+    err = np.abs(got[:, 0] - np.asarray(ora_lg)).max()
+    assert err <= TOL, err
+    cache = ms.Cache(gm, 1, wl.capacity)
+    _, am = cache.prefill(_dev(start.reshape(1, 1)), _dev(prefix))
+    toks, _ = cache.generate(wl.decode_steps)
+    assert cache.device_status() == ms.MS_OK
+    gpu_tok = np.concatenate([am.cpu().numpy()[None], toks.cpu().numpy()], 0).T
+    assert gpu_tok.shape == (1, wl.decode_steps + 1)
+    _greedy_agree(gpu_tok[0, : steps + 1], ora_tok, ora_lg)
