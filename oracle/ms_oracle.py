@@ -41,7 +41,11 @@ design notes of the repository):
   * fully causal attention over [prefix ; tokens], scale 1/sqrt(64), query head
     h reads kv head h // (H / Hk);
   * INT4 storage: u = q + 8 in a nibble, element 2i in the low nibble of byte i,
-    row-major [N][K/2] with row n = output feature n; scales fp32 [N][K/32].
+    row-major [N][K/2] with row n = output feature n; scales fp32 [N][K/32];
+  * ``accuracy_level=4`` (optional, ``act_int8``): activations quantised to INT8 per
+    row in blocks of 32 with the weight quantiser's rule at 127 levels a side, integer
+    block sums scaled by both scales.  The CUDA library has no such path: it keeps
+    fp32 activations.
 """
 from __future__ import annotations
 
@@ -53,11 +57,34 @@ from scipy.special import erf as _erf
 
 GROUP = 32
 QMAX = 7
+A8MAX = 127
 
 
 # ---------------------------------------------------------------------------
 # INT4 weight format  [W4A32, "Model variant": symmetric RTN INT4, group size 32]
 # ---------------------------------------------------------------------------
+
+def _symmetric_rtn_g32(a: np.ndarray, qmax: int):
+    """Symmetric round-to-nearest with one scale per 32 consecutive elements of a row.
+
+    ``a`` is rounded to fp32 [R, K].  For each group: scale = absmax / qmax (fp32
+    division), q = clamp(rint(a / scale), -qmax, qmax) (fp32 division, round half to
+    even).  An all-zero group has scale 0 and q 0.  Returns (q int8 [R, K], scale fp32
+    [R, K/32]).
+    """
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    n, k = a.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 32")
+    g = a.reshape(n, k // GROUP, GROUP)
+    absmax = np.max(np.abs(g), axis=2)                                    # fp32
+    scale = (absmax / np.float32(qmax)).astype(np.float32)                # fp32 IEEE division
+    safe = np.where(scale == 0, np.float32(1), scale).astype(np.float32)
+    ratio = (g / safe[:, :, None]).astype(np.float32)                     # fp32 IEEE division
+    q = np.clip(np.rint(ratio), -qmax, qmax)
+    q = np.where(scale[:, :, None] == 0, 0, q).astype(np.int8)
+    return q.reshape(n, k), scale
+
 
 def quantize_int4_g32(w: np.ndarray):
     """Symmetric round-to-nearest INT4 with one scale per 32 consecutive K elements.
@@ -67,18 +94,7 @@ def quantize_int4_g32(w: np.ndarray):
     (fp32 division, round half to even).  An all-zero group has scale 0 and q 0.
     Returns (q int8 [N, K], scale fp32 [N, K/32]).
     """
-    w = np.ascontiguousarray(w, dtype=np.float32)
-    n, k = w.shape
-    if k % GROUP:
-        raise ValueError("K must be a multiple of 32")
-    g = w.reshape(n, k // GROUP, GROUP)
-    absmax = np.max(np.abs(g), axis=2)                                    # fp32
-    scale = (absmax / np.float32(QMAX)).astype(np.float32)                # fp32 IEEE division
-    safe = np.where(scale == 0, np.float32(1), scale).astype(np.float32)
-    ratio = (g / safe[:, :, None]).astype(np.float32)                     # fp32 IEEE division
-    q = np.clip(np.rint(ratio), -QMAX, QMAX)
-    q = np.where(scale[:, :, None] == 0, 0, q).astype(np.int8)
-    return q.reshape(n, k), scale
+    return _symmetric_rtn_g32(w, QMAX)
 
 
 def pack_int4(q: np.ndarray) -> np.ndarray:
@@ -106,6 +122,46 @@ def dequantize(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
     n, k = q.shape
     s = np.repeat(scale.astype(np.float32), GROUP, axis=1)
     return (q.astype(np.float32) * s).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# INT8 activations, INT32 accumulation  [W4A32, "Model variant": accuracy_level=4]
+# ---------------------------------------------------------------------------
+
+def quantize_act_int8_g32(x: np.ndarray):
+    """Dynamic symmetric INT8 quantisation of activation rows, one scale per 32 elements.
+
+    [W4A32, "Model variant"]: with ``accuracy_level=4`` the CPU kernels quantise the
+    MatMul activations to INT8 at run time and accumulate in INT32.  The page gives
+    neither the block length nor the scale or rounding rule.  The reading used: blocks
+    of 32 consecutive K elements of a row (the weight group, so every block meets one
+    weight scale), with the weight quantiser's rule at 127 levels a side: scale =
+    absmax / 127, q = clamp(rint(x / scale), -127, 127), fp32 IEEE divisions, ties to
+    even; an all-zero block has scale 0 and q 0.  The graph's activations are fp32, so
+    ``x`` [M, K] is rounded to fp32 first.  Returns (q int8 [M, K], scale fp32 [M, K/32]).
+    """
+    return _symmetric_rtn_g32(x, A8MAX)
+
+
+def matmul_w4a8(x: np.ndarray, q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """y[m, n] = sum over blocks b of sa[m, b] * sw[n, b] * (sum_{k in b} qa[m, k] * q[n, k]).
+
+    ``x`` [M, K] activations (quantised here by :func:`quantize_act_int8_g32`), ``q``
+    INT4 codes [N, K] and ``scale`` fp32 [N, K/32] of the weight.  Each block's inner
+    sum is an exact integer (|sum| <= 32 * 127 * 7 = 28448, which INT32 holds); the
+    per-block products sa * sw are exact in float64 and the blocks are summed in
+    float64.  Returns float64 [M, N].
+    """
+    qa, sa = quantize_act_int8_g32(x)
+    m, k = qa.shape
+    n = q.shape[0]
+    y = np.zeros((m, n))
+    for b in range(k // GROUP):
+        cols = slice(b * GROUP, (b + 1) * GROUP)
+        # integers well below 2^53: the float64 matmul is exact
+        isum = qa[:, cols].astype(np.float64) @ q[:, cols].astype(np.float64).T
+        y += isum * (sa[:, b].astype(np.float64)[:, None] * scale[:, b].astype(np.float64)[None, :])
+    return y
 
 
 # ---------------------------------------------------------------------------
@@ -223,12 +279,20 @@ class OracleModel:
     "fp16": every backbone matrix is rounded to IEEE half (the half-precision
     weight variant of "MuScriptor for Core AI (.aimodel)", file table).  "fp32":
     the matrices as drawn.  Embeddings, LayerNorms and the LM head stay fp32.
+
+    ``act_int8`` (INT4 format only): the four backbone MatMuls of every layer take
+    their activations through :func:`matmul_w4a8` (the ``accuracy_level=4`` reading);
+    attention and the LM head stay as they are, since only the backbone MatMuls are
+    MatMulNBits nodes ([W4A32, "Model variant"]).
     """
 
-    def __init__(self, draw, weight_format: str = "int4", store=np.float64):
+    def __init__(self, draw, weight_format: str = "int4", store=np.float64, act_int8: bool = False):
         sh = draw.shape
         self.shape = sh
         self.weight_format = weight_format
+        if act_int8 and weight_format != "int4":
+            raise ValueError("int8 activations go with the INT4 weight format")
+        self.act_int8 = act_int8
         self.L, self.d, self.H, self.Hk = sh.n_layers, sh.d_model, sh.n_heads, sh.n_kv_heads
         self.hd, self.F, self.V = sh.head_dim, sh.d_ff, sh.vocab
         self.base, self.eps = sh.rope_base, sh.ln_eps
@@ -254,6 +318,12 @@ class OracleModel:
             self.layers.append(OracleLayer(ld.ln1_g, ld.ln1_b, ld.ln2_g, ld.ln2_b, ws,
                                            qs or None, ss or None, ps or None))
 
+    def _matmul(self, a: np.ndarray, ly: OracleLayer, i: int) -> np.ndarray:
+        """a @ W_i^T for backbone matrix i (QKV, O, FC1, FC2) of layer ``ly``."""
+        if self.act_int8:
+            return matmul_w4a8(a, ly.q[i], ly.s[i])
+        return a @ ly.w[i].T
+
     # -- one pass over new rows, attending to the cache plus themselves --------
     def _run(self, x: np.ndarray, cache: "OracleCache", all_logits: bool) -> np.ndarray:
         """Append the rows ``x`` [n, d] (in sequence order) to ``cache`` and return logits.
@@ -272,7 +342,7 @@ class OracleModel:
         x = np.asarray(x, np.float64)
         for l, ly in enumerate(self.layers):
             h = layer_norm(x, ly.ln1_g, ly.ln1_b, self.eps)
-            qkv = h @ ly.w[0].T
+            qkv = self._matmul(h, ly, 0)
             q = qkv[:, : H * hd].reshape(n, H, hd)
             k = qkv[:, H * hd: (H + Hk) * hd].reshape(n, Hk, hd)
             v = qkv[:, (H + Hk) * hd:].reshape(n, Hk, hd)
@@ -281,9 +351,9 @@ class OracleModel:
             cache.k[l][t0: t0 + n] = k
             cache.v[l][t0: t0 + n] = v
             a = attention(q, cache.k[l][: t0 + n], cache.v[l][: t0 + n], pos, kpos)
-            x = x + a.reshape(n, H * hd) @ ly.w[1].T
+            x = x + self._matmul(a.reshape(n, H * hd), ly, 1)
             h = layer_norm(x, ly.ln2_g, ly.ln2_b, self.eps)
-            x = x + gelu_erf(h @ ly.w[2].T) @ ly.w[3].T
+            x = x + self._matmul(gelu_erf(self._matmul(h, ly, 2)), ly, 3)
         cache.length = t0 + n
         rows = x if all_logits else x[-1:]
         y = layer_norm(rows, self.ln_f_g, self.ln_f_b, self.eps)

@@ -490,3 +490,205 @@ def test_guided_greedy_feeds_both_streams_the_same_token():
     assert np.abs(lc - tf_c).max() < 1e-9 and np.abs(lu - tf_u).max() < 1e-9
     for i in range(len(toks)):
         assert toks[i] == int(np.argmax(lu[i] + 2.0 * (lc[i] - lu[i])))
+
+
+# ---------------------------------------------------------------------------
+# INT8 activations with INT32 accumulation ("MuScriptor Medium — optimized W4A32 ONNX
+# Runtime", Model variant: accuracy_level=4; reading: blocks of 32, absmax / 127, ties to
+# even, integer block sums scaled by both scales)
+# ---------------------------------------------------------------------------
+
+def _a8_hand_row(g):
+    x = np.zeros((1, g["K"]), np.float32)
+    for b, blk in enumerate(g["blocks"]):
+        x[0, 32 * b: 32 * b + len(blk["x_head"])] = blk["x_head"]
+    return x
+
+
+def _a8_hand_mismatches(g):
+    """What of the hand example the oracle's quantiser gets wrong (empty when right)."""
+    bad = []
+    try:
+        qa, sa = O.quantize_act_int8_g32(_a8_hand_row(g))
+    except Exception as e:          # a planted mistake may not even run
+        return [repr(e)]
+    if qa.shape != (1, g["K"]) or sa.shape != (1, len(g["blocks"])):
+        return ["shapes"]
+    for b, blk in enumerate(g["blocks"]):
+        if float(sa[0, b]) != blk["scale"]:
+            bad.append(("scale", b, float(sa[0, b])))
+        head = [int(v) for v in qa[0, 32 * b: 32 * b + len(blk["q_head"])]]
+        if head != blk["q_head"]:
+            bad.append(("codes", b, head))
+        if np.any(qa[0, 32 * b + len(blk["q_head"]): 32 * (b + 1)] != 0):
+            bad.append(("tail", b))
+    return bad
+
+
+def _w4a8_bruteforce_err(seed):
+    """Largest gap between matmul_w4a8 and scalar loops over bytes and Python integers."""
+    x = synth.make_activations(2, 64, seed=seed)
+    x[1, 32:] = 0.0                                    # an all-zero block
+    w = synth.make_matrix(3, 64, seed=seed + 1)
+    q, s = O.quantize_int4_g32(w)
+    packed = O.pack_int4(q)
+    got = O.matmul_w4a8(x, q, s)
+    worst = 0.0
+    for m in range(2):
+        for n in range(3):
+            acc = 0.0
+            for b in range(2):
+                blk = [np.float32(v) for v in x[m, 32 * b: 32 * b + 32]]
+                amax = max(abs(v) for v in blk)
+                sa = np.float32(amax / np.float32(127))
+                isum = 0
+                for j, v in enumerate(blk):
+                    code = 0 if sa == 0 else max(-127, min(127, round(float(np.float32(v / sa)))))
+                    byte = int(packed[n, (32 * b + j) // 2])
+                    wq = ((byte >> 4) if (j & 1) else (byte & 15)) - 8
+                    isum += code * wq
+                acc += isum * (float(sa) * float(s[n, b]))
+            worst = max(worst, abs(acc - got[m, n]) / (1 + abs(acc)))
+    return worst
+
+
+def test_a8_hand_example():
+    g = _gold("a8_block_hand.json")
+    assert _a8_hand_mismatches(g) == []
+    mm = g["matmul"]
+    q = np.zeros((1, g["K"]), np.int8)
+    for b, (head, fill) in enumerate(zip(mm["w_q_head"], mm["w_q_fill"])):
+        q[0, 32 * b: 32 * (b + 1)] = fill
+        q[0, 32 * b: 32 * b + len(head)] = head
+    s = np.array([mm["w_scale"]], np.float32)
+    x = _a8_hand_row(g)
+    assert O.matmul_w4a8(x, q, s)[0, 0] == mm["y"]
+    # the same weights with fp32 activations, through the pinned dequantised path
+    assert (x.astype(np.float64) @ O.dequantize(q, s).astype(np.float64).T)[0, 0] == mm["y_fp32_activations"]
+
+
+def test_a8_error_bound_and_extremes():
+    x = synth.make_activations(5, 256, seed=51) * np.float32(3.0)
+    qa, sa = O.quantize_act_int8_g32(x)
+    assert qa.dtype == np.int8 and np.abs(qa.astype(np.int32)).max() <= 127
+    back = qa.astype(np.float64).reshape(5, 8, 32) * sa.astype(np.float64)[:, :, None]
+    err = np.abs(back - x.astype(np.float64).reshape(5, 8, 32))
+    assert np.all(err <= sa.astype(np.float64)[:, :, None] * (0.5 + 1e-6))
+    # each block's largest magnitude lands on +-127, with its sign
+    blocks = x.reshape(5, 8, 32)
+    arg = np.abs(blocks).argmax(axis=2)
+    top = np.take_along_axis(qa.reshape(5, 8, 32), arg[:, :, None], axis=2)[:, :, 0]
+    sign = np.sign(np.take_along_axis(blocks, arg[:, :, None], axis=2)[:, :, 0])
+    assert np.array_equal(top.astype(np.int32), (127 * sign).astype(np.int32))
+
+
+def test_a8_power_of_two_and_sign_invariance():
+    x = synth.make_activations(3, 128, seed=52)
+    w = synth.make_matrix(4, 128, seed=53)
+    q, s = O.quantize_int4_g32(w)
+    qa, sa = O.quantize_act_int8_g32(x)
+    y = O.matmul_w4a8(x, q, s)
+    for j in (-12, 5):
+        f = np.float32(2.0 ** j)
+        qa2, sa2 = O.quantize_act_int8_g32(x * f)
+        assert np.array_equal(qa2, qa) and np.array_equal(sa2, sa * f)
+        assert np.array_equal(O.matmul_w4a8(x * f, q, s), y * float(f))
+    qn, sn = O.quantize_act_int8_g32(-x)
+    assert np.array_equal(qn, -qa) and np.array_equal(sn, sa)
+
+
+def test_w4a8_matmul_bruteforce():
+    assert _w4a8_bruteforce_err(54) <= 1e-12
+
+
+def test_w4a8_reduces_to_w4a32_on_exact_activations():
+    """Blocks of integers whose largest magnitude is 127 have scale 1 and codes equal to the
+    values, so the INT8 path must give the plain product x W^T with W = q * s.  (W is formed
+    in float64 here: the INT8 path scales exact integer sums and never rounds q * s to fp32
+    the way the W4A32 dequantiser does.)"""
+    g = np.random.default_rng(55)
+    x = g.integers(-127, 128, size=(3, 96)).astype(np.float32)
+    x[:, ::32] = np.float32(127) * np.where(g.random((3, 3)) < 0.5, -1, 1)
+    qa, sa = O.quantize_act_int8_g32(x)
+    assert np.all(sa == 1) and np.array_equal(qa.astype(np.float32), x)
+    w = synth.make_matrix(5, 96, seed=56)
+    q, s = O.quantize_int4_g32(w)
+    wd = q.astype(np.float64) * np.repeat(s.astype(np.float64), 32, axis=1)
+    want = x.astype(np.float64) @ wd.T
+    assert np.allclose(O.matmul_w4a8(x, q, s), want, rtol=1e-13, atol=1e-13)
+
+
+def test_w4a8_model_is_causal_and_incremental():
+    sh = synth.tiny_shape()
+    m = O.OracleModel(synth.make_weights(sh, seed=0, std=0.05), "int4", act_int8=True)
+    plain = O.OracleModel(synth.make_weights(sh, seed=0, std=0.05), "int4")
+    prefix = synth.make_prefix(sh, 1, prefix_len=6, seed=57)[0]
+    toks = synth.make_token_sequence(5, 1, vocab=m.V, seed=58)[0]
+    full, _ = m.forward_full(prefix, toks)
+    cache = m.new_cache(16)
+    rows = [m.prefill(cache, prefix, toks[:1])] + [m.decode_step(cache, int(t)) for t in toks[1:]]
+    assert np.allclose(np.stack(rows), full[6:], rtol=0, atol=1e-12)
+    toks2 = toks.copy()
+    toks2[3] = (toks2[3] + 1) % m.V
+    full2, _ = m.forward_full(prefix, toks2)
+    assert np.array_equal(full[: 6 + 3], full2[: 6 + 3])
+    # the INT8 activations change the logits, but only by quantisation noise
+    ref, _ = plain.forward_full(prefix, toks)
+    rel = np.linalg.norm(full - ref) / np.linalg.norm(ref)
+    assert 0 < rel < 0.05, rel
+    with pytest.raises(ValueError):
+        O.OracleModel(synth.make_weights(sh, seed=0, std=0.05), "fp16", act_int8=True)
+
+
+_ORIG_A8 = O.quantize_act_int8_g32
+_ORIG_W4A8 = O.matmul_w4a8
+
+
+def _a8_divisor_128(x):
+    return O._symmetric_rtn_g32(x * np.float32(127.0 / 128.0), 127)
+
+
+def _a8_one_scale_per_row(x):
+    x = np.asarray(x, np.float32)
+    sa = (np.abs(x).max(axis=1) / np.float32(127)).astype(np.float32)
+    safe = np.where(sa == 0, np.float32(1), sa)
+    qa = np.clip(np.rint(x / safe[:, None]), -127, 127).astype(np.int8)
+    return qa, np.repeat(sa[:, None], x.shape[1] // 32, axis=1)
+
+
+def _a8_half_away_from_zero(x):
+    x = np.asarray(x, np.float32)
+    b = x.reshape(x.shape[0], -1, 32)
+    sa = (np.abs(b).max(axis=2) / np.float32(127)).astype(np.float32)
+    safe = np.where(sa == 0, np.float32(1), sa)
+    r = (b / safe[:, :, None]).astype(np.float32)
+    qa = (np.sign(r) * np.floor(np.abs(r) + 0.5)).astype(np.int8)
+    return qa.reshape(x.shape), sa
+
+
+def _w4a8_first_block_scale(x, q, s):
+    qa, sa = _ORIG_A8(x)
+    sa = np.repeat(sa[:, :1], sa.shape[1], axis=1)
+    y = np.zeros((qa.shape[0], q.shape[0]))
+    for b in range(qa.shape[1] // 32):
+        c = slice(32 * b, 32 * b + 32)
+        y += (qa[:, c].astype(np.float64) @ q[:, c].astype(np.float64).T) * (sa[:, b, None] * s[None, :, b])
+    return y
+
+
+def _w4a8_weight_transposed_blocks(x, q, s):
+    return _ORIG_W4A8(x, q, s[:, ::-1].copy())
+
+
+@pytest.mark.parametrize("name,attr,fn", [
+    ("activation divisor 128", "quantize_act_int8_g32", _a8_divisor_128),
+    ("one activation scale per row", "quantize_act_int8_g32", _a8_one_scale_per_row),
+    ("round half away from zero", "quantize_act_int8_g32", _a8_half_away_from_zero),
+    ("activation scale of the wrong block", "matmul_w4a8", _w4a8_first_block_scale),
+    ("weight scales in the wrong order", "matmul_w4a8", _w4a8_weight_transposed_blocks),
+])
+def test_w4a8_planted_mistakes_are_caught(monkeypatch, name, attr, fn):
+    monkeypatch.setattr(O, attr, fn)
+    g = _gold("a8_block_hand.json")
+    caught = bool(_a8_hand_mismatches(g)) or _w4a8_bruteforce_err(54) > 1e-12
+    assert caught, name
