@@ -117,7 +117,7 @@ ms_status ms_quantize_int4_g32(const float* w, int N, int K, uint8_t* packed, fl
 ms_status ms_model_create(const ms_config* cfg, const ms_weights* weights, int device,
                           ms_model** out);
 ms_status ms_model_destroy(ms_model* model);
-/* Bytes of device memory the model's weights occupy. */
+/* Bytes of device memory the model's weights occupy; 0 on NULL. */
 size_t ms_model_weight_bytes(const ms_model* model);
 
 /* ---- cache -------------------------------------------------------------------------
@@ -128,8 +128,8 @@ size_t ms_model_weight_bytes(const ms_model* model);
 ms_status ms_cache_create(ms_model* model, int batch, int capacity, ms_cache** out);
 ms_status ms_cache_reset(ms_cache* cache); /* length = 0; no device work */
 int ms_cache_length(const ms_cache* cache);   /* positions held (host view), -1 on NULL */
-int ms_cache_capacity(const ms_cache* cache);
-int ms_cache_batch(const ms_cache* cache);
+int ms_cache_capacity(const ms_cache* cache); /* positions per stream, -1 on NULL */
+int ms_cache_batch(const ms_cache* cache);    /* streams, -1 on NULL */
 ms_status ms_cache_destroy(ms_cache* cache);
 /* Bytes of K plus V for a cache of this shape (no allocation): 2 * L * batch * Hk *
  * capacity * 64 * 4.  For the medium model with Hk = 16 and capacity 2504 this is the
@@ -201,7 +201,7 @@ ms_status ms_cache_import(ms_cache* cache, const float* k, const float* v, int T
 ms_status ms_device_status(ms_cache* cache, void* stream);
 /* Number of CUDA kernels the calls on this cache have launched so far: direct launches
  * plus, for every replay of a captured graph, the kernels in that graph.  Host counter,
- * no device work. */
+ * no device work; 0 on NULL. */
 uint64_t ms_cache_kernel_launches(const ms_cache* cache);
 /* Message of the last error on the calling thread ("" if none). */
 const char* ms_last_error(void);

@@ -81,6 +81,31 @@ def test_calls_reject_null_handles_and_bad_sizes_on_the_host():
     assert ms.last_error()
 
 
+def test_every_handle_call_rejects_null_on_the_host():
+    """The documented answer of each call to a NULL handle, before any device work."""
+    L = ms._lib
+    bad = ms.MS_ERR_INVALID_ARG
+    assert L.ms_model_destroy(None) == bad
+    assert L.ms_cache_destroy(None) == bad
+    assert L.ms_cache_reset(None) == bad
+    assert L.ms_cache_set_decode_path(None, 1) == bad
+    assert L.ms_cache_import(None, None, None, 0) == bad
+    assert L.ms_cache_capacity(None) == -1 and L.ms_cache_batch(None) == -1
+    assert L.ms_cache_decode_path(None) == -1
+    assert L.ms_model_weight_bytes(None) == 0 and L.ms_cache_kernel_launches(None) == 0
+    assert L.ms_cache_kv_bytes(None, 1, 16) == 0
+    cfg = ms.make_config(synth.SMALL)
+    assert L.ms_cache_kv_bytes(ctypes.byref(cfg), 0, 16) == 0
+    assert L.ms_cache_kv_bytes(ctypes.byref(cfg), 1, 0) == 0
+    p = ctypes.c_void_p(16)
+    assert L.ms_op_matmul_f16(None, 1, 64, p, 8, p, None) == bad
+    assert L.ms_op_lm_head_argmax(None, 256, 1, 256, None, None, 1e-5, p, 10, p, p, None) == bad
+    # gamma without beta is refused before the scratch is touched
+    assert L.ms_op_lm_head_argmax_static(p, 256, 1, 256, p, None, 1e-5, p, 10, p, p, None) == bad
+    assert L.ms_op_lm_head_argmax_static(p, 256, 65, 256, None, None, 1e-5, p, 10, p, p, None) == ms.MS_ERR_SHAPE
+    assert "ms_op_lm_head_argmax_static" in ms.last_error()
+
+
 def test_guidance_rejects_null_cache():
     import ctypes
     assert ms._lib.ms_cache_set_guidance(None, ctypes.c_float(2.0)) == ms.MS_ERR_INVALID_ARG
