@@ -320,6 +320,56 @@ def test_causality():
     assert not np.allclose(a[8], b[8])
 
 
+def _sequence_mismatches(m, draw):
+    """Where [prefix ; E[tokens]] differs from its definition, checked row by row against
+    the drawn prefix and embedding table (muscriptor-small-lm.onnx of "MuScriptor small —
+    ONNX conversion": the prefix rows come first, then one embedding row per token)."""
+    prefix = synth.make_prefix(m.shape, 1, prefix_len=4, seed=45)[0]
+    toks = [3, 0, m.V - 1, 3]
+    seq = m.sequence(prefix, toks)
+    bad = []
+    if seq.shape != (4 + len(toks), m.d):
+        return ["shape"]
+    for i in range(4):
+        if not np.array_equal(seq[i], prefix[i].astype(np.float64)):
+            bad.append(("prefix row", i))
+    for i, t in enumerate(toks):
+        if not np.array_equal(seq[4 + i], draw.tok_emb[t].astype(np.float64)):
+            bad.append(("token row", i))
+    return bad
+
+
+def test_sequence_is_prefix_then_token_embeddings():
+    sh = synth.tiny_shape(n_layers=1, n_heads=2, n_kv_heads=1, vocab=37)
+    draw = synth.make_weights(sh, seed=31, std=0.08)
+    m = O.OracleModel(draw, "int4")
+    assert _sequence_mismatches(m, draw) == []
+    # the prefix conditions what follows it, and nothing after it reaches back
+    prefix = synth.make_prefix(sh, 1, prefix_len=4, seed=46)[0]
+    toks = synth.make_token_sequence(3, 1, vocab=m.V, seed=47)[0]
+    a, _ = m.forward_full(prefix, toks)
+    other = prefix.copy()
+    other[1] = -other[1]            # (a constant shift would vanish in the LayerNorm)
+    b, _ = m.forward_full(other, toks)
+    assert np.array_equal(a[:1], b[:1]) and not np.allclose(a[4], b[4])
+    toks2 = toks.copy()
+    toks2[0] = (toks2[0] + 1) % m.V
+    c, _ = m.forward_full(prefix, toks2)
+    assert np.array_equal(a[:4], c[:4])
+
+
+def test_sequence_order_mistake_is_caught(monkeypatch):
+    sh = synth.tiny_shape(n_layers=1, n_heads=2, n_kv_heads=1, vocab=37)
+    draw = synth.make_weights(sh, seed=31, std=0.08)
+    m = O.OracleModel(draw, "int4")
+
+    def tokens_first(prefix, tokens):
+        return np.concatenate([m.embed(tokens), np.asarray(prefix, np.float64)], axis=0)
+
+    monkeypatch.setattr(m, "sequence", tokens_first)
+    assert _sequence_mismatches(m, draw)
+
+
 def test_shapes_per_step_follow_the_pages():
     figs = _gold("pages_figures.json")
     m = _tiny_model(L=3, h=2, hk=1, vocab=figs["vocab"]["value"])
