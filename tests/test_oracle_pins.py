@@ -358,6 +358,19 @@ def test_sequence_is_prefix_then_token_embeddings():
     assert np.array_equal(a[:4], c[:4])
 
 
+def test_fp16_weights_are_the_ieee_half_of_the_draw():
+    """The fp16 variant ("MuScriptor for Core AI (.aimodel)", file table: weights cast to
+    half) against torch's own float32 -> float16 cast (round to nearest even)."""
+    sh = synth.tiny_shape(n_layers=2, n_heads=2, n_kv_heads=1, vocab=37)
+    draw = synth.make_weights(sh, seed=31, std=0.08)
+    m = O.OracleModel(draw, "fp16")
+    for ly, ld in zip(m.layers, draw.layers):
+        for w_oracle, w_drawn in zip(ly.w, ld.w):
+            want = torch.from_numpy(np.asarray(w_drawn, np.float32)).half().double().numpy()
+            assert np.array_equal(w_oracle, want)
+    assert np.array_equal(m.lm_head, np.asarray(draw.lm_head, np.float32).astype(np.float64))
+
+
 def test_sequence_order_mistake_is_caught(monkeypatch):
     sh = synth.tiny_shape(n_layers=1, n_heads=2, n_kv_heads=1, vocab=37)
     draw = synth.make_weights(sh, seed=31, std=0.08)
