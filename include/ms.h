@@ -210,12 +210,17 @@ const char* ms_last_error(void);
  * For kernel-level tests and for callers that assemble their own pipeline.  All
  * pointers are device pointers of the current device; all calls are asynchronous. */
 
-/* y[m][n] = sum_k x[m][k] * W[n][k] with W the INT4 g32 dequantised matrix
- * (W[n][k] = q[n][k] * s[n][k/32]).  x fp32 [M][K], y fp32 [M][N].  M <= 8 runs the
- * decode GEMV, larger M the prefill GEMM.  K a multiple of 256. */
+/* One backbone MatMul ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model
+ * variant: symmetric INT4 g32 weights, fp32 activations): y[m][n] = sum_k x[m][k] * W[n][k]
+ * with W[n][k] = q[n][k] * s[n][k/32].  x fp32 [M][K] and y fp32 [M][N], row-major;
+ * packed and scales as ms_quantize_int4_g32 writes them.  M in {1, 2, 4, 8} runs the
+ * decode GEMV when a CTA's slice of rows fits its shared memory; any other M runs the
+ * tcgen05 GEMM, which needs N a multiple of 64.  K a multiple of 256.  MS_ERR_INVALID_ARG
+ * for a NULL pointer, MS_ERR_SHAPE for other sizes; nothing is launched then. */
 ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, const float* scales,
                           int N, float* y, void* stream);
-/* The same with IEEE half weights w16 [N][K]. */
+/* The same with IEEE half weights w16 [N][K] (the half-precision weight variant of
+ * "MuScriptor for Core AI (.aimodel)", file table), same size rules. */
 ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y,
                            void* stream);
 /* SkipLayerNorm ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model variant):
@@ -223,9 +228,14 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
  * * gamma + beta with the biased variance, per row of d.  x, y, h fp32 [R][d]. */
 ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta,
                                float eps, int R, int d, float* h, void* stream);
-/* LM head and greedy choice: logits[m][v] = LN(x_m) . W[v] (LN skipped when gamma is
- * NULL), argmax[m] = lowest index of the largest logit.  x fp32 rows at stride ldx
- * floats, W fp32 [V][d].  M <= 64. */
+/* LM head and greedy choice ("MuScriptor small — ONNX conversion", muscriptor-small-lm.onnx:
+ * fp32 logits over the vocabulary; "MuScriptor — small (≈100M)" model card, Model
+ * description: greedy argmax): logits[m][v] = LN(x_m) . W[v] (LN skipped when gamma and
+ * beta are NULL), argmax[m] = lowest index of the largest logit.  x fp32 rows at stride
+ * ldx floats (ldx >= d, a multiple of 4), W fp32 [V][d], d a multiple of 128, 1 <= M <= 64.
+ * logits or argmax may be NULL.  The first call on a device allocates a scratch buffer
+ * (ms_op_lm_head_argmax_static does not).  MS_ERR_INVALID_ARG for a NULL x or W or for
+ * only one of gamma and beta, MS_ERR_SHAPE for other sizes. */
 ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const float* gamma,
                                const float* beta, float eps, const float* W, int V, float* logits,
                                int32_t* argmax, void* stream);
