@@ -369,7 +369,9 @@ def run_ours(a):
         e2e_ms.append(e0.elapsed_time(e1))
     h2d = prefix_h.numel() * 4 + start_h.numel() * 8
     d2h = out_h.numel() * 4 + am_h.numel() * 4
-    e2e_val = world * tokens_per_step / (statistics.mean(e2e_ms) / 1e3) if e2e_ms else None
+    # every rank ran the same e2e steps, so every rank takes part in the reduction
+    e2e_job_ms = max_over_ranks(statistics.mean(e2e_ms), dev) if e2e_ms else None
+    e2e_val = world * tokens_per_step / (e2e_job_ms / 1e3) if e2e_job_ms else None
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
