@@ -50,7 +50,23 @@ def _args():
                     help="override the workload's decode steps (short runs for profiling)")
     ap.add_argument("--cpu-decode-steps", type=int, default=256,
                     help="decode steps in the oracle's timed sample")
+    ap.add_argument("--no-batched", action="store_true",
+                    help="skip the batched-decode block (the 64-stream medium workload)")
+    ap.add_argument("--no-prefill-tensor", action="store_true",
+                    help="skip the prefill GEMM tensor-pipe block")
     return ap.parse_args()
+
+
+FALLBACK_BF16_TFLOPS = 1590.0
+# nominal dense tensor rates of a B200 (TFLOP/s): the tf32 peak is taken as the measured bf16
+# peak times this ratio
+NOMINAL_TF32_OVER_BF16 = 1.1 / 2.25
+
+# Arithmetic each path runs (the weights are INT4 codes times fp32 group scales, or halves):
+DTYPE = ("f32: fp32 activations, KV cache, LayerNorm, softmax and LM head; batch-1..8 decode "
+         "matrix products on warp MMAs with each activation as an exact fp16 hi+lo pair (22-bit "
+         "significand) and fp32 accumulation; prefill and batched-decode GEMMs 3xTF32 on tcgen05 "
+         "with fp32 accumulation")
 
 
 def _peaks():
@@ -61,6 +77,16 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def _bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def _config_json(wl: synth.Workload, world: int):
@@ -267,6 +293,120 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+# The batched-decode workload that goes with each batch-1 workload (same model and weights).
+_BATCHED = {"c3": "c4", "c5": "c5b16"}
+
+
+def _batched_block(ms, torch, model, key, dev, flush, steps=2, warmup=1):
+    """The batched half of the metric: the same model decoding many independent streams
+    (prefill all, then greedy decode), device-timed like the main line.  Its roofline is the
+    whole decode step's algorithmic bytes (weights + scales + LM head once, K and V of every
+    stream) over the measured decode time."""
+    wl = synth.WORKLOADS[key]
+    sh, B = wl.shape, wl.batch
+    stream = torch.cuda.current_stream(dev)
+    prefix = torch.from_numpy(synth.make_prefix(sh, B, wl.prefix_len, seed=1)).to(dev)
+    start = torch.from_numpy(synth.make_start_tokens(B, seed=2).reshape(B, 1)).to(dev)
+    cache = ms.Cache(model, B, wl.capacity)
+    out = torch.empty((wl.decode_steps, B), dtype=torch.int32, device=dev)
+
+    def one(ev=None):
+        cache.reset()
+        flush.zero_()
+        if ev:
+            ev[0].record(stream)
+        cache.prefill(start, prefix)
+        if ev:
+            ev[1].record(stream)
+        cache.generate(wl.decode_steps, out_tokens=out, logits=False)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    l0 = cache.kernel_launches
+    for i in range(steps):
+        one(evs[i])
+    torch.cuda.synchronize()
+    launches = cache.kernel_launches - l0
+    assert cache.device_status() == ms.MS_OK
+    pre = [e[0].elapsed_time(e[1]) for e in evs]
+    dec = [e[1].elapsed_time(e[2]) for e in evs]
+    tot = [e[0].elapsed_time(e[2]) for e in evs]
+    wbytes, kv = _decode_bytes_per_token(wl)
+    dec_bytes = wbytes * wl.decode_steps + sum(kv)
+    peak, kind = _peaks()
+    ach = dec_bytes / (statistics.mean(dec) / 1e3) / 1e9
+    path = cache.decode_path
+    cache.close()
+    return {
+        "workload": _config_json(wl, 1)["workload"],
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": statistics.mean(tot),
+        "tokens_per_s": B * (wl.decode_steps + 1) / (statistics.mean(tot) / 1e3),
+        "decode_ms_per_step": statistics.mean(dec) / wl.decode_steps,
+        "decode_tokens_per_s": B * wl.decode_steps / (statistics.mean(dec) / 1e3),
+        "prefill_ms": statistics.mean(pre),
+        "decode_path": "persistent kernel" if path == 1 else "one kernel per operation, CUDA graph per step",
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "kernel": "decode step (all kernels of one step over every stream)",
+                     "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_kind": kind,
+                     "algorithmic_bytes_per_step": dec_bytes / wl.decode_steps, "traffic": None},
+    }
+
+
+def _prefill_tensor_block(ms, torch, shape, rows_list, dev, flush, reps=5, warmup=2):
+    """Prefill GEMMs on the tensor cores: each backbone MatMul of one layer of `shape` at
+    M = prefill rows, device-timed (CUDA events around each call, L2 flushed before each),
+    through ms_op_matmul_w4 (the tcgen05 kernel with the launch policy the model uses).
+    Model arithmetic is 2 M N K per MatMul; the kernel issues three tf32 products per
+    product (3xTF32), so its tensor issue rate is three times that.  The tf32 peak is the
+    measured bf16 dense peak times the nominal tf32 / bf16 ratio (1.1 / 2.25)."""
+    bf16, kind = _bf16_peak()
+    tf32 = bf16 * NOMINAL_TF32_OVER_BF16
+    names = ["QKV", "O", "FC1", "FC2"]
+    stream = torch.cuda.current_stream(dev)
+    out = {"tf32_peak_tflops": tf32,
+           "tf32_peak_derivation": f"{kind} bf16 dense {bf16:.1f} TFLOP/s x nominal tf32/bf16 1.1/2.25",
+           "issue_products_per_model_product": 3, "cases": []}
+    g = torch.Generator(device="cpu")
+    g.manual_seed(5)
+    for M in rows_list:
+        kmax = max(k for (_, k) in shape.matmul_shapes())
+        nmax = max(n for (n, _) in shape.matmul_shapes())
+        x_all = torch.randn(M * kmax, generator=g, dtype=torch.float32).to(dev)
+        y_all = torch.empty(M * nmax, dtype=torch.float32, device=dev)
+        per, fl_tot, ms_tot = [], 0.0, 0.0
+        for name, (N, K) in zip(names, shape.matmul_shapes()):
+            w = (torch.randn(N, K, generator=g, dtype=torch.float32) * 0.02).to(dev)
+            pk, sc = ms.quantize_int4_g32(w)
+            x = x_all[: M * K].view(M, K)
+            y = y_all[: M * N].view(M, N)
+            times = []
+            for i in range(warmup + reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                ms.matmul_w4(x, pk, sc, out=y)
+                e1.record(stream)
+                e1.synchronize()
+                if i >= warmup:
+                    times.append(e0.elapsed_time(e1))
+            t = statistics.median(times)
+            fl = 2.0 * M * N * K
+            per.append({"matmul": name, "N": N, "K": K, "ms": t, "model_tflops": fl / t / 1e9})
+            fl_tot += fl
+            ms_tot += t
+            del w, pk, sc
+        model = fl_tot / ms_tot / 1e9
+        out["cases"].append({"M": M, "matmuls": per, "layer_ms": ms_tot, "model_tflops": model,
+                             "issue_tflops": 3 * model, "frac_of_tf32_peak": 3 * model / tf32})
+        del x_all, y_all
+    return out
+
+
 def run_ours(a):
     import torch
     import torch.distributed as dist
@@ -394,13 +534,21 @@ def run_ours(a):
         roof["traffic"] = tr["bytes"]
         roof["traffic_per"] = f"one launch of {tr['tokens']} decode steps, cache lengths {t_lo}..{t_hi} (ncu)"
         roof["traffic_over_algorithmic"] = tr["bytes"] / alg
+    batched = prefill_tc = None
+    if world == 1 and not a.no_batched and a.workload in _BATCHED:
+        batched = _batched_block(ms, torch, model, _BATCHED[a.workload], dev, flush)
+    if world == 1 and not a.no_prefill_tensor:
+        rows = [wl.prefix_len + 1]
+        if a.workload in _BATCHED:
+            rows.append(synth.WORKLOADS[_BATCHED[a.workload]].batch * (wl.prefix_len + 1))
+        prefill_tc = _prefill_tensor_block(ms, torch, sh, rows, dev, flush)
     if world > 1:
         dist.barrier()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": total_ms / a.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config_json(wl, world),
+            "vs_baseline": None, "dtype": DTYPE, "data": "synthetic", "config": _config_json(wl, world),
             "prefill_ms": {"mean": statistics.mean(pre_ms), "median": statistics.median(pre_ms)},
             "decode_ms_per_token": {"mean": statistics.mean(per_tok), "median": statistics.median(per_tok),
                                     "p90": float(np.percentile(per_tok, 90))},
@@ -413,6 +561,10 @@ def run_ours(a):
         }
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if batched is not None:
+            line["batched"] = batched
+        if prefill_tc is not None:
+            line["prefill_tensor"] = prefill_tc
         print(json.dumps(line), flush=True)
     cache.close()
     model.close()

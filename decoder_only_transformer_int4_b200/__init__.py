@@ -147,10 +147,11 @@ def quantize_int4_g32(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
     return packed, scales
 
 
-def matmul_w4(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+def matmul_w4(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
     m, k = x.shape
     n = packed.shape[0]
-    y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    y = torch.empty((m, n), dtype=torch.float32, device=x.device) if out is None else out
     _check(_lib.ms_op_matmul_w4(_ptr(x), m, k, _ptr(packed), _ptr(scales), n, _ptr(y), _stream()), "ms_op_matmul_w4")
     return y
 

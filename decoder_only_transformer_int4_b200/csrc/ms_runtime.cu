@@ -908,7 +908,13 @@ ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, c
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
   if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: N must be a multiple of 64 for this M");
-  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore), "gemm");
+  // the launch policy the model's own calls use (K split over a cluster when the tiles
+  // alone would leave SMs idle)
+  int dev = 0, nsm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  const ms::GemmWork gw{nsm > 0 ? nsm : 1};
+  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore, &gw), "gemm");
 }
 
 ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y, void* stream) {
@@ -920,7 +926,13 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
   if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: N must be a multiple of 64 for this M");
-  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore), "gemm");
+  // the launch policy the model's own calls use (K split over a cluster when the tiles
+  // alone would leave SMs idle)
+  int dev = 0, nsm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  const ms::GemmWork gw{nsm > 0 ? nsm : 1};
+  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore, &gw), "gemm");
 }
 
 ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta, float eps, int R, int d,

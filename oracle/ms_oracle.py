@@ -452,6 +452,17 @@ class OracleCache:
         self.k = [np.zeros((capacity, n_kv_heads, head_dim)) for _ in range(n_layers)]
         self.v = [np.zeros((capacity, n_kv_heads, head_dim)) for _ in range(n_layers)]
 
+    def load(self, k: np.ndarray, v: np.ndarray):
+        """Set the cache to T given positions of one stream, k and v [L, T, Hk, 64] (the
+        pages' past_k / past_v layout without the batch axis); the length becomes T."""
+        t = k.shape[1]
+        if t > self.capacity:
+            raise ValueError("cache capacity exceeded")
+        for l in range(len(self.k)):
+            self.k[l][:t] = k[l]
+            self.v[l][:t] = v[l]
+        self.length = t
+
     def export(self):
         """The pages' cache layout [L, 1, T, Hk, 64] ([ONNX-S] past_k / past_v)."""
         t = self.length

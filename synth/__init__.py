@@ -180,3 +180,19 @@ def make_matrix(n: int, k: int, seed: int, std: float = 0.02) -> np.ndarray:
 def make_activations(m: int, k: int, seed: int, std: float = 1.0) -> np.ndarray:
     """fp32 [m, k] N(0, std) activations (kernel-level tests)."""
     return _normal(_gen(seed), (m, k), std)
+
+
+def make_kv_cache(shape: Shape, batch: int, T: int, seed: int = 4, std: float = 1.0):
+    """A cache state of T positions for resuming decode late in a run, in the pages' layout
+    (past_k / past_v [L, B, T, Hk, 64]): keys and values N(0, std) fp32, drawn layer by layer
+    (all of layer l's keys, then its values).  Any contents are a valid state for the decoder
+    step (it reads the cache, it does not check how the cache was made), so parity tests
+    import the same draws into both sides."""
+    g = _gen(seed)
+    sz = (batch, T, shape.n_kv_heads, shape.head_dim)
+    k = np.empty((shape.n_layers,) + sz, np.float32)
+    v = np.empty_like(k)
+    for l in range(shape.n_layers):
+        k[l] = torch.randn(*sz, generator=g, dtype=torch.float32).numpy() * std
+        v[l] = torch.randn(*sz, generator=g, dtype=torch.float32).numpy() * std
+    return k, v

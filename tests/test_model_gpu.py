@@ -340,12 +340,61 @@ def test_full_c3_medium_gqa():
     assert tok.shape == (1, 2001)
 
 
+def _full_check(key, n, streams):
+    """A benchmark workload at full size, checked on the given streams with one oracle run
+    each: the oracle's greedy run (prefill + n steps) gives both the tokens the GPU is
+    teacher-forced on (logits compared at every step) and the tokens the GPU's own greedy
+    run over the workload's whole decode length must reproduce under the margin rule.  The
+    other streams are teacher-forced on a seeded sequence."""
+    wl = synth.WORKLOADS[key]
+    sh, B = wl.shape, wl.batch
+    _, om, gm = _build(sh, fmt=wl.weight_format)
+    prefix = synth.make_prefix(sh, B, seed=1)
+    start = synth.make_start_tokens(B, seed=2)
+    forced = synth.make_token_sequence(n, B, seed=3)
+    ref = {}
+    for b in streams:
+        t, lg = om.greedy(prefix[b], int(start[b]), n, capacity=wl.capacity)
+        ref[b] = (t, lg)
+        forced[b] = t[:n]
+    got, _ = _run_teacher_forced(gm, B, wl.capacity, prefix, forced, start)
+    for b in streams:
+        err = np.abs(got[:, b] - ref[b][1]).max()
+        assert err <= TOL, (key, b, err)
+    cache = ms.Cache(gm, B, wl.capacity)
+    _, am = cache.prefill(_dev(start.reshape(B, 1)), _dev(prefix))
+    toks, _ = cache.generate(wl.decode_steps)
+    assert cache.device_status() == ms.MS_OK
+    gpu_tok = np.concatenate([am.cpu().numpy()[None], toks.cpu().numpy()], 0).T
+    assert gpu_tok.shape == (B, wl.decode_steps + 1)
+    for b in streams:
+        _greedy_agree(gpu_tok[b, : n + 1], ref[b][0], ref[b][1])
+    return cache.decode_path
+
+
 @pytest.mark.slow
 def test_full_c4_medium_64_streams():
     # 64 independent streams through the batched path (tcgen05 GEMMs, split-K attention);
-    # streams 0 and 1 are checked against the oracle.
-    tok = _full_config("c4", 16, 16)
-    assert tok.shape == (64, 513)
+    # eight streams spread over the batch are checked against the oracle.
+    assert _full_check("c4", 16, [0, 9, 18, 27, 36, 45, 54, 63]) == 2
+
+
+@pytest.mark.slow
+def test_full_c5_large_16_streams():
+    assert _full_check("c5b16", 8, [0, 7, 15]) == 2
+
+
+@pytest.mark.slow
+def test_full_c5_large_fp16():
+    # "MuScriptor for Core AI (.aimodel)", file table: the large model with its weights cast
+    # to half; fp32 accumulation, persistent decode kernel
+    assert _full_check("c5fp16", 8, [0]) == 1
+
+
+@pytest.mark.slow
+def test_full_c3pages_medium_mha():
+    # kv heads = heads = 16 (the 469.5 MiB cache at 2504 positions of the W4A32 page)
+    assert _full_check("c3pages", 24, [0]) == 1
 
 
 @pytest.mark.slow

@@ -455,6 +455,49 @@ def test_greedy_feeds_argmax_back():
     assert O.argmax_lowest(tie) == 1
 
 
+def _top2_margin_mismatches(fn):
+    """The checks top2_margin must pass (it decides where the greedy comparisons stop):
+    a hand-worked batch of rows, ties, a single row, and a brute-force scan on random rows.
+    Returns the names of the checks that fail."""
+    bad = []
+    # rows: max 3.5 over 3.0; a tie at the top (margin 0); max 5 over a tied 4.25
+    hand = np.array([[1.0, 3.5, 2.0, 3.0], [0.0, -1.0, -1.0, 0.0], [5.0, 4.25, -3.0, 4.25]])
+    try:
+        if not np.array_equal(np.asarray(fn(hand)), np.array([0.5, 0.0, 0.75])):
+            bad.append("hand rows")
+        if float(fn(np.array([2.0, -7.0, 1.5]))) != 0.5:
+            bad.append("single row")
+        rng = np.random.default_rng(7)
+        x = rng.standard_normal((5, 11))
+        want = []
+        for row in x:
+            i = max(range(len(row)), key=lambda j: row[j])
+            second = max(row[j] for j in range(len(row)) if j != i)
+            want.append(row[i] - second)
+        if not np.allclose(np.asarray(fn(x)), want, rtol=0, atol=0):
+            bad.append("brute force")
+    except Exception:            # a planted mistake may not even run
+        bad.append("raised")
+    return bad
+
+
+def test_top2_margin_pins():
+    assert _top2_margin_mismatches(O.top2_margin) == []
+
+
+def test_top2_margin_wrong_axis_is_caught():
+    def wrong_axis(logits):
+        part = np.sort(np.asarray(logits, np.float64), axis=0)
+        return part[..., -1] - part[..., -2]
+
+    def abs_gap_of_ends(logits):
+        part = np.sort(np.asarray(logits, np.float64), axis=-1)
+        return part[..., -1] - part[..., 0]
+
+    assert _top2_margin_mismatches(wrong_axis)
+    assert _top2_margin_mismatches(abs_gap_of_ends)
+
+
 # ----------------------------------------------------------------------------
 # Planted mistakes: each must be caught by at least one pin above
 # ----------------------------------------------------------------------------
