@@ -469,7 +469,9 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
       bidx[warp * M + m] = bi[m];
     }
   }
-  __syncthreads();
+  // a CTA whose weight rows never arrived marks its result with index -1, so the failure
+  // reaches the argmax even when the caller passed no status word
+  const int cta_failed = __syncthreads_or(!ok);
   if (tid < M) {
     float bv = -FLT_MAX;
     int bx = INT_MAX;
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
         bx = bidx[w * M + tid];
       }
     a.part_val[(size_t)blockIdx.x * 64 + a.m_base + tid] = bv;
-    a.part_idx[(size_t)blockIdx.x * 64 + a.m_base + tid] = bx;
+    a.part_idx[(size_t)blockIdx.x * 64 + a.m_base + tid] = cta_failed ? -1 : bx;
   }
   __threadfence();
   __syncthreads();
@@ -489,6 +491,7 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
   __threadfence();
   const int len = a.dlen ? *reinterpret_cast<volatile int*>(a.dlen) : 0;
   // every thread takes a share of the per-CTA results, then a block argmax
+  bool any_failed = false;
   for (int m = 0; m < M; ++m) {
     const int mg = a.m_base + m;
     float bv = -FLT_MAX;
@@ -496,7 +499,8 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
     for (int c = tid; c < (int)gridDim.x; c += kLmThreads) {
       const float v = __ldcg(a.part_val + (size_t)c * 64 + mg);
       const int i = __ldcg(a.part_idx + (size_t)c * 64 + mg);
-      if (argmax_better(v, i, bv, bx)) {
+      if (i < 0) any_failed = true;
+      else if (argmax_better(v, i, bv, bx)) {
         bv = v;
         bx = i;
       }
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
       bidx[warp * M + m] = bx;
     }
   }
-  __syncthreads();
+  const int failed = __syncthreads_or(any_failed);
   if (tid < M) {
     const int mg = a.m_base + tid;
     float bv = -FLT_MAX;
@@ -518,6 +522,7 @@ __global__ void __launch_bounds__(kLmThreads) lm_head_kernel(LmArgs a) {
         bx = bidx[w * M + tid];
       }
     if (bx == INT_MAX) bx = 0;
+    if (failed) bx = -1;   // some CTA's weight rows never arrived: no valid choice
     if (a.argmax) a.argmax[mg] = bx;
     if (a.hist) a.hist[(size_t)(len + a.hist_off) * a.hist_B + mg] = bx;
   }

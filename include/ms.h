@@ -235,7 +235,9 @@ ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, con
  * ldx floats (ldx >= d, a multiple of 4), W fp32 [V][d], d a multiple of 128, 1 <= M <= 64.
  * logits or argmax may be NULL.  The first call on a device allocates a scratch buffer
  * (ms_op_lm_head_argmax_static does not).  MS_ERR_INVALID_ARG for a NULL x or W or for
- * only one of gamma and beta, MS_ERR_SHAPE for other sizes. */
+ * only one of gamma and beta, MS_ERR_SHAPE for other sizes.  The call is asynchronous, so
+ * a device-side failure cannot change its return value: if the kernel's bounded wait for
+ * its weight rows ran out, argmax[m] is -1 for every row (and those logits are unwritten). */
 ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const float* gamma,
                                const float* beta, float eps, const float* W, int V, float* logits,
                                int32_t* argmax, void* stream);
@@ -256,7 +258,8 @@ ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const floa
  * capture.  Every call shares the one array and keeps the last call's contents; the
  * counter that must start at zero is cleared on the stream before each launch.  Calls
  * that overlap on the GPU (different streams, or different host threads) race on the
- * array: order them on one stream.  It calls no cudaMalloc or cudaFree. */
+ * array: order them on one stream.  It calls no cudaMalloc or cudaFree.  A wait that ran
+ * out on the device shows as argmax -1, as for ms_op_lm_head_argmax. */
 ms_status ms_op_lm_head_argmax_static(const float* x, int ldx, int M, int d, const float* gamma,
                                       const float* beta, float eps, const float* W, int V,
                                       float* logits, int32_t* argmax, void* stream);

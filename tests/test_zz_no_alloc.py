@@ -4,11 +4,13 @@ Some callers cannot allocate device memory at the point where they need the LM h
 code running while a stream is captured into a CUDA graph, code whose device memory
 belongs to another allocator, latency-critical loops where an allocation could
 synchronise the device.  This entry point serves them from a fixed scratch array inside
-the library.  The test calls it through the C ABI twice in a row (the array keeps the
-previous call's contents, so the second call checks that nothing stale leaks through) and
-compares each result with the allocating entry point's on the same inputs, within the
-fp32 dot-product bound the kernel tests use.  It lives in its own file, collected last,
-and works both alone in a fresh process and after the other tests.
+the library.  The test calls it through the C ABI three times in a row and compares each result
+with the allocating entry point's on the same inputs, within the fp32 dot-product bound the
+kernel tests use.  The array keeps the previous call's contents: the second call has a
+smaller vocabulary, so it launches fewer CTAs than the first and the first call's extra
+per-CTA slots stay behind in the array (the result must not pick them up); a third call
+follows a call the library rejected, on the same stream.  It lives in its own file,
+collected last, and works both alone in a fresh process and after the other tests.
 """
 import numpy as np
 import pytest
@@ -27,13 +29,27 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def test_static_lm_head_matches_the_allocating_entry_point_on_two_calls():
-    d, V = 1024, 1393
-    W = synth.make_matrix(V, d, seed=1801)
+def _rejected_call():
+    x = torch.zeros((65, 256), dtype=torch.float32, device="cuda")
+    W = torch.zeros((50, 256), dtype=torch.float32, device="cuda")
+    st = ms._lib.ms_op_lm_head_argmax_static(ms._ptr(x), 256, 65, 256, None, None, 1e-5, ms._ptr(W), 50, None, None,
+                                             ms._stream())
+    assert st == ms.MS_ERR_SHAPE
+
+
+def test_static_lm_head_matches_the_allocating_entry_point_on_calls_in_a_row():
+    d = 1024
+    W_all = synth.make_matrix(1393, d, seed=1801)
     g = 1 + 0.1 * synth.make_activations(1, d, seed=1802)[0]
     b = 0.1 * synth.make_activations(1, d, seed=1803)[0]
-    Wd, gd, bd = _dev(W), _dev(g), _dev(b)
-    for call, M in enumerate((3, 8)):
+    gd, bd = _dev(g), _dev(b)
+    # the vocabulary shrinks from call to call (fewer CTAs, stale slots left behind); the
+    # third call comes right after a rejected call
+    for call, (M, V) in enumerate(((3, 1393), (8, 300), (5, 97))):
+        if call == 2:
+            _rejected_call()
+        W = W_all[:V]
+        Wd = _dev(W)
         x = synth.make_activations(M, d, seed=1810 + call)
         xd = _dev(x)
         ref_lg, ref_am = ms.lm_head_argmax(xd, Wd, gd, bd, 1e-5)
