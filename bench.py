@@ -58,15 +58,11 @@ def _args():
 
 
 FALLBACK_BF16_TFLOPS = 1590.0
-# nominal dense tensor rates of a B200 (TFLOP/s): the tf32 peak is taken as the measured bf16
-# peak times this ratio
-NOMINAL_TF32_OVER_BF16 = 1.1 / 2.25
-
 # Arithmetic each path runs (the weights are INT4 codes times fp32 group scales, or halves):
 DTYPE = ("f32: fp32 activations, KV cache, LayerNorm, softmax and LM head; batch-1..8 decode "
          "matrix products on warp MMAs with each activation as an exact fp16 hi+lo pair (22-bit "
-         "significand) and fp32 accumulation; prefill and batched-decode GEMMs 3xTF32 on tcgen05 "
-         "with fp32 accumulation")
+         "significand) and fp32 accumulation; prefill and batched-decode GEMMs on tcgen05 kind::f16 "
+         "with both operands as fp16 hi+lo pairs (three products) and fp32 accumulation")
 
 
 def _peaks():
@@ -357,53 +353,48 @@ def _batched_block(ms, torch, model, key, dev, flush, steps=2, warmup=1):
     }
 
 
-def _prefill_tensor_block(ms, torch, shape, rows_list, dev, flush, reps=5, warmup=2):
-    """Prefill GEMMs on the tensor cores: each backbone MatMul of one layer of `shape` at
-    M = prefill rows, device-timed (CUDA events around each call, L2 flushed before each),
-    through ms_op_matmul_w4 (the tcgen05 kernel with the launch policy the model uses).
-    Model arithmetic is 2 M N K per MatMul; the kernel issues three tf32 products per
-    product (3xTF32), so its tensor issue rate is three times that.  The tf32 peak is the
-    measured bf16 dense peak times the nominal tf32 / bf16 ratio (1.1 / 2.25)."""
+def _prefill_tensor_block(ms, torch, model, shape, rows_list, dev, flush, reps=5, warmup=2):
+    """Prefill GEMMs on the tensor cores: each backbone MatMul of layer 0 of the benchmark's
+    model at M = prefill rows, through ms_model_matmul (the tcgen05 GEMM prefill runs, on the
+    model's own tile-packed INT4 weights, from activation planes split beforehand),
+    device-timed (CUDA events around each call, L2 flushed before each).  Model arithmetic is
+    2 M N K per MatMul; the kernel issues three fp16 products per product (hi*hi, hi*lo,
+    lo*hi), so its tensor issue rate is three times that, against the measured bf16 dense
+    peak (fp16 and bf16 share the dense rate)."""
     bf16, kind = _bf16_peak()
-    tf32 = bf16 * NOMINAL_TF32_OVER_BF16
     names = ["QKV", "O", "FC1", "FC2"]
     stream = torch.cuda.current_stream(dev)
-    out = {"tf32_peak_tflops": tf32,
-           "tf32_peak_derivation": f"{kind} bf16 dense {bf16:.1f} TFLOP/s x nominal tf32/bf16 1.1/2.25",
+    out = {"f16_peak_tflops": bf16, "f16_peak_derivation": f"{kind} bf16 dense {bf16:.1f} TFLOP/s (fp16 dense rate = bf16)",
            "issue_products_per_model_product": 3, "cases": []}
     g = torch.Generator(device="cpu")
     g.manual_seed(5)
     for M in rows_list:
-        kmax = max(k for (_, k) in shape.matmul_shapes())
-        nmax = max(n for (n, _) in shape.matmul_shapes())
-        x_all = torch.randn(M * kmax, generator=g, dtype=torch.float32).to(dev)
-        y_all = torch.empty(M * nmax, dtype=torch.float32, device=dev)
         per, fl_tot, ms_tot = [], 0.0, 0.0
-        for name, (N, K) in zip(names, shape.matmul_shapes()):
-            w = (torch.randn(N, K, generator=g, dtype=torch.float32) * 0.02).to(dev)
-            pk, sc = ms.quantize_int4_g32(w)
-            x = x_all[: M * K].view(M, K)
-            y = y_all[: M * N].view(M, N)
+        for i, (name, (N, K)) in enumerate(zip(names, shape.matmul_shapes())):
+            x = torch.randn(M, K, generator=g, dtype=torch.float32).to(dev)
+            hi, lo = ms.split_f16(x)
+            del x
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
             times = []
-            for i in range(warmup + reps):
+            for it in range(warmup + reps):
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                ms.matmul_w4(x, pk, sc, out=y)
+                model.matmul(0, i, hi, lo, out=y)
                 e1.record(stream)
                 e1.synchronize()
-                if i >= warmup:
+                if it >= warmup:
                     times.append(e0.elapsed_time(e1))
             t = statistics.median(times)
             fl = 2.0 * M * N * K
-            per.append({"matmul": name, "N": N, "K": K, "ms": t, "model_tflops": fl / t / 1e9})
+            per.append({"matmul": name, "N": N, "K": K, "ms": t, "model_tflops": fl / t / 1e9,
+                        "issue_tflops": 3 * fl / t / 1e9})
             fl_tot += fl
             ms_tot += t
-            del w, pk, sc
-        model = fl_tot / ms_tot / 1e9
-        out["cases"].append({"M": M, "matmuls": per, "layer_ms": ms_tot, "model_tflops": model,
-                             "issue_tflops": 3 * model, "frac_of_tf32_peak": 3 * model / tf32})
-        del x_all, y_all
+            del hi, lo, y
+        model_tf = fl_tot / ms_tot / 1e9
+        out["cases"].append({"M": M, "matmuls": per, "layer_ms": ms_tot, "model_tflops": model_tf,
+                             "issue_tflops": 3 * model_tf, "frac_of_f16_peak": 3 * model_tf / bf16})
     return out
 
 
@@ -541,7 +532,7 @@ def run_ours(a):
         rows = [wl.prefix_len + 1]
         if a.workload in _BATCHED:
             rows.append(synth.WORKLOADS[_BATCHED[a.workload]].batch * (wl.prefix_len + 1))
-        prefill_tc = _prefill_tensor_block(ms, torch, sh, rows, dev, flush)
+        prefill_tc = _prefill_tensor_block(ms, torch, model, sh, rows, dev, flush)
     if world > 1:
         dist.barrier()
     if rank == 0:

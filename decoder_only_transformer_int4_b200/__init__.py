@@ -87,6 +87,8 @@ _PROTOS = {
     "ms_op_matmul_w4": (_I, [_P, _I, _I, _P, _P, _I, _P, _P]),
     "ms_op_matmul_f16": (_I, [_P, _I, _I, _P, _I, _P, _P]),
     "ms_op_skip_layernorm": (_I, [_P, _P, _P, _P, _F, _I, _I, _P, _P]),
+    "ms_op_split_f16": (_I, [_P, _I, _I, _I, _P, _P, _I, _P]),
+    "ms_model_matmul": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _P]),
     "ms_op_lm_head_argmax": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
     "ms_op_lm_head_argmax_static": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
 }
@@ -162,6 +164,16 @@ def matmul_f16(x: torch.Tensor, w16: torch.Tensor) -> torch.Tensor:
     y = torch.empty((m, n), dtype=torch.float32, device=x.device)
     _check(_lib.ms_op_matmul_f16(_ptr(x), m, k, _ptr(w16), n, _ptr(y), _stream()), "ms_op_matmul_f16")
     return y
+
+
+def split_f16(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """fp32 [M, K] -> (hi, lo) fp16 [M, K] with hi + lo carrying x to a 22-bit significand
+    (the tcgen05 GEMM's operand form)."""
+    m, k = x.shape
+    hi = torch.empty((m, k), dtype=torch.float16, device=x.device)
+    lo = torch.empty((m, k), dtype=torch.float16, device=x.device)
+    _check(_lib.ms_op_split_f16(_ptr(x), k, m, k, _ptr(hi), _ptr(lo), k, _stream()), "ms_op_split_f16")
+    return hi, lo
 
 
 def skip_layernorm(x: torch.Tensor, y: Optional[torch.Tensor], gamma: torch.Tensor, beta: torch.Tensor,
@@ -249,6 +261,18 @@ class Model:
         W = Weights(up(draw.tok_emb), up(draw.lm_head), up(draw.ln_f_g), up(draw.ln_f_b), layers)
         torch.cuda.current_stream(dev).synchronize()
         return cls(cfg, W, device, _keep=keep)
+
+    def matmul(self, layer: int, which: int, x_hi: torch.Tensor, x_lo: torch.Tensor,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Backbone MatMul `which` (0 QKV, 1 O, 2 FC1, 3 FC2) of `layer` on split activation
+        planes [M, K] (see split_f16) -> fp32 [M, N] (ms_model_matmul)."""
+        m, k = x_hi.shape
+        c = self.cfg
+        n = [(c.n_heads + 2 * c.n_kv_heads) * 64, c.d_model, c.d_ff, c.d_model][which]
+        y = torch.empty((m, n), dtype=torch.float32, device=x_hi.device) if out is None else out
+        _check(_lib.ms_model_matmul(self._h, layer, which, _ptr(x_hi), _ptr(x_lo), k, m, _ptr(y), n, _stream()),
+               "ms_model_matmul")
+        return y
 
     @property
     def weight_bytes(self) -> int:

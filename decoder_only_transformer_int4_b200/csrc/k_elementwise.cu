@@ -121,7 +121,9 @@ cudaError_t launch_embed_decode(const Launch& L, const int32_t* tokens, const in
 template <int NVMAX>
 __global__ void __launch_bounds__(256) skipln_kernel(float* __restrict__ x, const float* __restrict__ y,
                                                      const float* __restrict__ g, const float* __restrict__ bta,
-                                                     float eps, int R, int d, float* __restrict__ h) {
+                                                     float eps, int R, int d, float* __restrict__ h,
+                                                     __half* __restrict__ hh, __half* __restrict__ hl, int ldh,
+                                                     unsigned* status) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -161,7 +163,8 @@ __global__ void __launch_bounds__(256) skipln_kernel(float* __restrict__ x, cons
   const float rstd = 1.0f / sqrtf(var + eps);
   const float4* g4 = reinterpret_cast<const float4*>(g);
   const float4* b4 = reinterpret_cast<const float4*>(bta);
-  float4* hr = reinterpret_cast<float4*>(h + (size_t)row * d);
+  float4* hr = h ? reinterpret_cast<float4*>(h + (size_t)row * d) : nullptr;
+  bool big = false;
 #pragma unroll
   for (int j = 0; j < NVMAX; ++j) {
     if (j < nv) {
@@ -172,16 +175,31 @@ __global__ void __launch_bounds__(256) skipln_kernel(float* __restrict__ x, cons
       o.y = (v[j].y - mean) * rstd * gg.y + bb.y;
       o.z = (v[j].z - mean) * rstd * gg.z + bb.z;
       o.w = (v[j].w - mean) * rstd * gg.w + bb.w;
-      hr[f] = o;
+      if (hr) hr[f] = o;
+      if (hh) {
+        // fp16 hi / lo planes: hi = fp16(v), lo = fp16(v - hi)
+        const __half2 h0 = __floats2half2_rn(o.x, o.y), h1 = __floats2half2_rn(o.z, o.w);
+        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+        const __half2 l0 = __floats2half2_rn(o.x - f0.x, o.y - f0.y), l1 = __floats2half2_rn(o.z - f1.x, o.w - f1.y);
+        big |= fabsf(o.x) >= 65504.f || fabsf(o.y) >= 65504.f || fabsf(o.z) >= 65504.f || fabsf(o.w) >= 65504.f;
+        __half2* ph = reinterpret_cast<__half2*>(hh + (size_t)row * ldh + 4 * f);
+        __half2* pl = reinterpret_cast<__half2*>(hl + (size_t)row * ldh + 4 * f);
+        ph[0] = h0;
+        ph[1] = h1;
+        pl[0] = l0;
+        pl[1] = l1;
+      }
     }
   }
+  if (big) flag_error(status, kErrShape);
 }
 
 cudaError_t launch_skipln(const Launch& L, float* x, const float* y, const float* g, const float* b, float eps,
-                          int R, int d, float* h) {
+                          int R, int d, float* h, __half* hh, __half* hl, int ldh) {
   if (R <= 0) return cudaSuccess;
   if (d % 128 != 0 || d > 16 * 128) return cudaErrorInvalidValue;
-  return launch_k(L, skipln_kernel<16>, dim3((R + 7) / 8), dim3(256), 0, x, y, g, b, eps, R, d, h);
+  return launch_k(L, skipln_kernel<16>, dim3((R + 7) / 8), dim3(256), 0, x, y, g, b, eps, R, d, h, hh, hl, ldh,
+                  L.status);
 }
 
 // ---------------------------------------------------------------------------------

@@ -1,5 +1,6 @@
 // Host-side launchers of the decoder kernels (internal to the library).
 #pragma once
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,7 +46,6 @@ void set_last_error(const char* msg);
 // Opt every kernel that needs it into large dynamic shared memory on the current device.
 cudaError_t init_attrs_gemv();
 cudaError_t init_attrs_attn();
-cudaError_t init_attrs_gemm_tc();
 
 cudaError_t launch_quantize_int4(const float* w, int N, int K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
@@ -58,9 +58,12 @@ cudaError_t launch_embed_prefill(const Launch& L, const int64_t* tokens, int S, 
 cudaError_t launch_embed_decode(const Launch& L, const int32_t* tokens, const int32_t* hist,
                                 const int* dlen, const float* tok_emb, int V, int d, int B, float* x);
 
-// x <- x + y (y may be null), h = LN(x) * g + b, per row.
+// x <- x + y (y may be null), h = LN(x) * g + b, per row.  h (fp32 [R][d]) may be null;
+// with hh, the result is also written as fp16 hi / lo planes hh, hl [R][ldh] (the tcgen05
+// GEMM's operand form).
 cudaError_t launch_skipln(const Launch& L, float* x, const float* y, const float* g, const float* b,
-                          float eps, int R, int d, float* h);
+                          float eps, int R, int d, float* h, __half* hh = nullptr, __half* hl = nullptr,
+                          int ldh = 0);
 
 // RoPE on the q and k parts of qkv rows (row r = b * n + i at position len + i, len read
 // from dlen) and append post-RoPE k and v to the layer's cache slices.
@@ -73,14 +76,33 @@ cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx
                         const float* ln_g, const float* ln_b, float eps, float* y, int ldy, int epi);
 bool gemv_fits(const WView& w, int M);
 
-// General-M path on the tensor cores (tcgen05, 3xTF32): prefill and batched decode.  With
-// gw, K is split over a cluster of CTAs per output tile when the tiles alone would leave SMs
-// idle.
+// Launch policy of the tcgen05 GEMM: with gw, K is split over a cluster of CTAs per output
+// tile when the tiles alone would leave SMs idle.
 struct GemmWork {
   int sms;             // SMs of the device
 };
-cudaError_t launch_gemm_tc(const Launch& L, const WView& w, const float* x, int ldx, int M, float* y,
-                           int ldy, int epi, const GemmWork* gw = nullptr);
+
+// The warp-specialised tcgen05 GEMM on fp16 hi / lo operand planes (kind::f16, three
+// products).  INT4 weights come from a tile-packed copy made once (launch_gemm_repack): per
+// 128-row tile and 64-wide K stage, 128 x 32 bytes of codes then 128 x 2 scales, the scales
+// of row n multiplied by 2^e_n, with rinv[n] = 2^-e_n; half weights are read in place.
+struct GemmWeights {
+  const unsigned char* wt;   // INT4 tile-packed blocks, gemm_tiles_bytes(w) bytes
+  const float* rinv;         // [gemm_rows_padded(w)]
+};
+size_t gemm_tiles_bytes(const WView& w);
+size_t gemm_rows_padded(const WView& w);
+// rexp_scratch: gemm_rows_padded(w) floats of device memory.
+cudaError_t launch_gemm_repack(const WView& w, GemmWeights& g, float* rexp_scratch, cudaStream_t s);
+// y (fp32 [M][ldy], store / add / GELU) and / or yh, yl (fp16 planes [M][ldyh] of the result)
+// from activation planes xh, xl [M][ldx] (ldx a multiple of 8, 16-byte aligned).
+cudaError_t launch_gemm_f16(const Launch& L, const WView& w, const GemmWeights& g, const __half* xh,
+                            const __half* xl, int ldx, int M, float* y, int ldy, __half* yh, __half* yl,
+                            int ldyh, int epi, const GemmWork* gw);
+// fp32 rows [M][ldx] -> planes xh, xl [M][ldh] (|v| >= 65504 flags kErrShapeBit).
+cudaError_t launch_split_f16(const Launch& L, const float* x, int ldx, int M, int K, __half* xh, __half* xl,
+                             int ldh);
+cudaError_t init_attrs_gemm_f16();
 
 // Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
 // the combine done by the last CTA of each (stream, kv head).

@@ -6,6 +6,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 #include <new>
@@ -82,6 +83,7 @@ struct DevLayer {
   float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
   ms::WView w[4];
   uint8_t* wt[4];  // tile-packed copies for the persistent decode kernel
+  ms::GemmWeights gw[4];  // tile-packed INT4 copies for the tcgen05 GEMM (prefill, batched decode)
 };
 
 bool shape_ok(const ms_config* c, std::string* why) {
@@ -141,7 +143,7 @@ cudaError_t ensure_kernel_attributes() {
   e = ms::init_attrs_gemv();
   if (e == cudaSuccess) e = ms::init_attrs_attn();
   if (e == cudaSuccess) e = ms::init_attrs_persistent();
-  if (e == cudaSuccess) e = ms::init_attrs_gemm_tc();
+  if (e == cudaSuccess) e = ms::init_attrs_gemm_f16();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -159,6 +161,7 @@ struct ms_model {
   float *tok_emb = nullptr, *lm_head = nullptr, *ln_f_g = nullptr, *ln_f_b = nullptr;
   std::vector<DevLayer> layers;
   ms::PLayer* d_players = nullptr;  // the same pointers, on the device, for the persistent kernel
+  float* rexp = nullptr;             // per-row powers of two while the GEMM copies are made
 };
 
 struct ms_cache {
@@ -178,6 +181,9 @@ struct ms_cache {
   int* lm_idx = nullptr;
   unsigned* lm_counter = nullptr;
   float *x = nullptr, *h = nullptr, *y = nullptr, *qkv = nullptr, *q = nullptr, *o = nullptr, *u = nullptr;
+  __half *hh = nullptr, *hl = nullptr;     // GEMM operand planes [rows][kh] (LayerNorm or attention output)
+  __half *uh = nullptr, *ul = nullptr;     // FC1's GELU output as planes [rows][d_ff] (they share u's memory)
+  int kh = 0;                              // row stride of hh / hl: max(d, H * 64)
   float* logits = nullptr;                 // [B][V] internal
   size_t rows_cap = 0;
   cudaGraphExec_t gen_exec = nullptr;
@@ -218,18 +224,29 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
   const int nq = (H + 2 * Hk) * 64;
   ms::Launch L0 = launch_of(c, st, false), L = launch_of(c, st, true);
   cudaError_t e = ms::launch_embed_prefill(L0, tokens, S, prefix, P, m->tok_emb, g.vocab, d, B, c->x);
+  const int kh = c->kh, F = g.d_ff;
   for (int l = 0; l < g.n_layers && e == cudaSuccess; ++l) {
     const DevLayer& ly = m->layers[l];
     float* kc = c->k + l * layer_stride(c);
     float* vc = c->v + l * layer_stride(c);
-    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore, &gw);
+    // LN1 -> planes -> QKV -> RoPE + append -> attention -> planes -> O -> SkipLN2 -> planes
+    // -> FC1 + GELU -> planes -> FC2
+    if (e == cudaSuccess)
+      e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, nullptr, c->hh, c->hl,
+                            kh);
+    if (e == cudaSuccess)
+      e = ms::launch_gemm_f16(L, ly.w[0], ly.gw[0], c->hh, c->hl, kh, R, c->qkv, nq, nullptr, nullptr, 0, ms::kStore, &gw);
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore, &gw);
-    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, R, c->u, g.d_ff, ms::kGelu, &gw);
-    if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, g.d_ff, R, c->y, d, ms::kStore, &gw);
+    if (e == cudaSuccess) e = ms::launch_split_f16(L, c->o, H * 64, R, H * 64, c->hh, c->hl, kh);
+    if (e == cudaSuccess)
+      e = ms::launch_gemm_f16(L, ly.w[1], ly.gw[1], c->hh, c->hl, kh, R, c->y, d, nullptr, nullptr, 0, ms::kStore, &gw);
+    if (e == cudaSuccess)
+      e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, nullptr, c->hh, c->hl, kh);
+    if (e == cudaSuccess)
+      e = ms::launch_gemm_f16(L, ly.w[2], ly.gw[2], c->hh, c->hl, kh, R, nullptr, 0, c->uh, c->ul, F, ms::kGelu, &gw);
+    if (e == cudaSuccess)
+      e = ms::launch_gemm_f16(L, ly.w[3], ly.gw[3], c->uh, c->ul, F, R, c->y, d, nullptr, nullptr, 0, ms::kStore, &gw);
   }
   if (e == cudaSuccess)
     e = ms::launch_skipln(L, c->x, g.n_layers > 0 ? c->y : nullptr, m->ln_f_g, m->ln_f_b, g.ln_eps, R, d, c->h);
@@ -261,8 +278,10 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
     if (gv) {
       e = ms::launch_gemv(L, ly.w[0], c->x, d, B, ly.ln1_g, ly.ln1_b, g.ln_eps, c->qkv, nq, ms::kStore);
     } else {
-      e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore, &gw);
+      e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, nullptr, c->hh, c->hl, c->kh);
+      if (e == cudaSuccess)
+        e = ms::launch_gemm_f16(L, ly.w[0], ly.gw[0], c->hh, c->hl, c->kh, B, c->qkv, nq, nullptr, nullptr, 0, ms::kStore,
+                                &gw);
     }
     if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
     if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o);
@@ -271,10 +290,15 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[3], c->u, F, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
     } else {
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd, &gw);
-      if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[2], c->h, d, B, c->u, F, ms::kGelu, &gw);
-      if (e == cudaSuccess) e = ms::launch_gemm_tc(L, ly.w[3], c->u, F, B, c->x, d, ms::kAdd, &gw);
+      if (e == cudaSuccess) e = ms::launch_split_f16(L, c->o, H * 64, B, H * 64, c->hh, c->hl, c->kh);
+      if (e == cudaSuccess)
+        e = ms::launch_gemm_f16(L, ly.w[1], ly.gw[1], c->hh, c->hl, c->kh, B, c->x, d, nullptr, nullptr, 0, ms::kAdd, &gw);
+      if (e == cudaSuccess)
+        e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, nullptr, c->hh, c->hl, c->kh);
+      if (e == cudaSuccess)
+        e = ms::launch_gemm_f16(L, ly.w[2], ly.gw[2], c->hh, c->hl, c->kh, B, nullptr, 0, c->uh, c->ul, F, ms::kGelu, &gw);
+      if (e == cudaSuccess)
+        e = ms::launch_gemm_f16(L, ly.w[3], ly.gw[3], c->uh, c->ul, F, B, c->x, d, nullptr, nullptr, 0, ms::kAdd, &gw);
     }
   }
   ms::LmHeadWork w{c->lm_val, c->lm_idx, c->lm_counter};
@@ -451,7 +475,18 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
           w.h = a.take<uint16_t>((size_t)N * K);
         }
         L.wt[i] = a.take<uint8_t>(ms::tile_packed_bytes(w));
+        L.gw[i].wt = w.fmt == ms::kInt4 ? a.take<unsigned char>(ms::gemm_tiles_bytes(w)) : nullptr;
+        L.gw[i].rinv = w.fmt == ms::kInt4 ? a.take<float>(ms::gemm_rows_padded(w)) : nullptr;
       }
+    }
+    {
+      size_t rmax = 1;
+      for (int i = 0; i < 4; ++i) {
+        int N, K;
+        mat_nk(c, i, &N, &K);
+        rmax = std::max(rmax, (size_t)(N + 127) / 128 * 128);
+      }
+      m->rexp = a.take<float>(rmax);
     }
     if (pass == 0) {
       a.size = round_up(a.used, 256);
@@ -494,6 +529,9 @@ ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device
   // tile-packed copies, made on the device from the rows just copied
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l)
     for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = ms::launch_repack_tiles(m->layers[l].w[i], m->layers[l].wt[i], 0);
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l)
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+      e = ms::launch_gemm_repack(m->layers[l].w[i], m->layers[l].gw[i], m->rexp, 0);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e == cudaSuccess && c.n_layers > 0) {
     std::vector<ms::PLayer> pl(c.n_layers);
@@ -626,6 +664,11 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->q = a.take<float>(R * g.n_heads * 64);
     c->o = a.take<float>(R * g.n_heads * 64);
     c->u = a.take<float>(R * g.d_ff);
+    c->kh = std::max(g.d_model, g.n_heads * 64);
+    c->hh = a.take<__half>(R * c->kh);
+    c->hl = a.take<__half>(R * c->kh);
+    c->uh = reinterpret_cast<__half*>(c->u);
+    c->ul = c->uh ? c->uh + R * g.d_ff : nullptr;
     c->logits = a.take<float>((size_t)batch * g.vocab);
     if (pass == 0) {
       a.size = round_up(a.used, 256);
@@ -898,6 +941,49 @@ ms_status ms_device_status(ms_cache* c, void* stream) {
 }
 
 // ---- single operations ---------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+// The tcgen05 GEMM for a single-operation call on caller arrays: the weights' tile-packed copy
+// and the activation planes are made in stream-ordered temporaries (cudaMallocAsync) that are
+// released on the stream after the GEMM; the launch policy is the model's own.
+ms_status op_gemm(const ms::WView& w, const float* x, int M, float* y, cudaStream_t st, const char* who) {
+  int dev = 0, nsm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  const ms::GemmWork gw{nsm > 0 ? nsm : 1};
+  ms::Launch L{st, false, nullptr};
+  const size_t tiles = ms::gemm_tiles_bytes(w), rows = ms::gemm_rows_padded(w);
+  const size_t planes = (size_t)M * w.K * sizeof(__half);
+  const size_t bytes = round_up(tiles, 256) + 2 * round_up(rows * 4, 256) + 2 * round_up(planes, 256);
+  char* tmp = nullptr;
+  CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&tmp), bytes, st));
+  char* p = tmp;
+  ms::GemmWeights g{nullptr, nullptr};
+  float* rexp = nullptr;
+  if (w.fmt == ms::kInt4) {
+    g.wt = reinterpret_cast<unsigned char*>(p);
+    p += round_up(tiles, 256);
+    g.rinv = reinterpret_cast<float*>(p);
+    p += round_up(rows * 4, 256);
+    rexp = reinterpret_cast<float*>(p);
+    p += round_up(rows * 4, 256);
+  }
+  __half* xh = reinterpret_cast<__half*>(p);
+  __half* xl = reinterpret_cast<__half*>(p + round_up(planes, 256));
+  cudaError_t e = cudaSuccess;
+  if (w.fmt == ms::kInt4) e = ms::launch_gemm_repack(w, g, rexp, st);
+  if (e == cudaSuccess) e = ms::launch_split_f16(L, x, w.K, M, w.K, xh, xl, w.K);
+  if (e == cudaSuccess) e = ms::launch_gemm_f16(L, w, g, xh, xl, w.K, M, y, w.N, nullptr, nullptr, 0, ms::kStore, &gw);
+  const cudaError_t ef = cudaFreeAsync(tmp, st);
+  if (e != cudaSuccess) return fail(MS_ERR_CUDA, "%s: gemm: %s", who, cudaGetErrorString(e));
+  if (ef != cudaSuccess) return fail(MS_ERR_CUDA, "%s: cudaFreeAsync: %s", who, cudaGetErrorString(ef));
+  return MS_OK;
+}
+}  // namespace
+
+extern "C" {
+
 ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, const float* scales, int N, float* y,
                           void* stream) {
   if (!x || !packed || !scales || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_w4: null pointer");
@@ -907,14 +993,7 @@ ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, c
   ms::Launch L{(cudaStream_t)stream, false, nullptr};
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
-  if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4: N must be a multiple of 64 for this M");
-  // the launch policy the model's own calls use (K split over a cluster when the tiles
-  // alone would leave SMs idle)
-  int dev = 0, nsm = 0;
-  CUDA_TRY(cudaGetDevice(&dev));
-  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-  const ms::GemmWork gw{nsm > 0 ? nsm : 1};
-  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore, &gw), "gemm");
+  return op_gemm(w, x, M, y, (cudaStream_t)stream, "ms_op_matmul_w4");
 }
 
 ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y, void* stream) {
@@ -925,14 +1004,43 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
   ms::Launch L{(cudaStream_t)stream, false, nullptr};
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
-  if (N % 64 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_f16: N must be a multiple of 64 for this M");
-  // the launch policy the model's own calls use (K split over a cluster when the tiles
-  // alone would leave SMs idle)
-  int dev = 0, nsm = 0;
-  CUDA_TRY(cudaGetDevice(&dev));
-  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  return op_gemm(w, x, M, y, (cudaStream_t)stream, "ms_op_matmul_f16");
+}
+
+ms_status ms_op_split_f16(const float* x, int ldx, int M, int K, uint16_t* x_hi, uint16_t* x_lo, int ldh,
+                          void* stream) {
+  if (!x || !x_hi || !x_lo) return fail(MS_ERR_INVALID_ARG, "ms_op_split_f16: null pointer");
+  if (M < 0 || K < 4 || K % 4 != 0 || ldx < K || ldx % 4 != 0 || ldh < K || ldh % 4 != 0)
+    return fail(MS_ERR_SHAPE, "ms_op_split_f16: need K a multiple of 4, ldx and ldh >= K and multiples of 4");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(x_hi) & 7) ||
+      (reinterpret_cast<uintptr_t>(x_lo) & 7))
+    return fail(MS_ERR_INVALID_ARG, "ms_op_split_f16: x must be 16-byte and the planes 8-byte aligned");
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  return check_launch(ms::launch_split_f16(L, x, ldx, M, K, reinterpret_cast<__half*>(x_hi),
+                                           reinterpret_cast<__half*>(x_lo), ldh),
+                      "split_f16");
+}
+
+ms_status ms_model_matmul(const ms_model* m, int layer, int which, const uint16_t* x_hi, const uint16_t* x_lo,
+                          int ldx, int M, float* y, int ldy, void* stream) {
+  if (!m || !x_hi || !x_lo || !y) return fail(MS_ERR_INVALID_ARG, "ms_model_matmul: null argument");
+  if (layer < 0 || layer >= m->cfg.n_layers || which < 0 || which > 3)
+    return fail(MS_ERR_INVALID_ARG, "ms_model_matmul: no matrix %d of layer %d", which, layer);
+  const DevLayer& ly = m->layers[layer];
+  const ms::WView& w = ly.w[which];
+  if (M < 1 || ldx < w.K || ldx % 8 != 0 || ldy < w.N)
+    return fail(MS_ERR_SHAPE, "ms_model_matmul: need M >= 1, ldx >= K (a multiple of 8), ldy >= N");
+  if ((reinterpret_cast<uintptr_t>(x_hi) & 15) || (reinterpret_cast<uintptr_t>(x_lo) & 15))
+    return fail(MS_ERR_INVALID_ARG, "ms_model_matmul: the planes must be 16-byte aligned");
+  DeviceGuard dg(m->device);
+  int nsm = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, m->device));
   const ms::GemmWork gw{nsm > 0 ? nsm : 1};
-  return check_launch(ms::launch_gemm_tc(L, w, x, K, M, y, N, ms::kStore, &gw), "gemm");
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  return check_launch(ms::launch_gemm_f16(L, w, ly.gw[which], reinterpret_cast<const __half*>(x_hi),
+                                          reinterpret_cast<const __half*>(x_lo), ldx, M, y, ldy, nullptr, nullptr, 0,
+                                          ms::kStore, &gw),
+                      "model matmul");
 }
 
 ms_status ms_op_skip_layernorm(float* x, const float* y, const float* gamma, const float* beta, float eps, int R, int d,

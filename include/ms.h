@@ -214,8 +214,10 @@ const char* ms_last_error(void);
  * variant: symmetric INT4 g32 weights, fp32 activations): y[m][n] = sum_k x[m][k] * W[n][k]
  * with W[n][k] = q[n][k] * s[n][k/32].  x fp32 [M][K] and y fp32 [M][N], row-major;
  * packed and scales as ms_quantize_int4_g32 writes them.  M in {1, 2, 4, 8} runs the
- * decode GEMV when a CTA's slice of rows fits its shared memory; any other M runs the
- * tcgen05 GEMM, which needs N a multiple of 64.  K a multiple of 256.  MS_ERR_INVALID_ARG
+ * decode GEMV (fp32) when a CTA's slice of rows fits its shared memory; any other M runs the
+ * tcgen05 GEMM (fp16 hi + lo operand pairs, three products, fp32 accumulation), after making
+ * the weights' tile-packed copy and the activation planes in stream-ordered temporaries
+ * (cudaMallocAsync / cudaFreeAsync on `stream`).  K a multiple of 256.  MS_ERR_INVALID_ARG
  * for a NULL pointer, MS_ERR_SHAPE for other sizes; nothing is launched then. */
 ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, const float* scales,
                           int N, float* y, void* stream);
@@ -223,6 +225,24 @@ ms_status ms_op_matmul_w4(const float* x, int M, int K, const uint8_t* packed, c
  * "MuScriptor for Core AI (.aimodel)", file table), same size rules. */
 ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, int N, float* y,
                            void* stream);
+/* The operand form of the tcgen05 GEMM: each fp32 value v of x (rows of K at stride ldx)
+ * as an IEEE half pair, x_hi = fp16(v) and x_lo = fp16(v - x_hi) (round to nearest even,
+ * a 22-bit significand together), written to x_hi and x_lo (rows at stride ldh halves).
+ * K, ldx and ldh multiples of 4 (ldx, ldh >= K); x 16-byte aligned, the planes 8-byte
+ * aligned.  A |v| of 65504 or more does not fit a half: the pair is then inf and the call
+ * cannot report it (the calls of a cache flag it in the status word, MS_ERR_SHAPE). */
+ms_status ms_op_split_f16(const float* x, int ldx, int M, int K, uint16_t* x_hi, uint16_t* x_lo, int ldh,
+                          void* stream);
+
+/* Backbone MatMul `which` (0 QKV, 1 O, 2 FC1, 3 FC2) of layer `layer` of the model, on M
+ * activation rows given as ms_op_split_f16 planes (row stride ldx halves, a multiple of 8,
+ * 16-byte aligned): y[m][n] = sum_k (x_hi + x_lo)[m][k] W[n][k], y fp32 [M][ldy].  This is
+ * the tcgen05 GEMM the prefill and batched decode run ("MuScriptor Medium — optimized W4A32
+ * ONNX Runtime", Model variant: MatMulNBits), with the model's own tile-packed weights.
+ * MS_ERR_INVALID_ARG for no such matrix or a NULL pointer, MS_ERR_SHAPE for other sizes. */
+ms_status ms_model_matmul(const ms_model* model, int layer, int which, const uint16_t* x_hi,
+                          const uint16_t* x_lo, int ldx, int M, float* y, int ldy, void* stream);
+
 /* SkipLayerNorm ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model variant):
  * s = x + y (y may be NULL: plain LayerNorm), x <- s, h = (s - mean) / sqrt(var + eps)
  * * gamma + beta with the biased variance, per row of d.  x, y, h fp32 [R][d]. */

@@ -49,8 +49,8 @@ def test_quantizer_edge_groups():
     assert list(pg.cpu().numpy()[0, :4]) == [207, 138, 25, 24]
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 3, 16, 64, 130])
-@pytest.mark.parametrize("N,K", [(2304, 768), (768, 3072), (1536, 1024), (1024, 4096), (1536, 6144)])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 3, 16, 64, 130, 504])
+@pytest.mark.parametrize("N,K", [(2304, 768), (768, 3072), (1536, 1024), (1024, 4096), (1536, 6144), (200, 512)])
 def test_matmul_w4(M, N, K):
     w = synth.make_matrix(N, K, seed=200 + K)
     x = synth.make_activations(M, K, seed=300 + M)
@@ -138,3 +138,42 @@ def test_lm_head_argmax_ties_pick_the_lowest_index_across_ctas():
     lg = lg.cpu().numpy()
     assert lg[0, 5] == lg[0, 700] == lg[0, 1300]
     assert list(am.cpu().numpy()) == [5, 5]
+
+
+# ---- the tcgen05 GEMM's operand planes and the model's own MatMuls ---------------------------
+
+def test_split_f16_planes_bit_exact():
+    """hi = fp16(x), lo = fp16(x - hi) with round-to-nearest-even, over magnitudes from
+    subnormal halves to near the half maximum, signed zeros and a ragged row stride."""
+    rng = np.random.default_rng(5)
+    M, K = 37, 520
+    x = (rng.standard_normal((M, K)) * np.exp2(rng.integers(-30, 15, (M, K)))).astype(np.float32)
+    x[0, :4] = [0.0, -0.0, 65000.0, -6.0e-8]
+    hi, lo = ms.split_f16(_dev(x))
+    want_hi = x.astype(np.float16)
+    want_lo = (x - want_hi.astype(np.float32)).astype(np.float16)
+    assert np.array_equal(hi.cpu().numpy().view(np.uint16), want_hi.view(np.uint16))
+    assert np.array_equal(lo.cpu().numpy().view(np.uint16), want_lo.view(np.uint16))
+
+
+@pytest.mark.parametrize("fmt", ["int4", "fp16"])
+@pytest.mark.parametrize("M", [1, 3, 64, 200, 504])
+def test_model_matmul_against_the_oracle_weights(fmt, M):
+    """ms_model_matmul (the GEMM prefill and batched decode run, on the model's tile-packed
+    weights) against the oracle's dequantised matrices, on split activation planes, every
+    matrix of a 2-layer shape; M from one row to several 256-row tiles with a ragged tail.
+    (Ragged N is covered through ms_op_matmul_w4 with N = 200.)"""
+    sh = synth.Shape("gemm", 2, 768, 12, 4, 1280, vocab=64)
+    draw = synth.make_weights(sh, seed=7, std=0.05)
+    om = O.OracleModel(draw, fmt)
+    gm = ms.Model.from_draw(draw, fmt)
+    for l in range(sh.n_layers):
+        for i, (N, K) in enumerate(sh.matmul_shapes()):
+            x = synth.make_activations(M, K, seed=900 + 10 * l + i)
+            hi, lo = ms.split_f16(_dev(x))
+            xs = hi.cpu().numpy().astype(np.float64) + lo.cpu().numpy().astype(np.float64)
+            assert np.all(np.abs(xs - x) <= 2.0 ** -22 * np.abs(x) + 2.0 ** -25)
+            y = gm.matmul(l, i, hi, lo).cpu().numpy().astype(np.float64)
+            W = om.layers[l].w[i]
+            ref = xs @ W.T
+            assert np.all(np.abs(y - ref) <= _dot_bound(x, W.astype(np.float32))), (l, i)
