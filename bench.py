@@ -54,6 +54,8 @@ def _args():
                     help="skip the batched-decode block (the 64-stream medium workload)")
     ap.add_argument("--no-prefill-tensor", action="store_true",
                     help="skip the prefill GEMM tensor-pipe block")
+    ap.add_argument("--decode-path", type=int, default=0, choices=[0, 1, 2],
+                    help="0 automatic, 1 persistent decode kernel, 2 one kernel per operation")
     return ap.parse_args()
 
 
@@ -426,6 +428,7 @@ def run_ours(a):
     prefix = prefix_h.to(dev)
     start = start_h.to(dev)
     cache = ms.Cache(model, B, wl.capacity)
+    cache.set_decode_path(a.decode_path)
     out_tok = torch.empty((wl.decode_steps, B), dtype=torch.int32, device=dev)
     flush = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)

@@ -21,8 +21,8 @@
 //      split holding pos appends to the cache with v), scores over its run of positions,
 //      partial (m, l, o); one CTA per head then merges the splits' partials  -> o
 //   C  O rows
-//   D  x += O parts, LN2, FC1 rows (GELU applied by the consumer when FC1 is split)
-//   E  GELU of the FC1 parts' sum, FC2 rows
+//   D  x += O parts, LN2, FC1 rows (GELU applied by the producer when FC1's tiles are whole)
+//   E  GELU of the FC1 parts' sum when FC1 is split along K, FC2 rows
 // Every CTA keeps its own copy of the residual rows x (each thread its own elements) and
 // adds the published partial sums itself, so no CTA owns output rows.
 //   after the last layer: x, LN_f, LM head rows, per-CTA argmax (guided for stream pairs
@@ -360,16 +360,18 @@ struct VecSrc {
 // values (and gamma, beta) are staged in shared memory, each thread reading back only the
 // pairs it wrote.  Returns false (this thread) on a failed wait; the caller ORs the outcome
 // over the CTA.
+// Only pairs [p0, P) are loaded (a phase whose work units all lie in one K range needs no
+// more); a LayerNorm'd row is always loaded whole.
 template <bool PLANES, int S>
-__device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* g, const float* bt, float eps,
-                                         uint32_t* phi, uint32_t* plo, float* inv, float* act, const Region& rg,
-                                         Red& red, const PersistArgs& a) {
+__device__ __forceinline__ bool load_row(const VecSrc& src, int K, int p0, int P, const float* g, const float* bt,
+                                         float eps, uint32_t* phi, uint32_t* plo, float* inv, float* act,
+                                         const Region& rg, Red& red, const PersistArgs& a) {
   constexpr int PR = kPairBatch / S;   // pairs per round per thread
-  const int tid = threadIdx.x, P = K >> 1;
+  const int tid = threadIdx.x;
   float2* xin = rg.xin;
   bool ok = true;
 #pragma unroll 1
-  for (int base = 0; base < P; base += kThreads * PR) {
+  for (int base = p0; base < P; base += kThreads * PR) {
     uint64_t w0[kPairBatch], w1[kPairBatch];
     const uint64_t* pp[kPairBatch];
     bool use[kPairBatch];
@@ -425,13 +427,13 @@ __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* 
   float mean = 0.f, rstd = 1.f, bound = 0.f;
   if (g) {
     float s = 0.f;
-    for (int p = tid; p < P; p += kThreads) {
+    for (int p = p0 + tid; p < P; p += kThreads) {
       const float2 x = xin[p];
       s += x.x + x.y;
     }
     mean = block_red(s, 0.f, 0.f, red).x / K;
     float q = 0.f, am = 0.f, bm = 0.f;
-    for (int p = tid; p < P; p += kThreads) {
+    for (int p = p0 + tid; p < P; p += kThreads) {
       const float2 x = xin[p];
       const float4 gb = rg.gb[p];
       const float d0 = x.x - mean, d1 = x.y - mean;
@@ -444,7 +446,7 @@ __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* 
     bound = rstd * r.y + r.z;   // |LN(x)_k| <= rstd |x_k - mean| |g_k| + |b_k|
   } else if (PLANES) {
     float am = 0.f;
-    for (int p = tid; p < P; p += kThreads) {
+    for (int p = p0 + tid; p < P; p += kThreads) {
       const float2 x = xin[p];
       am = fmaxf(am, fmaxf(fabsf(x.x), fabsf(x.y)));
     }
@@ -456,7 +458,7 @@ __device__ __forceinline__ bool load_row(const VecSrc& src, int K, const float* 
     sc = exp2i(e);
     if (tid == 0) *inv = exp2i(-e);
   }
-  for (int p = tid; p < P; p += kThreads) {
+  for (int p = p0 + tid; p < P; p += kThreads) {
     const float2 x = xin[p];
     float y0 = x.x, y1 = x.y;
     if (g) {
@@ -594,6 +596,7 @@ struct MvJob {
   uint64_t* out;
   long long stride;
   unsigned ep;
+  bool gelu;   // publish GELU of the sums (only when the tiles are not split along K)
 };
 
 __device__ __forceinline__ unsigned atom_add_acq_rel_shared(unsigned* p, unsigned v) {
@@ -715,7 +718,9 @@ __device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, const MvJ
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) v += pp[w * M * kTile];
     const int u = jb.u0 + ul, t = u / S, h = u - t * S;
-    st_stamp(jb.out + h * jb.stride + (size_t)m * jb.N + t * kTile + rr, v * inv_s[m], jb.ep);
+    v *= inv_s[m];
+    if (jb.gelu) v = gelu_ool(v);
+    st_stamp(jb.out + h * jb.stride + (size_t)m * jb.N + t * kTile + rr, v, jb.ep);
   }
   consumer_bar();  // the region is reused by the next phase
   return true;
@@ -1133,8 +1138,8 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
   // The phase input: row m of a vector into A planes rows 2m, 2m + 1.  st: the S slices of
   // the vector (stride between slices, ld between rows) or null for the token embedding;
   // res: add and update the residual copy; gelu: GELU of the sum.
-  auto load_planes = [&](const uint64_t* st, long long stride, int S, int ld, int K, unsigned ep, const float* g,
-                         const float* bt, bool res, bool gelu) -> bool {
+  auto load_planes = [&](const uint64_t* st, long long stride, int S, int ld, int K, int p0, int p1, unsigned ep,
+                         const float* g, const float* bt, bool res, bool gelu) -> bool {
     bool ok = true;
     const int pw = (K >> 1) + 16;
 #pragma unroll 1
@@ -1143,9 +1148,9 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
                        res ? xres + (size_t)m * (d / 2) : nullptr, gelu};
       uint32_t* phi = rg.planes + (2 * m) * pw;
       uint32_t* plo = rg.planes + (2 * m + 1) * pw;
-      if (S == 1) ok = load_row<true, 1>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
-      else if (S == 2) ok = load_row<true, 2>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
-      else ok = load_row<true, 4>(src, K, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
+      if (S == 1) ok = load_row<true, 1>(src, K, p0, p1, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
+      else if (S == 2) ok = load_row<true, 2>(src, K, p0, p1, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
+      else ok = load_row<true, 4>(src, K, p0, p1, g, bt, a.eps, phi, plo, &inv_s[m], nullptr, rg, red, a) && ok;
     }
     return !consumer_bar_or(!ok);
   };
@@ -1200,7 +1205,27 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
         const int S_in = (emb || pm < 0) ? 1 : sched[18 + pm];   // the embedding and o are single vectors
         const float* g = ph == 0 ? ly.ln1_g : ph == 3 ? ly.ln2_g : nullptr;
         const float* bt = ph == 0 ? ly.ln1_b : ph == 3 ? ly.ln2_b : nullptr;
-        if (!load_planes(src, stride, S_in, K, K, epA + ph - 1, g, bt, ph == 0 || ph == 3, ph == 4)) return false;
+        // GELU of FC1's output: applied by FC1's producers when its tiles are whole, else by
+        // the consumers after adding the K-range parts
+        const bool fc1_whole = sched[18 + 2] == 1;
+        // O and FC2 (no LayerNorm on their input): load only the K range of this CTA's units
+        // when they all lie in one part of a K-split matrix, nothing when it has none
+        int p0 = 0, p1 = K >> 1;
+        if (mi == 1 || mi == 3) {
+          const int Sm = sched[18 + mi], u0 = sched[10 + mi], u1 = sched[14 + mi], KG = K >> 5;
+          if (u1 <= u0) {
+            p1 = 0;
+          } else if (Sm > 1) {
+            const int h0 = u0 % Sm, h1 = (u1 - 1) % Sm;
+            if (u1 - u0 <= Sm && h0 <= h1) {
+              p0 = (KG * h0 / Sm) * 16;
+              p1 = (KG * (h1 + 1) / Sm) * 16;
+            }
+          }
+        }
+        if (!load_planes(src, stride, S_in, K, K, p0, p1, epA + ph - 1, g, bt, ph == 0 || ph == 3,
+                         ph == 4 && !fc1_whole))
+          return false;
         MvJob jb;
         jb.K = K;
         jb.N = mat_N(a, mi);
@@ -1212,6 +1237,7 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
         jb.out = a.vs[mi];
         jb.stride = a.vstride[mi];
         jb.ep = epA + ph;
+        jb.gelu = mi == 2 && fc1_whole;
         if (!mv_phase<M, FMT>(ring, rg, jb, inv_s)) return false;
       }
     }
@@ -1225,13 +1251,13 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
                          false};
         const int S3 = sched[18 + 3];
         if (S3 == 1)
-          ok = load_row<false, 1>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+          ok = load_row<false, 1>(src, d, 0, d >> 1, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
                                   red, a) && ok;
         else if (S3 == 2)
-          ok = load_row<false, 2>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+          ok = load_row<false, 2>(src, d, 0, d >> 1, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
                                   red, a) && ok;
         else
-          ok = load_row<false, 4>(src, d, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
+          ok = load_row<false, 4>(src, d, 0, d >> 1, a.lnf_g, a.lnf_b, a.eps, nullptr, nullptr, nullptr, act + (size_t)m * d, rg,
                                   red, a) && ok;
       }
       if (consumer_bar_or(!ok)) return false;
