@@ -76,6 +76,7 @@ _PROTOS = {
     "ms_cache_decode_path": (_I, [_P]),
     "ms_cache_set_guidance": (_I, [_P, ctypes.c_float]),
     "ms_cache_guidance": (ctypes.c_float, [_P]),
+    "ms_cache_set_wait_limits": (_I, [_P, ctypes.c_longlong, _I]),
     "ms_cache_destroy": (_I, [_P]),
     "ms_cache_kv_bytes": (ctypes.c_size_t, [ctypes.POINTER(Config), _I, _I]),
     "ms_prefill": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _P]),
@@ -317,6 +318,11 @@ class Cache:
         """Classifier-free guidance over stream pairs (2p, 2p+1) = (conditional,
         unconditional): both take the argmax of u + scale (k - u); 0 turns it off."""
         _check(_lib.ms_cache_set_guidance(self._h, ctypes.c_float(scale)), "ms_cache_set_guidance")
+
+    def set_wait_limits(self, polls: int, stall: int = 0):
+        """Persistent kernel's wait limits (0 = defaults); stall 1 or 2 injects a wait that
+        nothing satisfies (tests of the timeout path only)."""
+        _check(_lib.ms_cache_set_wait_limits(self._h, polls, stall), "ms_cache_set_wait_limits")
 
     @property
     def guidance(self) -> float:

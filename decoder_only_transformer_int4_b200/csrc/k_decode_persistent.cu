@@ -56,7 +56,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kSlot = 16384;
-constexpr long long kGridSpinLimit = 1ll << 24;  // polls of the barrier count (~10 s)
 constexpr int kAttSub = 64;
 constexpr int kAttMaxSplits = 128;
 constexpr int kMinPerSplit = 16;
@@ -231,14 +230,13 @@ __device__ __forceinline__ void ld_stamp2(const uint64_t* p, uint64_t& w0, uint6
 // again together (all in flight), with one backoff per round — never one round trip per
 // word.  Pairs (two consecutive words per load) and single words.  Returns false if the
 // wait ran out or another CTA gave up.
-constexpr long long kSettleLimit = 1ll << 23;  // rounds (each >= 64 ns apart) before giving up
 __device__ __forceinline__ bool stale2(uint64_t w0, uint64_t w1, unsigned ep) {
   return ((unsigned)(w0 >> 32) != ep) | ((unsigned)(w1 >> 32) != ep);
 }
 __device__ __forceinline__ bool settle_wait(long long it, unsigned& ns, const PersistArgs& a) {
   if ((it & 15) == 15) {
     if (*reinterpret_cast<volatile unsigned*>(a.abort)) return false;
-    if (it > kSettleLimit) {
+    if (it > a.settle_limit) {
       flag_error(a.status, kErrTimeout);
       atomicExch(a.abort, 1u);
       return false;
@@ -735,7 +733,7 @@ __device__ bool grid_sync(const PersistArgs& a, unsigned& epoch, int* ok_s) {
     int ok = 1;
     __threadfence();  // the CTA's stores (seen through the named barrier) before the release
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a.bar_count), "r"(1u) : "memory");
-    const unsigned target = epoch * gridDim.x;
+    const unsigned target = epoch * gridDim.x + (a.test_stall == 2 ? 1u : 0u);
     long long it = 0;
     for (;;) {
       unsigned v;
@@ -746,7 +744,7 @@ __device__ bool grid_sync(const PersistArgs& a, unsigned& epoch, int* ok_s) {
           ok = 0;
           break;
         }
-        if (it > kGridSpinLimit) {
+        if (it > a.grid_limit) {
           flag_error(a.status, kErrTimeout);
           atomicExch(a.abort, 1u);
           ok = 0;
@@ -834,7 +832,8 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
   use[3] = use[4] = owner && tid < 32;
 #pragma unroll
   for (int k = 0; k < 5; ++k) w[k] = use[k] ? ld_stamp(pp[k]) : 0;
-  const bool ok = settle_words<5>(w, pp, use, ep, a);
+  // (a test may make this wait for an epoch that no phase writes)
+  const bool ok = settle_words<5>(w, pp, use, a.test_stall == 1 ? (ep ^ 0x80000000u) : ep, a);
   if (use[0]) {
     const float x0 = __uint_as_float((unsigned)w[0]), x1 = __uint_as_float((unsigned)w[1]);
     const float c = cs[qj], s = sn[qj];

@@ -51,7 +51,14 @@ struct PersistArgs {
   int nslot;
   int sched_cap;             // capacity of the per-CTA slice table (entries)
   float guidance;            // 0, or classifier-free guidance over stream pairs (2p, 2p+1)
+  long long settle_limit;    // rounds a stamped-word wait may take before it gives up
+  long long grid_limit;      // polls of the grid barrier before it gives up
+  int test_stall;            // tests only: 1 = an attention unit waits for a stamp no phase writes,
+                             // 2 = the grid barrier waits for one arrival more than the grid makes
 };
+// Default wait limits (far above any legitimate wait, far below a hang).
+constexpr long long kDefaultSettleLimit = 1ll << 23;
+constexpr long long kDefaultGridLimit = 1ll << 24;
 
 cudaError_t init_attrs_persistent();
 // Ring slots that fit next to the kernel's other shared memory (0: the kernel does not fit).

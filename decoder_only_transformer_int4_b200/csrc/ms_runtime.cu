@@ -201,6 +201,8 @@ struct ms_cache {
   size_t persist_smem = 0;
   int persist_sched_cap = 0;
   float guidance = 0.f;              // classifier-free guidance scale (0: off)
+  long long wait_limit = 0;          // persistent kernel's wait limits (0: the defaults)
+  int test_stall = 0;                // tests only: an injected wait nothing satisfies
   int nsm = 148;                     // SMs of the device
   int path_request = 0;                  // 0 auto, 1 persistent kernel, 2 one kernel per operation
   unsigned long long launches = 0;  // kernels launched for this cache
@@ -319,6 +321,8 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
                            int32_t* argmax, cudaStream_t st) {
   const ms_config& g = m->cfg;
   cudaError_t e = cudaMemsetAsync(c->sync3, 0, 3 * sizeof(unsigned), st);
+  // the last-CTA ticket of the LM head starts at zero (a launch that gave up may have left it set)
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->lm_counter, 0, sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
   // epochs of the stamped vectors: fresh for every launch; restart from zeroed words
   // before the 32-bit counter would wrap
@@ -373,6 +377,9 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.nslot = c->persist_nslot;
   a.sched_cap = c->persist_sched_cap;
   a.guidance = c->guidance;
+  a.settle_limit = c->wait_limit > 0 ? c->wait_limit : ms::kDefaultSettleLimit;
+  a.grid_limit = c->wait_limit > 0 ? c->wait_limit : ms::kDefaultGridLimit;
+  a.test_stall = c->test_stall;
   return ms::launch_decode_persistent(a, c->B, c->persist_grid, c->persist_smem, st);
 }
 
@@ -758,6 +765,15 @@ ms_status ms_cache_set_guidance(ms_cache* c, float scale) {
 }
 
 float ms_cache_guidance(const ms_cache* c) { return c ? c->guidance : 0.f; }
+
+ms_status ms_cache_set_wait_limits(ms_cache* c, long long polls, int stall) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_wait_limits: null cache");
+  if (polls < 0 || stall < 0 || stall > 2)
+    return fail(MS_ERR_INVALID_ARG, "ms_cache_set_wait_limits: need polls >= 0 and stall in {0, 1, 2}");
+  c->wait_limit = polls;
+  c->test_stall = stall;
+  return MS_OK;
+}
 
 int ms_cache_decode_path(const ms_cache* c) {
   if (!c) return -1;

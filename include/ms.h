@@ -189,6 +189,19 @@ ms_status ms_cache_set_guidance(ms_cache* cache, float scale);
 /* The current guidance scale (0 when off or on NULL). */
 float ms_cache_guidance(const ms_cache* cache);
 
+/* Wait limits of the persistent decode kernel, for tests of its failure path.  No passage of
+ * the pages corresponds to this call.  Every wait of that kernel (a stamped activation word
+ * from another CTA, the grid barrier between steps) gives up after a limit, sets the timeout
+ * bit of the status word (ms_device_status then returns MS_ERR_TIMEOUT) and makes every CTA
+ * leave; the launch then returns with the cache's contents undefined (reset it or use
+ * another cache).  polls: the limit in polls (0 restores the defaults, about ten seconds of
+ * waiting).  stall (tests only, 0 in normal use): 1 makes the attention units wait for an
+ * activation word that no phase writes, 2 makes the grid barrier wait for one arrival more
+ * than the grid makes; either wait then runs out after `polls`.  Host state only; applies to
+ * the next persistent launch on this cache.  MS_ERR_INVALID_ARG for a negative limit or an
+ * unknown stall. */
+ms_status ms_cache_set_wait_limits(ms_cache* cache, long long polls, int stall);
+
 /* ---- cache transfer (host pointers, synchronous) --------------------------------------
  * Export in the pages' layout [L][batch][T][Hk][64] (T = current length);
  * import T positions in the same layout and set the length to T. */
