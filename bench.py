@@ -54,6 +54,8 @@ def _args():
                     help="skip the batched-decode block (the 64-stream medium workload)")
     ap.add_argument("--no-prefill-tensor", action="store_true",
                     help="skip the prefill GEMM tensor-pipe block")
+    ap.add_argument("--no-pages", action="store_true",
+                    help="skip the page-faithful block (kv heads = heads, fp32 and fp16 caches)")
     ap.add_argument("--decode-path", type=int, default=0, choices=[0, 1, 2],
                     help="0 automatic, 1 persistent decode kernel, 2 one kernel per operation")
     return ap.parse_args()
@@ -123,9 +125,10 @@ def _kernel_sha16():
         return None
 
 
-def _decode_bytes_per_token(wl: synth.Workload):
+def _decode_bytes_per_token(wl: synth.Workload, kv_elem: int = 4):
     """Algorithmic bytes of one decode step per stream set: backbone weights (+ scales for
-    INT4), LM head, one embedding row per stream, and K and V over every cached position.
+    INT4), LM head, one embedding row per stream, and K and V over every cached position
+    (kv_elem bytes per cache element: 4 for fp32, 2 for the half-precision cache).
     Returns (weight bytes per step, list of KV bytes per step over the run)."""
     sh = wl.shape
     w = 0
@@ -134,7 +137,7 @@ def _decode_bytes_per_token(wl: synth.Workload):
     w *= sh.n_layers
     w += sh.vocab * sh.d_model * 4 + wl.batch * sh.d_model * 4
     p0 = wl.prefix_len + 1
-    kv = [2 * sh.n_layers * wl.batch * sh.n_kv_heads * (p0 + i + 1) * 64 * 4 for i in range(wl.decode_steps)]
+    kv = [2 * sh.n_layers * wl.batch * sh.n_kv_heads * (p0 + i + 1) * 64 * kv_elem for i in range(wl.decode_steps)]
     return w, kv
 
 
@@ -355,6 +358,51 @@ def _batched_block(ms, torch, model, key, dev, flush, steps=2, warmup=1):
     }
 
 
+def _pages_block(ms, torch, dev, flush, steps=2, warmup=1):
+    """The page-faithful medium shape (kv heads = heads = 16: the W4A32 page's 469.5 MiB
+    cache at 2504 positions) at batch 1, the whole prefill + 2000-step greedy run, once with
+    the pages' fp32 cache and once with the half-precision cache option.  Each line's roofline
+    counts the cache at its own element size."""
+    wl = synth.WORKLOADS["c3pages"]
+    sh = wl.shape
+    stream = torch.cuda.current_stream(dev)
+    draw = synth.make_weights(sh, seed=0)
+    model = ms.Model.from_draw(draw, wl.weight_format, device=dev.index or 0)
+    del draw
+    prefix = torch.from_numpy(synth.make_prefix(sh, 1, wl.prefix_len, seed=1)).to(dev)
+    start = torch.from_numpy(synth.make_start_tokens(1, seed=2).reshape(1, 1)).to(dev)
+    out = torch.empty((wl.decode_steps, 1), dtype=torch.int32, device=dev)
+    peak, kind = _peaks()
+    res = {"workload": _config_json(wl, 1)["workload"], "steps": steps, "warmup": warmup}
+    for name, fmt, es in (("kv_f32", ms.MS_KV_F32, 4), ("kv_f16", ms.MS_KV_F16, 2)):
+        cache = ms.Cache(model, 1, wl.capacity, kv_format=fmt)
+        dec = []
+        for i in range(warmup + steps):
+            cache.reset()
+            flush.zero_()
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            cache.prefill(start, prefix)
+            e1.record(stream)
+            cache.generate(wl.decode_steps, out_tokens=out, logits=False)
+            e2.record(stream)
+            e2.synchronize()
+            if i >= warmup:
+                dec.append(e1.elapsed_time(e2))
+        assert cache.device_status() == ms.MS_OK
+        wbytes, kv = _decode_bytes_per_token(wl, es)
+        tot = wbytes * wl.decode_steps + sum(kv)
+        ach = tot / (statistics.mean(dec) / 1e3) / 1e9
+        res[name] = {"decode_ms_per_token": statistics.mean(dec) / wl.decode_steps,
+                     "decode_tokens_per_s": wl.decode_steps / (statistics.mean(dec) / 1e3),
+                     "algorithmic_bytes_per_token": tot / wl.decode_steps,
+                     "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                                  "peak_kind": kind}}
+        cache.close()
+    model.close()
+    return res
+
+
 def _prefill_tensor_block(ms, torch, model, shape, rows_list, dev, flush, reps=5, warmup=2):
     """Prefill GEMMs on the tensor cores: each backbone MatMul of layer 0 of the benchmark's
     model at M = prefill rows, through ms_model_matmul (the tcgen05 GEMM prefill runs, on the
@@ -528,9 +576,11 @@ def run_ours(a):
         roof["traffic"] = tr["bytes"]
         roof["traffic_per"] = f"one launch of {tr['tokens']} decode steps, cache lengths {t_lo}..{t_hi} (ncu)"
         roof["traffic_over_algorithmic"] = tr["bytes"] / alg
-    batched = prefill_tc = None
+    batched = prefill_tc = pages = None
     if world == 1 and not a.no_batched and a.workload in _BATCHED:
         batched = _batched_block(ms, torch, model, _BATCHED[a.workload], dev, flush)
+    if world == 1 and not a.no_pages and a.workload == "c3":
+        pages = _pages_block(ms, torch, dev, flush)
     if world == 1 and not a.no_prefill_tensor:
         rows = [wl.prefix_len + 1]
         if a.workload in _BATCHED:
@@ -559,6 +609,8 @@ def run_ours(a):
             line["batched"] = batched
         if prefill_tc is not None:
             line["prefill_tensor"] = prefill_tc
+        if pages is not None:
+            line["pages"] = pages
         print(json.dumps(line), flush=True)
     cache.close()
     model.close()

@@ -31,6 +31,7 @@ STATUS_NAMES = {0: "MS_OK", 1: "MS_ERR_INVALID_ARG", 2: "MS_ERR_SHAPE", 3: "MS_E
                 4: "MS_ERR_TOKEN_RANGE", 5: "MS_ERR_OOM", 6: "MS_ERR_CUDA", 7: "MS_ERR_TIMEOUT",
                 8: "MS_ERR_UNSUPPORTED"}
 MS_W_INT4_G32, MS_W_FP16 = 0, 1
+MS_KV_F32, MS_KV_F16 = 0, 1
 
 
 class MsError(RuntimeError):
@@ -67,6 +68,9 @@ _PROTOS = {
     "ms_model_destroy": (_I, [_P]),
     "ms_model_weight_bytes": (ctypes.c_size_t, [_P]),
     "ms_cache_create": (_I, [_P, _I, _I, ctypes.POINTER(_P)]),
+    "ms_cache_create_ex": (_I, [_P, _I, _I, _I, ctypes.POINTER(_P)]),
+    "ms_cache_kv_format": (_I, [_P]),
+    "ms_cache_kv_bytes_ex": (ctypes.c_size_t, [ctypes.POINTER(Config), _I, _I, _I]),
     "ms_cache_reset": (_I, [_P]),
     "ms_cache_length": (_I, [_P]),
     "ms_cache_capacity": (_I, [_P]),
@@ -77,6 +81,10 @@ _PROTOS = {
     "ms_cache_set_guidance": (_I, [_P, ctypes.c_float]),
     "ms_cache_guidance": (ctypes.c_float, [_P]),
     "ms_cache_set_wait_limits": (_I, [_P, ctypes.c_longlong, _I]),
+    "ms_cache_set_act_int8": (_I, [_P, _I]),
+    "ms_cache_act_int8": (_I, [_P]),
+    "ms_op_quantize_act_int8": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "ms_op_matmul_w4a8": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _P]),
     "ms_cache_destroy": (_I, [_P]),
     "ms_cache_kv_bytes": (ctypes.c_size_t, [ctypes.POINTER(Config), _I, _I]),
     "ms_prefill": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _P]),
@@ -135,8 +143,8 @@ def make_config(shape, weight_format: int = MS_W_INT4_G32) -> Config:
                   shape.vocab, shape.rope_base, shape.ln_eps, weight_format)
 
 
-def cache_kv_bytes(cfg: Config, batch: int, capacity: int) -> int:
-    return int(_lib.ms_cache_kv_bytes(ctypes.byref(cfg), batch, capacity))
+def cache_kv_bytes(cfg: Config, batch: int, capacity: int, kv_format: int = MS_KV_F32) -> int:
+    return int(_lib.ms_cache_kv_bytes_ex(ctypes.byref(cfg), batch, capacity, kv_format))
 
 
 # ---- single operations --------------------------------------------------------------
@@ -175,6 +183,24 @@ def split_f16(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
     lo = torch.empty((m, k), dtype=torch.float16, device=x.device)
     _check(_lib.ms_op_split_f16(_ptr(x), k, m, k, _ptr(hi), _ptr(lo), k, _stream()), "ms_op_split_f16")
     return hi, lo
+
+
+def quantize_act_int8(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """fp32 [M, K] -> (codes int8 [M, K], scales fp32 [M, K/32]) (ms_op_quantize_act_int8)."""
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    s = torch.empty((m, k // 32), dtype=torch.float32, device=x.device)
+    _check(_lib.ms_op_quantize_act_int8(_ptr(x), k, m, k, _ptr(q), _ptr(s), _stream()), "ms_op_quantize_act_int8")
+    return q, s
+
+
+def matmul_w4a8(qa: torch.Tensor, sa: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    m, k = qa.shape
+    n = packed.shape[0]
+    y = torch.empty((m, n), dtype=torch.float32, device=qa.device)
+    _check(_lib.ms_op_matmul_w4a8(_ptr(qa), _ptr(sa), m, k, _ptr(packed), _ptr(scales), n, _ptr(y), _stream()),
+           "ms_op_matmul_w4a8")
+    return y
 
 
 def skip_layernorm(x: torch.Tensor, y: Optional[torch.Tensor], gamma: torch.Tensor, beta: torch.Tensor,
@@ -294,10 +320,10 @@ class Model:
 class Cache:
     """A fixed-capacity KV cache for `batch` streams (ms_cache_create) and the calls on it."""
 
-    def __init__(self, model: Model, batch: int, capacity: int):
+    def __init__(self, model: Model, batch: int, capacity: int, kv_format: int = MS_KV_F32):
         self.model = model
         h = ctypes.c_void_p()
-        _check(_lib.ms_cache_create(model._h, batch, capacity, ctypes.byref(h)), "ms_cache_create")
+        _check(_lib.ms_cache_create_ex(model._h, batch, capacity, kv_format, ctypes.byref(h)), "ms_cache_create_ex")
         self._h = h
         self.batch = batch
         self.capacity = capacity
@@ -309,6 +335,10 @@ class Cache:
         return int(_lib.ms_cache_length(self._h))
 
     @property
+    def kv_format(self) -> int:
+        return int(_lib.ms_cache_kv_format(self._h))
+
+    @property
     def kernel_launches(self) -> int:
         return int(_lib.ms_cache_kernel_launches(self._h))
 
@@ -318,6 +348,14 @@ class Cache:
         """Classifier-free guidance over stream pairs (2p, 2p+1) = (conditional,
         unconditional): both take the argmax of u + scale (k - u); 0 turns it off."""
         _check(_lib.ms_cache_set_guidance(self._h, ctypes.c_float(scale)), "ms_cache_set_guidance")
+
+    def set_act_int8(self, on: bool):
+        """W4A8: the backbone MatMuls on INT8 activation codes (ms_cache_set_act_int8)."""
+        _check(_lib.ms_cache_set_act_int8(self._h, 1 if on else 0), "ms_cache_set_act_int8")
+
+    @property
+    def act_int8(self) -> bool:
+        return bool(_lib.ms_cache_act_int8(self._h))
 
     def set_wait_limits(self, polls: int, stall: int = 0):
         """Persistent kernel's wait limits (0 = defaults); stall 1 or 2 injects a wait that

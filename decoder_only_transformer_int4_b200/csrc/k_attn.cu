@@ -28,8 +28,8 @@ constexpr int kMaxSplits = 128;    // partials one (stream, kv head) may have
 
 struct AttnDecArgs {
   const float* q;
-  const float* kc;
-  const float* vc;
+  const void* kc;   // fp32 or IEEE half elements (the kernel's KV parameter)
+  const void* vc;
   int B, H, Hk, cap;
   const int* dlen;
   int add;
@@ -49,7 +49,7 @@ int attn_decode_splits(int B, int Hk, int cap) {
   return s;
 }
 
-template <int HPG>
+template <int HPG, int KV>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a) {
   __shared__ float qs[HPG][64];
   __shared__ float Ks[kDecSub][65];
@@ -84,12 +84,10 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
 #pragma unroll
   for (int k = 0; k < kSlots; ++k) oacc[k] = 0.f;
 
-  const size_t head = ((size_t)b * a.Hk + g) * a.cap;
-  const float* kb = a.kc + head * 64;
-  const float* vb = a.vc + head * 64;
+  const size_t head = ((size_t)b * a.Hk + g) * a.cap * 64;   // first element of the head's rows
 
   // K/V of the next run of positions are loaded into registers while the current run is
-  // computed (each thread: float4 i = tid + 128 j of the run, j < 8)
+  // computed (each thread: elements 4f .. 4f + 3 of row p, i = tid + 128 j of the run, j < 8)
   constexpr int kPf = kDecSub * 16 / kDecThreads;
   float4 pk[kPf], pv[kPf];
   auto fetch = [&](int c0, int cn) {
@@ -97,8 +95,8 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
     for (int j = 0; j < kPf; ++j) {
       const int i = tid + j * kDecThreads, p = i >> 4, f = i & 15;
       if (p < cn) {
-        pk[j] = reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64)[f];
-        pv[j] = reinterpret_cast<const float4*>(vb + (size_t)(c0 + p) * 64)[f];
+        pk[j] = kv_load4<KV>(a.kc, head + (size_t)(c0 + p) * 64 + 4 * f);
+        pv[j] = kv_load4<KV>(a.vc, head + (size_t)(c0 + p) * 64 + 4 * f);
       }
     }
   };
@@ -214,12 +212,14 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
 }
 
 template <int HPG>
-static cudaError_t attn_dec_go(const Launch& L, const AttnDecArgs& a) {
-  return launch_k(L, attn_decode_kernel<HPG>, dim3(a.splits, a.Hk, a.B), dim3(kDecThreads), 0, a);
+static cudaError_t attn_dec_go(const Launch& L, const AttnDecArgs& a, int kv16) {
+  if (kv16) return launch_k(L, attn_decode_kernel<HPG, 1>, dim3(a.splits, a.Hk, a.B), dim3(kDecThreads), 0, a);
+  return launch_k(L, attn_decode_kernel<HPG, 0>, dim3(a.splits, a.Hk, a.B), dim3(kDecThreads), 0, a);
 }
 
-cudaError_t launch_attn_decode(const Launch& L, const float* q, const float* kc, const float* vc, int B, int H,
-                               int Hk, int cap, const int* dlen, int add, const AttnDecodeWork& w, float* o) {
+cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, const void* vc, int B, int H,
+                               int Hk, int cap, const int* dlen, int add, const AttnDecodeWork& w, float* o,
+                               int kv16) {
   AttnDecArgs a;
   a.q = q;
   a.kc = kc;
@@ -235,12 +235,12 @@ cudaError_t launch_attn_decode(const Launch& L, const float* q, const float* kc,
   a.counters = w.counters;
   a.o = o;
   switch (H / Hk) {
-    case 1: return attn_dec_go<1>(L, a);
-    case 2: return attn_dec_go<2>(L, a);
-    case 3: return attn_dec_go<3>(L, a);
-    case 4: return attn_dec_go<4>(L, a);
-    case 6: return attn_dec_go<6>(L, a);
-    case 8: return attn_dec_go<8>(L, a);
+    case 1: return attn_dec_go<1>(L, a, kv16);
+    case 2: return attn_dec_go<2>(L, a, kv16);
+    case 3: return attn_dec_go<3>(L, a, kv16);
+    case 4: return attn_dec_go<4>(L, a, kv16);
+    case 6: return attn_dec_go<6>(L, a, kv16);
+    case 8: return attn_dec_go<8>(L, a, kv16);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -257,8 +257,8 @@ constexpr int kPrePad = kPreT + 4;
 
 struct AttnPreArgs {
   const float* q;
-  const float* kc;
-  const float* vc;
+  const void* kc;   // fp32 or IEEE half elements (the kernel's KV parameter)
+  const void* vc;
   int B, n, H, Hk, cap;
   const int* dlen;
   float* o;
@@ -267,6 +267,7 @@ struct AttnPreArgs {
 constexpr size_t kPreSmem = sizeof(float) * (3 * 64 * kPrePad + 64 * 64);
 }  // namespace
 
+template <int KV>
 __global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
   extern __shared__ __align__(16) float sm[];
   float(*Qs)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm);                   // [d][row]
@@ -302,9 +303,7 @@ __global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) O[i][j] = 0.f;
   }
-  const size_t head = ((size_t)b * a.Hk + g) * a.cap;
-  const float* kb = a.kc + head * 64;
-  const float* vb = a.vc + head * 64;
+  const size_t head = ((size_t)b * a.Hk + g) * a.cap * 64;   // first element of the head's rows
 
   for (int c0 = 0; c0 < kend; c0 += kPreT) {
     __syncthreads();
@@ -312,8 +311,8 @@ __global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
       const int r = idx >> 4, f = idx & 15;
       float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
       if (c0 + r < kend) {
-        kv = reinterpret_cast<const float4*>(kb + (size_t)(c0 + r) * 64)[f];
-        vv = reinterpret_cast<const float4*>(vb + (size_t)(c0 + r) * 64)[f];
+        kv = kv_load4<KV>(a.kc, head + (size_t)(c0 + r) * 64 + 4 * f);
+        vv = kv_load4<KV>(a.vc, head + (size_t)(c0 + r) * 64 + 4 * f);
       }
       Ks[4 * f + 0][r] = kv.x;
       Ks[4 * f + 1][r] = kv.y;
@@ -392,10 +391,14 @@ __global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
   }
 }
 
-cudaError_t init_attrs_attn() { return allow_smem(attn_prefill_kernel, kMaxDynSmem); }
+cudaError_t init_attrs_attn() {
+  cudaError_t e = allow_smem(attn_prefill_kernel<0>, kMaxDynSmem);
+  if (e == cudaSuccess) e = allow_smem(attn_prefill_kernel<1>, kMaxDynSmem);
+  return e;
+}
 
-cudaError_t launch_attn_prefill(const Launch& L, const float* q, const float* kc, const float* vc, int B, int n,
-                                int H, int Hk, int cap, const int* dlen, float* o) {
+cudaError_t launch_attn_prefill(const Launch& L, const float* q, const void* kc, const void* vc, int B, int n,
+                                int H, int Hk, int cap, const int* dlen, float* o, int kv16) {
   if (n <= 0) return cudaSuccess;
   AttnPreArgs a;
   a.q = q;
@@ -408,7 +411,9 @@ cudaError_t launch_attn_prefill(const Launch& L, const float* q, const float* kc
   a.cap = cap;
   a.dlen = dlen;
   a.o = o;
-  return launch_k(L, attn_prefill_kernel, dim3((n + kPreT - 1) / kPreT, H, B), dim3(256), kPreSmem, a);
+  const dim3 grid((n + kPreT - 1) / kPreT, H, B);
+  if (kv16) return launch_k(L, attn_prefill_kernel<1>, grid, dim3(256), kPreSmem, a);
+  return launch_k(L, attn_prefill_kernel<0>, grid, dim3(256), kPreSmem, a);
 }
 
 }  // namespace ms

@@ -775,7 +775,7 @@ __device__ __forceinline__ void att_split_count(int T, int S, int& s_act, int& c
 // (m, l, o) per head as stamped words (epoch ep_out) for the merge.  Returns false on a
 // failed wait.
 __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scratch, int b, int g, int split, int S,
-                                            int s_act, int chunk, int T, int pos, float* kc, float* vc, unsigned ep,
+                                            int s_act, int chunk, int T, int pos, void* kc, void* vc, unsigned ep,
                                             unsigned ep_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = a.H, Hk = a.Hk, hpg = H / Hk;
@@ -795,9 +795,8 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
   const uint64_t* row = a.vs[0] + (size_t)b * nq;   // QKV is one slice
   const float* cs = a.cosv + (size_t)pos * 32;
   const float* sn = a.sinv + (size_t)pos * 32;
-  const size_t head = ((size_t)b * Hk + g) * a.cap;
-  float* kb = kc + head * 64;
-  float* vb = vc + head * 64;
+  const size_t head = ((size_t)b * Hk + g) * a.cap * 64;   // first element of the head's rows
+  const bool h16 = a.kv16 != 0;
   if (tid < 8) {
     mh[tid] = -INFINITY;
     lh[tid] = 0.f;
@@ -807,12 +806,13 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     for (int i = tid; i < cn * 16; i += kThreads) {
       const int p = i >> 4, f = i & 15;
       if (c0 + p == pos) continue;  // the new position comes from qkv
-      const float4 kv = __ldcg(reinterpret_cast<const float4*>(kb + (size_t)(c0 + p) * 64) + f);
+      const size_t e = head + (size_t)(c0 + p) * 64 + 4 * f;
+      const float4 kv = h16 ? kv_load4<1>(kc, e) : kv_load4<0>(kc, e);
       Ks[p * 65 + 4 * f + 0] = kv.x;
       Ks[p * 65 + 4 * f + 1] = kv.y;
       Ks[p * 65 + 4 * f + 2] = kv.z;
       Ks[p * 65 + 4 * f + 3] = kv.w;
-      reinterpret_cast<float4*>(Vs + p * 64)[f] = __ldcg(reinterpret_cast<const float4*>(vb + (size_t)(c0 + p) * 64) + f);
+      reinterpret_cast<float4*>(Vs + p * 64)[f] = h16 ? kv_load4<1>(vc, e) : kv_load4<0>(vc, e);
     }
   };
   stage(t0, min(kAttSub, t1 - t0));
@@ -841,17 +841,31 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     qs[qh * 64 + qj + 32] = (x0 * s + x1 * c) * 0.125f;
   }
   if (use[2]) {
-    const float v = __uint_as_float((unsigned)w[2]);
+    // the new row: appended to the cache, and used by this step in the cache's precision
+    const size_t e = head + (size_t)pos * 64;
+    float v = __uint_as_float((unsigned)w[2]);
+    if (h16) {
+      v = __half2float(__float2half_rn(v));
+      kv_store<1>(vc, e + tid, v);
+    } else {
+      kv_store<0>(vc, e + tid, v);
+    }
     vnew[tid] = v;
-    vb[(size_t)pos * 64 + tid] = v;
     if (use[3]) {
       const float x0 = __uint_as_float((unsigned)w[3]), x1 = __uint_as_float((unsigned)w[4]);
       const float c = cs[tid], s = sn[tid];
-      const float k0 = x0 * c - x1 * s, k1 = x0 * s + x1 * c;
+      float k0 = x0 * c - x1 * s, k1 = x0 * s + x1 * c;
+      if (h16) {
+        k0 = __half2float(__float2half_rn(k0));
+        k1 = __half2float(__float2half_rn(k1));
+        kv_store<1>(kc, e + tid, k0);
+        kv_store<1>(kc, e + tid + 32, k1);
+      } else {
+        kv_store<0>(kc, e + tid, k0);
+        kv_store<0>(kc, e + tid + 32, k1);
+      }
       knew[tid] = k0;
       knew[tid + 32] = k1;
-      kb[(size_t)pos * 64 + tid] = k0;
-      kb[(size_t)pos * 64 + tid + 32] = k1;
     }
   }
   if (consumer_bar_or(!ok)) return false;
@@ -1171,8 +1185,9 @@ __device__ __forceinline__ bool decode_steps(const PersistArgs& a, Ring& ring, c
     att_split_count(T, S, s_act, chunk);
     for (int l = 0; l < a.L; ++l) {
       const PLayer& ly = layers[l];
-      float* kc = a.kc + (size_t)l * a.layer_stride;
-      float* vc = a.vc + (size_t)l * a.layer_stride;
+      const size_t es = a.kv16 ? 2 : 4;
+      void* kc = static_cast<char*>(a.kc) + (size_t)l * a.layer_stride * es;
+      void* vc = static_cast<char*>(a.vc) + (size_t)l * a.layer_stride * es;
       const unsigned epA = ep0 + 5u * l;
       // phases A (LN1 + QKV), B (attention), C (O + residual), D (LN2 + FC1 + GELU),
       // E (FC2 + residual); one call site for the four matrix phases

@@ -208,13 +208,15 @@ cudaError_t launch_skipln(const Launch& L, float* x, const float* y, const float
 // post-RoPE k and of v at the row's position into the fixed-capacity cache
 // ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model variant: past and present
 // share one preallocated buffer).  Positions are implicit: len + i for the i-th new row
-// ("MuScriptor small — ONNX conversion", muscriptor-small-lm.onnx).
+// ("MuScriptor small — ONNX conversion", muscriptor-small-lm.onnx).  The cache holds fp32
+// (KV = 0) or, in the half-precision cache option, the IEEE half of each value (KV = 1).
 // ---------------------------------------------------------------------------------
+template <int KV>
 __global__ void __launch_bounds__(128) rope_append_kernel(const float* __restrict__ qkv, int n, int H, int Hk,
                                                           const float* __restrict__ cosv,
                                                           const float* __restrict__ sinv, const int* __restrict__ dlen,
-                                                          float* __restrict__ q_out, float* __restrict__ kc,
-                                                          float* __restrict__ vc, int cap, unsigned* status) {
+                                                          float* __restrict__ q_out, void* __restrict__ kc,
+                                                          void* __restrict__ vc, int cap, unsigned* status) {
   pdl_wait();
   pdl_trigger();
   const int r = blockIdx.x;
@@ -239,21 +241,25 @@ __global__ void __launch_bounds__(128) rope_append_kernel(const float* __restric
       dst[j] = a2;
       dst[j + 32] = b2;
     } else {
-      float* dst = kc + (((size_t)b * Hk + (hh - H)) * cap + pos) * 64;
-      dst[j] = a2;
-      dst[j + 32] = b2;
+      const size_t e = (((size_t)b * Hk + (hh - H)) * cap + pos) * 64;
+      kv_store<KV>(kc, e + j, a2);
+      kv_store<KV>(kc, e + j + 32, b2);
     }
   }
   for (int idx = threadIdx.x; idx < Hk * 64; idx += blockDim.x) {
     const int g = idx >> 6, dd = idx & 63;
-    vc[(((size_t)b * Hk + g) * cap + pos) * 64 + dd] = row[(H + Hk) * 64 + idx];
+    kv_store<KV>(vc, (((size_t)b * Hk + g) * cap + pos) * 64 + dd, row[(H + Hk) * 64 + idx]);
   }
 }
 
 cudaError_t launch_rope_append(const Launch& L, const float* qkv, int B, int n, int H, int Hk, const float* cosv,
-                               const float* sinv, const int* dlen, float* q_out, float* kc, float* vc, int cap) {
+                               const float* sinv, const int* dlen, float* q_out, void* kc, void* vc, int cap,
+                               int kv16) {
   if (B * n <= 0) return cudaSuccess;
-  return launch_k(L, rope_append_kernel, dim3(B * n), dim3(128), 0, qkv, n, H, Hk, cosv, sinv, dlen, q_out, kc, vc,
+  if (kv16)
+    return launch_k(L, rope_append_kernel<1>, dim3(B * n), dim3(128), 0, qkv, n, H, Hk, cosv, sinv, dlen, q_out, kc,
+                    vc, cap, L.status);
+  return launch_k(L, rope_append_kernel<0>, dim3(B * n), dim3(128), 0, qkv, n, H, Hk, cosv, sinv, dlen, q_out, kc, vc,
                   cap, L.status);
 }
 

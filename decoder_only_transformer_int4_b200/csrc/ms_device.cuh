@@ -128,6 +128,23 @@ __device__ __forceinline__ float nib_to_q(uint32_t u4) {
   return __int_as_float(0x4B000000u | u4) - 8388616.0f;
 }
 
+// ---- KV cache elements: fp32 (KV = 0) or IEEE half (KV = 1, round to nearest even) ---------
+// Four consecutive elements e .. e + 3 of a cache row as floats (16-byte / 8-byte loads,
+// through L2: the rows may have been written by another CTA of the same kernel).
+template <int KV>
+__device__ __forceinline__ float4 kv_load4(const void* base, size_t e) {
+  if (KV == 0) return __ldcg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + e));
+  const uint2 u = __ldcg(reinterpret_cast<const uint2*>(static_cast<const __half*>(base) + e));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+template <int KV>
+__device__ __forceinline__ void kv_store(void* base, size_t e, float v) {
+  if (KV == 0) static_cast<float*>(base)[e] = v;
+  else static_cast<__half*>(base)[e] = __float2half_rn(v);
+}
+
 __device__ __forceinline__ float gelu_erf(float u) {
   return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
 }

@@ -67,9 +67,11 @@ cudaError_t launch_skipln(const Launch& L, float* x, const float* y, const float
 
 // RoPE on the q and k parts of qkv rows (row r = b * n + i at position len + i, len read
 // from dlen) and append post-RoPE k and v to the layer's cache slices.
+// The cache elements are fp32, or IEEE halves with kv16 (every kernel that touches the cache
+// takes the same flag).
 cudaError_t launch_rope_append(const Launch& L, const float* qkv, int B, int n, int H, int Hk,
                                const float* cosv, const float* sinv, const int* dlen, float* q_out,
-                               float* kc, float* vc, int cap);
+                               void* kc, void* vc, int cap, int kv16);
 
 // Smallest-M path (decode): M <= 8.  Optional LayerNorm of x in the prologue (ln_g != null).
 cudaError_t launch_gemv(const Launch& L, const WView& w, const float* x, int ldx, int M,
@@ -104,6 +106,15 @@ cudaError_t launch_split_f16(const Launch& L, const float* x, int ldx, int M, in
                              int ldh);
 cudaError_t init_attrs_gemm_f16();
 
+// W4A8 (accuracy_level=4 reading): INT8 activation codes per 32-element block (q [M][ldq],
+// scales [M][lds]) and the MatMul on them (dp4a GEMV for M in {1, 2, 4, 8}, dp4a tiled GEMM
+// otherwise); INT4 weights only, K a multiple of 128, ldqa a multiple of 16.
+cudaError_t launch_quantize_act_int8(const Launch& L, const float* x, int ldx, int M, int K, int8_t* q, int ldq,
+                                     float* s, int lds);
+cudaError_t launch_matmul_w4a8(const Launch& L, const WView& w, const int8_t* qa, int ldqa, const float* sa, int ldsa,
+                               int M, float* y, int ldy, int epi, int sms);
+cudaError_t init_attrs_w4a8();
+
 // Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
 // the combine done by the last CTA of each (stream, kv head).
 struct AttnDecodeWork {
@@ -111,14 +122,14 @@ struct AttnDecodeWork {
   unsigned* counters; // [B][Hk], zero between launches
   int splits;         // grid splits (max)
 };
-cudaError_t launch_attn_decode(const Launch& L, const float* q, const float* kc, const float* vc,
+cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, const void* vc,
                                int B, int H, int Hk, int cap, const int* dlen, int add,
-                               const AttnDecodeWork& w, float* o);
+                               const AttnDecodeWork& w, float* o, int kv16);
 int attn_decode_splits(int B, int Hk, int cap);
 
 // Causal prefill attention for n new rows per stream at positions len .. len + n - 1.
-cudaError_t launch_attn_prefill(const Launch& L, const float* q, const float* kc, const float* vc,
-                                int B, int n, int H, int Hk, int cap, const int* dlen, float* o);
+cudaError_t launch_attn_prefill(const Launch& L, const float* q, const void* kc, const void* vc,
+                                int B, int n, int H, int Hk, int cap, const int* dlen, float* o, int kv16);
 
 // LM head + argmax over rows x[m * ldx], m < M.  Writes logits (may be null), argmax
 // (may be null), hist[(len + hist_off) * B + m] (may be null) and, in its last CTA,

@@ -21,9 +21,10 @@ struct PersistArgs {
   const float* lnf_b;
   const PLayer* layers;      // device array [L]
   int cap;
-  float* kc;                 // K cache base; layer l at kc + l * layer_stride
-  float* vc;
-  size_t layer_stride;
+  void* kc;                  // K cache base; layer l at element l * layer_stride
+  void* vc;
+  size_t layer_stride;       // elements
+  int kv16;                  // cache elements are IEEE halves (else fp32)
   const float* cosv;         // RoPE table [cap][32]
   const float* sinv;
   int* dlen;                 // cache length (device)

@@ -144,6 +144,7 @@ cudaError_t ensure_kernel_attributes() {
   if (e == cudaSuccess) e = ms::init_attrs_attn();
   if (e == cudaSuccess) e = ms::init_attrs_persistent();
   if (e == cudaSuccess) e = ms::init_attrs_gemm_f16();
+  if (e == cudaSuccess) e = ms::init_attrs_w4a8();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -169,7 +170,8 @@ struct ms_cache {
   int B = 0, cap = 0, len = 0;
   bool has_next = false;  // hist holds the argmax of position len - 1
   Arena arena;
-  float *k = nullptr, *v = nullptr;        // [L][B][Hk][cap][64]
+  void *k = nullptr, *v = nullptr;         // [L][B][Hk][cap][64] fp32, or IEEE half with kv16
+  int kv16 = 0;                            // the cache holds IEEE halves
   float *cosv = nullptr, *sinv = nullptr;  // [cap][32]
   int* dlen = nullptr;
   int32_t* hist = nullptr;                 // [cap][B]
@@ -184,6 +186,10 @@ struct ms_cache {
   __half *hh = nullptr, *hl = nullptr;     // GEMM operand planes [rows][kh] (LayerNorm or attention output)
   __half *uh = nullptr, *ul = nullptr;     // FC1's GELU output as planes [rows][d_ff] (they share u's memory)
   int kh = 0;                              // row stride of hh / hl: max(d, H * 64)
+  int act_int8 = 0;                        // W4A8: backbone MatMuls on INT8 activation codes
+  int8_t* qa = nullptr;                    // INT8 activation codes [rows][ka]
+  float* sa = nullptr;                     // their block scales [rows][ka / 32]
+  int ka = 0;                              // max(d, H * 64, d_ff)
   float* logits = nullptr;                 // [B][V] internal
   size_t rows_cap = 0;
   cudaGraphExec_t gen_exec = nullptr;
@@ -216,6 +222,19 @@ size_t layer_stride(const ms_cache* c) {
 
 ms::Launch launch_of(ms_cache* c, cudaStream_t s, bool pdl) { return ms::Launch{s, pdl, c->status}; }
 
+// Layer l of a cache buffer (K or V): fp32 or half elements.
+void* kv_layer(const ms_cache* c, void* base, int l) {
+  return static_cast<char*>(base) + (size_t)l * layer_stride(c) * (c->kv16 ? sizeof(__half) : sizeof(float));
+}
+
+// W4A8: quantise fp32 rows x [R][ldx] (K columns) to the cache's INT8 codes, then MatMul i.
+cudaError_t w4a8(const ms::Launch& L, ms_cache* c, const ms::WView& w, const float* x, int ldx, int R, float* y,
+                 int ldy, int epi) {
+  cudaError_t e = ms::launch_quantize_act_int8(L, x, ldx, R, w.K, c->qa, c->ka, c->sa, c->ka / 32);
+  if (e == cudaSuccess) e = ms::launch_matmul_w4a8(L, w, c->qa, c->ka, c->sa, c->ka / 32, R, y, ldy, epi, c->nsm);
+  return e;
+}
+
 // ---- one decoder call, kernel by kernel ----------------------------------------------
 // Prefill of n = P + S rows per stream.  Rows of stream b are b * n + i.
 cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, const float* prefix, int P,
@@ -227,10 +246,25 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
   ms::Launch L0 = launch_of(c, st, false), L = launch_of(c, st, true);
   cudaError_t e = ms::launch_embed_prefill(L0, tokens, S, prefix, P, m->tok_emb, g.vocab, d, B, c->x);
   const int kh = c->kh, F = g.d_ff;
-  for (int l = 0; l < g.n_layers && e == cudaSuccess; ++l) {
+  for (int l = 0; l < g.n_layers && e == cudaSuccess && c->act_int8; ++l) {
+    // W4A8: each backbone MatMul on the INT8 codes of its fp32 input
     const DevLayer& ly = m->layers[l];
-    float* kc = c->k + l * layer_stride(c);
-    float* vc = c->v + l * layer_stride(c);
+    void* kc = kv_layer(c, c->k, l);
+    void* vc = kv_layer(c, c->v, l);
+    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
+    if (e == cudaSuccess)
+      e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
+    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, c->kv16);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], c->h, d, R, c->u, F, ms::kGelu);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], c->u, F, R, c->y, d, ms::kStore);
+  }
+  for (int l = 0; l < g.n_layers && e == cudaSuccess && !c->act_int8; ++l) {
+    const DevLayer& ly = m->layers[l];
+    void* kc = kv_layer(c, c->k, l);
+    void* vc = kv_layer(c, c->v, l);
     // LN1 -> planes -> QKV -> RoPE + append -> attention -> planes -> O -> SkipLN2 -> planes
     // -> FC1 + GELU -> planes -> FC2
     if (e == cudaSuccess)
@@ -238,8 +272,9 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
                             kh);
     if (e == cudaSuccess)
       e = ms::launch_gemm_f16(L, ly.w[0], ly.gw[0], c->hh, c->hl, kh, R, c->qkv, nq, nullptr, nullptr, 0, ms::kStore, &gw);
-    if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
-    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o);
+    if (e == cudaSuccess)
+      e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
+    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, c->kv16);
     if (e == cudaSuccess) e = ms::launch_split_f16(L, c->o, H * 64, R, H * 64, c->hh, c->hl, kh);
     if (e == cudaSuccess)
       e = ms::launch_gemm_f16(L, ly.w[1], ly.gw[1], c->hh, c->hl, kh, R, c->y, d, nullptr, nullptr, 0, ms::kStore, &gw);
@@ -273,10 +308,24 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
   cudaError_t e = ms::launch_embed_decode(L0, tokens, c->hist, c->dlen, m->tok_emb, g.vocab, d, B, c->x);
   for (int l = 0; l < g.n_layers && e == cudaSuccess; ++l) {
     const DevLayer& ly = m->layers[l];
-    float* kc = c->k + l * layer_stride(c);
-    float* vc = c->v + l * layer_stride(c);
+    void* kc = kv_layer(c, c->k, l);
+    void* vc = kv_layer(c, c->v, l);
     const bool gv = small && ms::gemv_fits(ly.w[0], B) && ms::gemv_fits(ly.w[1], B) && ms::gemv_fits(ly.w[2], B) &&
                     ms::gemv_fits(ly.w[3], B);
+    if (c->act_int8) {
+      // W4A8: each backbone MatMul on the INT8 codes of its fp32 input
+      e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
+      if (e == cudaSuccess)
+        e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
+      if (e == cudaSuccess)
+        e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o, c->kv16);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
+      continue;
+    }
     if (gv) {
       e = ms::launch_gemv(L, ly.w[0], c->x, d, B, ly.ln1_g, ly.ln1_b, g.ln_eps, c->qkv, nq, ms::kStore);
     } else {
@@ -285,8 +334,9 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
         e = ms::launch_gemm_f16(L, ly.w[0], ly.gw[0], c->hh, c->hl, c->kh, B, c->qkv, nq, nullptr, nullptr, 0, ms::kStore,
                                 &gw);
     }
-    if (e == cudaSuccess) e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap);
-    if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o);
+    if (e == cudaSuccess)
+      e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
+    if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o, c->kv16);
     if (gv) {
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[1], c->o, H * 64, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
@@ -311,7 +361,7 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
 }
 
 bool use_persistent(const ms_cache* c) {
-  if (c->path_request == 2) return false;
+  if (c->path_request == 2 || c->act_int8) return false;
   return c->persist_grid > 0;
 }
 
@@ -349,6 +399,7 @@ cudaError_t run_persistent(ms_model* m, ms_cache* c, const int32_t* tokens, int 
   a.cap = c->cap;
   a.kc = c->k;
   a.vc = c->v;
+  a.kv16 = c->kv16;
   a.layer_stride = layer_stride(c);
   a.cosv = c->cosv;
   a.sinv = c->sinv;
@@ -406,8 +457,14 @@ ms_status ms_quantize_int4_g32(const float* w, int N, int K, uint8_t* packed, fl
 }
 
 size_t ms_cache_kv_bytes(const ms_config* cfg, int batch, int capacity) {
+  return ms_cache_kv_bytes_ex(cfg, batch, capacity, MS_KV_F32);
+}
+
+size_t ms_cache_kv_bytes_ex(const ms_config* cfg, int batch, int capacity, int kv_format) {
   if (!cfg || batch < 1 || capacity < 1 || cfg->n_layers < 0 || cfg->n_kv_heads < 1) return 0;
-  return (size_t)2 * cfg->n_layers * batch * cfg->n_kv_heads * (size_t)capacity * 64 * sizeof(float);
+  if (kv_format != MS_KV_F32 && kv_format != MS_KV_F16) return 0;
+  const size_t es = kv_format == MS_KV_F16 ? 2 : 4;
+  return (size_t)2 * cfg->n_layers * batch * cfg->n_kv_heads * (size_t)capacity * 64 * es;
 }
 
 ms_status ms_model_create(const ms_config* cfg, const ms_weights* wt, int device, ms_model** out) {
@@ -573,15 +630,24 @@ ms_status ms_model_destroy(ms_model* m) {
 size_t ms_model_weight_bytes(const ms_model* m) { return m ? m->arena.used : 0; }
 
 ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) {
+  return ms_cache_create_ex(m, batch, capacity, MS_KV_F32, out);
+}
+
+int ms_cache_kv_format(const ms_cache* c) { return c ? (c->kv16 ? MS_KV_F16 : MS_KV_F32) : -1; }
+
+ms_status ms_cache_create_ex(ms_model* m, int batch, int capacity, int kv_format, ms_cache** out) {
   if (!m || !out) return fail(MS_ERR_INVALID_ARG, "ms_cache_create: null argument");
   *out = nullptr;
   if (batch < 1 || batch > 64) return fail(MS_ERR_SHAPE, "ms_cache_create: batch must be in [1, 64]");
   if (capacity < 1) return fail(MS_ERR_SHAPE, "ms_cache_create: capacity must be >= 1");
+  if (kv_format != MS_KV_F32 && kv_format != MS_KV_F16)
+    return fail(MS_ERR_INVALID_ARG, "ms_cache_create_ex: unknown kv_format %d", kv_format);
   DeviceGuard dg(m->device);
   const ms_config& g = m->cfg;
   ms_cache* c = new (std::nothrow) ms_cache;
   if (!c) return fail(MS_ERR_OOM, "ms_cache_create: host allocation failed");
   c->m = m;
+  c->kv16 = kv_format == MS_KV_F16;
   c->B = batch;
   c->cap = capacity;
   c->splits = ms::attn_decode_splits(batch, g.n_kv_heads, capacity);
@@ -628,8 +694,9 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
   for (int pass = 0; pass < 2; ++pass) {
     Arena& a = c->arena;
     a.used = 0;
-    c->k = a.take<float>((size_t)g.n_layers * layer_stride(c) + 64);
-    c->v = a.take<float>((size_t)g.n_layers * layer_stride(c) + 64);
+    const size_t es = c->kv16 ? sizeof(__half) : sizeof(float);
+    c->k = a.take<unsigned char>(((size_t)g.n_layers * layer_stride(c) + 64) * es);
+    c->v = a.take<unsigned char>(((size_t)g.n_layers * layer_stride(c) + 64) * es);
     c->cosv = a.take<float>((size_t)capacity * 32);
     c->sinv = a.take<float>((size_t)capacity * 32);
     c->dlen = a.take<int>(4);
@@ -674,6 +741,9 @@ ms_status ms_cache_create(ms_model* m, int batch, int capacity, ms_cache** out) 
     c->kh = std::max(g.d_model, g.n_heads * 64);
     c->hh = a.take<__half>(R * c->kh);
     c->hl = a.take<__half>(R * c->kh);
+    c->ka = std::max(c->kh, g.d_ff);
+    c->qa = a.take<int8_t>(R * c->ka);
+    c->sa = a.take<float>(R * (c->ka / 32));
     c->uh = reinterpret_cast<__half*>(c->u);
     c->ul = c->uh ? c->uh + R * g.d_ff : nullptr;
     c->logits = a.take<float>((size_t)batch * g.vocab);
@@ -751,6 +821,8 @@ ms_status ms_cache_set_decode_path(ms_cache* c, int path) {
   if (path < 0 || path > 2) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_decode_path: path must be 0, 1 or 2");
   if (path == 1 && c->persist_grid == 0)
     return fail(MS_ERR_UNSUPPORTED, "ms_cache_set_decode_path: the persistent kernel does not fit this model/batch");
+  if (path == 1 && c->act_int8)
+    return fail(MS_ERR_UNSUPPORTED, "ms_cache_set_decode_path: INT8 activations run one kernel per operation");
   c->path_request = path;
   return MS_OK;
 }
@@ -765,6 +837,23 @@ ms_status ms_cache_set_guidance(ms_cache* c, float scale) {
 }
 
 float ms_cache_guidance(const ms_cache* c) { return c ? c->guidance : 0.f; }
+
+ms_status ms_cache_set_act_int8(ms_cache* c, int on) {
+  if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_act_int8: null cache");
+  if (on && c->m->cfg.weight_format != MS_W_INT4_G32)
+    return fail(MS_ERR_UNSUPPORTED, "ms_cache_set_act_int8: INT8 activations go with INT4 weights");
+  if (on && c->path_request == 1)
+    return fail(MS_ERR_UNSUPPORTED, "ms_cache_set_act_int8: the persistent decode path was requested on this cache");
+  if (!!on != !!c->act_int8 && c->gen_exec) {
+    // the captured decode graph belongs to the other arithmetic
+    cudaGraphExecDestroy(c->gen_exec);
+    c->gen_exec = nullptr;
+  }
+  c->act_int8 = on ? 1 : 0;
+  return MS_OK;
+}
+
+int ms_cache_act_int8(const ms_cache* c) { return c ? c->act_int8 : -1; }
 
 ms_status ms_cache_set_wait_limits(ms_cache* c, long long polls, int stall) {
   if (!c) return fail(MS_ERR_INVALID_ARG, "ms_cache_set_wait_limits: null cache");
@@ -894,23 +983,38 @@ ms_status ms_generate(ms_model* m, ms_cache* c, int n_steps, int32_t* out_tokens
   return MS_OK;
 }
 
+// Host-side conversion between fp32 and IEEE half (round to nearest even), for the cache
+// transfer calls of a half-precision cache.
+namespace {
+uint16_t f32_to_f16_bits(float f) { return __half_as_ushort(__float2half_rn(f)); }
+float f16_bits_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+}  // namespace
+
 ms_status ms_cache_export(const ms_cache* c, float* k, float* v) {
   if (!c || !k || !v) return fail(MS_ERR_INVALID_ARG, "ms_cache_export: null argument");
   DeviceGuard dg(c->m->device);
   CUDA_TRY(cudaDeviceSynchronize());
   const ms_config& g = c->m->cfg;
   const int T = c->len, Hk = g.n_kv_heads;
-  std::vector<float> buf((size_t)T * 64);
+  const size_t es = c->kv16 ? sizeof(__half) : sizeof(float);
+  std::vector<unsigned char> buf((size_t)T * 64 * es);
   for (int which = 0; which < 2; ++which) {
-    const float* src = which ? c->v : c->k;
+    void* src = which ? c->v : c->k;
     float* dst = which ? v : k;
     for (int l = 0; l < g.n_layers; ++l)
       for (int b = 0; b < c->B; ++b)
         for (int gg = 0; gg < Hk; ++gg) {
-          const float* s = src + l * layer_stride(c) + (((size_t)b * Hk + gg) * c->cap) * 64;
-          if (T > 0) CUDA_TRY(cudaMemcpy(buf.data(), s, (size_t)T * 64 * 4, cudaMemcpyDeviceToHost));
-          for (int t = 0; t < T; ++t)
-            memcpy(dst + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64, buf.data() + (size_t)t * 64, 64 * 4);
+          const char* s = static_cast<const char*>(kv_layer(c, src, l)) + (((size_t)b * Hk + gg) * c->cap) * 64 * es;
+          if (T > 0) CUDA_TRY(cudaMemcpy(buf.data(), s, (size_t)T * 64 * es, cudaMemcpyDeviceToHost));
+          for (int t = 0; t < T; ++t) {
+            float* o = dst + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64;
+            if (c->kv16) {
+              const uint16_t* hb = reinterpret_cast<const uint16_t*>(buf.data()) + (size_t)t * 64;
+              for (int e = 0; e < 64; ++e) o[e] = f16_bits_to_f32(hb[e]);
+            } else {
+              memcpy(o, buf.data() + (size_t)t * 64 * 4, 64 * 4);
+            }
+          }
         }
   }
   return MS_OK;
@@ -923,17 +1027,25 @@ ms_status ms_cache_import(ms_cache* c, const float* k, const float* v, int T) {
   CUDA_TRY(cudaDeviceSynchronize());
   const ms_config& g = c->m->cfg;
   const int Hk = g.n_kv_heads;
-  std::vector<float> buf((size_t)T * 64);
+  const size_t es = c->kv16 ? sizeof(__half) : sizeof(float);
+  std::vector<unsigned char> buf((size_t)T * 64 * es);
   for (int which = 0; which < 2; ++which) {
-    float* dst = which ? c->v : c->k;
+    void* dst = which ? c->v : c->k;
     const float* src = which ? v : k;
     for (int l = 0; l < g.n_layers; ++l)
       for (int b = 0; b < c->B; ++b)
         for (int gg = 0; gg < Hk; ++gg) {
-          for (int t = 0; t < T; ++t)
-            memcpy(buf.data() + (size_t)t * 64, src + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64, 64 * 4);
-          float* d = dst + l * layer_stride(c) + (((size_t)b * Hk + gg) * c->cap) * 64;
-          if (T > 0) CUDA_TRY(cudaMemcpy(d, buf.data(), (size_t)T * 64 * 4, cudaMemcpyHostToDevice));
+          for (int t = 0; t < T; ++t) {
+            const float* in = src + ((((size_t)l * c->B + b) * T + t) * Hk + gg) * 64;
+            if (c->kv16) {
+              uint16_t* hb = reinterpret_cast<uint16_t*>(buf.data()) + (size_t)t * 64;
+              for (int e = 0; e < 64; ++e) hb[e] = f32_to_f16_bits(in[e]);
+            } else {
+              memcpy(buf.data() + (size_t)t * 64 * 4, in, 64 * 4);
+            }
+          }
+          char* d = static_cast<char*>(kv_layer(c, dst, l)) + (((size_t)b * Hk + gg) * c->cap) * 64 * es;
+          if (T > 0) CUDA_TRY(cudaMemcpy(d, buf.data(), (size_t)T * 64 * es, cudaMemcpyHostToDevice));
         }
   }
   CUDA_TRY(cudaMemcpy(c->dlen, &T, sizeof(int), cudaMemcpyHostToDevice));
@@ -1021,6 +1133,29 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
   if ((M == 1 || M == 2 || M == 4 || M == 8) && ms::gemv_fits(w, M))
     return check_launch(ms::launch_gemv(L, w, x, K, M, nullptr, nullptr, 0.f, y, N, ms::kStore), "gemv");
   return op_gemm(w, x, M, y, (cudaStream_t)stream, "ms_op_matmul_f16");
+}
+
+ms_status ms_op_quantize_act_int8(const float* x, int ldx, int M, int K, int8_t* q, float* scales, void* stream) {
+  if (!x || !q || !scales) return fail(MS_ERR_INVALID_ARG, "ms_op_quantize_act_int8: null pointer");
+  if (M < 0 || K < 32 || K % 32 != 0 || ldx < K) return fail(MS_ERR_SHAPE, "ms_op_quantize_act_int8: need K a multiple of 32, ldx >= K");
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  return check_launch(ms::launch_quantize_act_int8(L, x, ldx, M, K, q, K, scales, K / 32), "quantize_act_int8");
+}
+
+ms_status ms_op_matmul_w4a8(const int8_t* qa, const float* sa, int M, int K, const uint8_t* packed, const float* scales,
+                            int N, float* y, void* stream) {
+  if (!qa || !sa || !packed || !scales || !y) return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_w4a8: null pointer");
+  if (M < 1 || N < 1 || K < 128 || K % 128 != 0) return fail(MS_ERR_SHAPE, "ms_op_matmul_w4a8: need M, N >= 1, K a multiple of 128");
+  if ((reinterpret_cast<uintptr_t>(qa) & 15) || (reinterpret_cast<uintptr_t>(packed) & 15))
+    return fail(MS_ERR_INVALID_ARG, "ms_op_matmul_w4a8: qa and packed must be 16-byte aligned");
+  CUDA_TRY(ensure_kernel_attributes());
+  int dev = 0, nsm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  ms::WView w{packed, scales, nullptr, N, K, ms::kInt4, K / 2, K / 32};
+  ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  return check_launch(ms::launch_matmul_w4a8(L, w, qa, K, sa, K / 32, M, y, N, ms::kStore, nsm > 0 ? nsm : 1),
+                      "matmul_w4a8");
 }
 
 ms_status ms_op_split_f16(const float* x, int ldx, int M, int K, uint16_t* x_hi, uint16_t* x_lo, int ldh,

@@ -120,12 +120,23 @@ ms_status ms_model_destroy(ms_model* model);
 /* Bytes of device memory the model's weights occupy; 0 on NULL. */
 size_t ms_model_weight_bytes(const ms_model* model);
 
+/* Element format of the KV cache.  F32 is the pages' ("MuScriptor Medium — optimized W4A32
+ * ONNX Runtime", Model variant: fp32 KV cache).  F16 stores each post-RoPE key and value as
+ * its IEEE half (round to nearest even) and halves the bytes every decode step reads; all
+ * arithmetic stays fp32 (the attention converts each half back to fp32). */
+typedef enum { MS_KV_F32 = 0, MS_KV_F16 = 1 } ms_kv_format;
+
 /* ---- cache -------------------------------------------------------------------------
  * A fixed-capacity fp32 KV cache for `batch` independent streams that advance together
  * (every call appends the same number of positions to each stream), plus the work
  * buffers one call needs.  Layout on the device: K and V each [L][batch][Hk][capacity][64].
  * Allocates device memory; length starts at 0.  Synchronous. */
 ms_status ms_cache_create(ms_model* model, int batch, int capacity, ms_cache** out);
+/* The same with the cache's element format (ms_kv_format); ms_cache_create is
+ * ms_cache_create_ex(..., MS_KV_F32, ...).  MS_ERR_INVALID_ARG for an unknown format. */
+ms_status ms_cache_create_ex(ms_model* model, int batch, int capacity, int kv_format, ms_cache** out);
+/* The cache's element format (ms_kv_format), -1 on NULL. */
+int ms_cache_kv_format(const ms_cache* cache);
 ms_status ms_cache_reset(ms_cache* cache); /* length = 0; no device work */
 int ms_cache_length(const ms_cache* cache);   /* positions held (host view), -1 on NULL */
 int ms_cache_capacity(const ms_cache* cache); /* positions per stream, -1 on NULL */
@@ -135,6 +146,8 @@ ms_status ms_cache_destroy(ms_cache* cache);
  * capacity * 64 * 4.  For the medium model with Hk = 16 and capacity 2504 this is the
  * W4A32 page's "about 469.5 MiB". Returns 0 on an invalid argument. */
 size_t ms_cache_kv_bytes(const ms_config* cfg, int batch, int capacity);
+/* The same for a cache of the given element format (half the bytes for MS_KV_F16). */
+size_t ms_cache_kv_bytes_ex(const ms_config* cfg, int batch, int capacity, int kv_format);
 
 /* ---- one decoder call ----------------------------------------------------------------
  * Prefill: appends P prefix rows followed by S token rows to every stream (positions
@@ -189,6 +202,21 @@ ms_status ms_cache_set_guidance(ms_cache* cache, float scale);
 /* The current guidance scale (0 when off or on NULL). */
 float ms_cache_guidance(const ms_cache* cache);
 
+/* W4A8 ("MuScriptor Medium — optimized W4A32 ONNX Runtime", Model variant: MatMulNBits with
+ * accuracy_level=4, activations quantised to INT8 at run time, INT32 accumulation).  With
+ * on != 0 the four backbone MatMuls of every layer, in prefill and decode, take their fp32
+ * input as INT8 codes: per 32-element block of a row, scale = absmax / 127 and
+ * q = clamp(rint(x / scale), -127, 127) (fp32 IEEE divisions, ties to even; an all-zero block
+ * has scale 0), the block's integer sum with the INT4 codes is exact and is multiplied by
+ * both scales, the blocks summed in fp32.  (The page does not state the block or the rule;
+ * this is the weight quantiser's rule at 127 levels.)  Attention, LayerNorm and the LM head
+ * stay fp32.  Decoding then runs one kernel per operation (ms_cache_set_decode_path(1) is
+ * refused).  MS_ERR_UNSUPPORTED for half weights or when the persistent path was requested.
+ * Host state only; applies to the next call. */
+ms_status ms_cache_set_act_int8(ms_cache* cache, int on);
+/* 1 when INT8 activations are on, 0 when off, -1 on NULL. */
+int ms_cache_act_int8(const ms_cache* cache);
+
 /* Wait limits of the persistent decode kernel, for tests of its failure path.  No passage of
  * the pages corresponds to this call.  Every wait of that kernel (a stamped activation word
  * from another CTA, the grid barrier between steps) gives up after a limit, sets the timeout
@@ -204,7 +232,8 @@ ms_status ms_cache_set_wait_limits(ms_cache* cache, long long polls, int stall);
 
 /* ---- cache transfer (host pointers, synchronous) --------------------------------------
  * Export in the pages' layout [L][batch][T][Hk][64] (T = current length);
- * import T positions in the same layout and set the length to T. */
+ * import T positions in the same layout and set the length to T.  Always fp32 on the host: a
+ * half-precision cache converts on the way (import rounds to nearest even). */
 ms_status ms_cache_export(const ms_cache* cache, float* k, float* v);
 ms_status ms_cache_import(ms_cache* cache, const float* k, const float* v, int T);
 
@@ -246,6 +275,16 @@ ms_status ms_op_matmul_f16(const float* x, int M, int K, const uint16_t* w16, in
  * cannot report it (the calls of a cache flag it in the status word, MS_ERR_SHAPE). */
 ms_status ms_op_split_f16(const float* x, int ldx, int M, int K, uint16_t* x_hi, uint16_t* x_lo, int ldh,
                           void* stream);
+
+/* The INT8 activation codes of the W4A8 reading (see ms_cache_set_act_int8): x fp32 rows of K
+ * at stride ldx -> q int8 [M][K] and scales fp32 [M][K/32].  K a multiple of 32. */
+ms_status ms_op_quantize_act_int8(const float* x, int ldx, int M, int K, int8_t* q, float* scales, void* stream);
+/* The W4A8 MatMul: y[m][n] = sum over blocks b of (sa[m][b] * s[n][b]) * (sum_{k in b}
+ * qa[m][k] * q[n][k]), y fp32 [M][N]; qa, sa as ms_op_quantize_act_int8 writes them, packed
+ * and scales as ms_quantize_int4_g32 writes them.  A dp4a GEMV for M in {1, 2, 4, 8}, a dp4a
+ * tiled GEMM otherwise.  K a multiple of 128; qa and packed 16-byte aligned. */
+ms_status ms_op_matmul_w4a8(const int8_t* qa, const float* sa, int M, int K, const uint8_t* packed,
+                            const float* scales, int N, float* y, void* stream);
 
 /* Backbone MatMul `which` (0 QKV, 1 O, 2 FC1, 3 FC2) of layer `layer` of the model, on M
  * activation rows given as ms_op_split_f16 planes (row stride ldx halves, a multiple of 8,

@@ -280,16 +280,25 @@ class OracleModel:
     weight variant of "MuScriptor for Core AI (.aimodel)", file table).  "fp32":
     the matrices as drawn.  Embeddings, LayerNorms and the LM head stay fp32.
 
+    ``kv_store`` "fp16" (the half-precision cache option; the pages keep the cache in fp32):
+    every post-RoPE key and every value is rounded to IEEE half, to nearest with ties to
+    even, when it enters the cache, and attention reads the rounded values (the current
+    position's included).  Everything else is unchanged.
+
     ``act_int8`` (INT4 format only): the four backbone MatMuls of every layer take
     their activations through :func:`matmul_w4a8` (the ``accuracy_level=4`` reading);
     attention and the LM head stay as they are, since only the backbone MatMuls are
     MatMulNBits nodes ([W4A32, "Model variant"]).
     """
 
-    def __init__(self, draw, weight_format: str = "int4", store=np.float64, act_int8: bool = False):
+    def __init__(self, draw, weight_format: str = "int4", store=np.float64, act_int8: bool = False,
+                 kv_store: str = "fp32"):
         sh = draw.shape
         self.shape = sh
         self.weight_format = weight_format
+        if kv_store not in ("fp32", "fp16"):
+            raise ValueError(kv_store)
+        self.kv_store = kv_store
         if act_int8 and weight_format != "int4":
             raise ValueError("int8 activations go with the INT4 weight format")
         self.act_int8 = act_int8
@@ -348,6 +357,9 @@ class OracleModel:
             v = qkv[:, (H + Hk) * hd:].reshape(n, Hk, hd)
             q = rope(q, pos, self.base)
             k = rope(k, pos, self.base)
+            if self.kv_store == "fp16":
+                k = k.astype(np.float16).astype(np.float64)
+                v = v.astype(np.float16).astype(np.float64)
             cache.k[l][t0: t0 + n] = k
             cache.v[l][t0: t0 + n] = v
             a = attention(q, cache.k[l][: t0 + n], cache.v[l][: t0 + n], pos, kpos)

@@ -798,3 +798,102 @@ def test_w4a8_planted_mistakes_are_caught(monkeypatch, name, attr, fn):
     g = _gold("a8_block_hand.json")
     caught = bool(_a8_hand_mismatches(g)) or _w4a8_bruteforce_err(54) > 1e-12
     assert caught, name
+
+
+# ---------------------------------------------------------------------------
+# Half-precision KV cache option (kv_store="fp16"): keys and values rounded to IEEE half,
+# to nearest with ties to even, when they enter the cache
+# ---------------------------------------------------------------------------
+
+def _f16_rne_bits(x: float) -> int:
+    """IEEE binary16 bits of x by the definition: sign, exponent and the 10-bit fraction
+    rounded to nearest, ties to the even fraction, subnormals below 2^-14 (no library
+    conversion involved)."""
+    import fractions
+    sign = 0x8000 if math.copysign(1.0, x) < 0 else 0
+    a = fractions.Fraction(abs(x))
+    if a == 0:
+        return sign
+    e = math.floor(math.log2(a)) if a >= fractions.Fraction(1, 2 ** 14) else -14
+    while a >= 2 ** (e + 1):
+        e += 1
+    while e > -14 and a < 2 ** e:
+        e -= 1
+    ulp = fractions.Fraction(2) ** (e - 10)
+    m = a / ulp                                  # in [1024, 2048) for normals, [0, 1024) below
+    mi = math.floor(m)
+    rem = m - mi
+    if rem > fractions.Fraction(1, 2) or (rem == fractions.Fraction(1, 2) and mi % 2 == 1):
+        mi += 1
+    if e > -14 or mi >= 1024:
+        if mi == 2048:
+            mi, e = 1024, e + 1
+        if e > 15:
+            return sign | 0x7C00
+        return sign | ((e + 15) << 10) | (mi - 1024)
+    return sign | mi
+
+
+def test_f16_reference_rounding_by_hand():
+    assert _f16_rne_bits(1.0 + 2.0 ** -11) == 0x3C00          # tie -> even (1.0)
+    assert _f16_rne_bits(1.0 + 3 * 2.0 ** -11) == 0x3C02      # tie -> even (1 + 2^-9)
+    assert _f16_rne_bits(-2.5) == 0xC100
+    assert _f16_rne_bits(2.0 ** -24) == 0x0001                # smallest subnormal
+    assert _f16_rne_bits(65504.0) == 0x7BFF
+
+
+def test_fp16_cache_holds_the_rounded_keys_and_values():
+    """Layer 0's cache rows depend only on the inputs, so with kv_store="fp16" they must be
+    the round-to-nearest-even halves of the fp32-cache model's rows, element by element."""
+    m32 = _tiny_model(L=2, h=2, hk=1)
+    draw = synth.make_weights(m32.shape, seed=0, std=0.05, ln_random=True)
+    m16 = O.OracleModel(draw, "int4", kv_store="fp16")
+    m32 = O.OracleModel(draw, "int4")
+    prefix = synth.make_prefix(m32.shape, 1, prefix_len=6, seed=61)[0]
+    c32, c16 = m32.new_cache(16), m16.new_cache(16)
+    m32.prefill(c32, prefix, [3, 4])
+    m16.prefill(c16, prefix, [3, 4])
+    for which in ("k", "v"):
+        a32 = getattr(c32, which)[0][:8].ravel()
+        a16 = getattr(c16, which)[0][:8].ravel()
+        want = np.array([_f16_rne_bits(float(x)) for x in a32], np.uint16).view(np.float16).astype(np.float64)
+        assert np.array_equal(a16, want), which
+
+
+def test_fp16_cache_incremental_equals_full_and_stays_close_to_fp32():
+    draw = synth.make_weights(synth.tiny_shape(2, 64, 2, 1, 128, 37), seed=0, std=0.05, ln_random=True)
+    m16 = O.OracleModel(draw, "int4", kv_store="fp16")
+    m32 = O.OracleModel(draw, "int4")
+    prefix = synth.make_prefix(m16.shape, 1, prefix_len=5, seed=62)[0]
+    toks = [1, 5, 9, 2, 7]
+    full = m16.teacher_forced(prefix, toks)
+    c = m16.new_cache(16)
+    inc = [m16.prefill(c, prefix, toks[:1])] + [m16.decode_step(c, t) for t in toks[1:]]
+    assert np.allclose(np.stack(inc), full, rtol=0, atol=1e-12)
+    # the stated distance of the half cache from the fp32 one on this model: below 1e-2
+    d = np.abs(full - m32.teacher_forced(prefix, toks)).max()
+    assert 0 < d < 1e-2
+
+
+def test_fp16_cache_truncation_mistake_is_caught(monkeypatch):
+    """Planted mistake: rounding toward zero instead of to nearest."""
+    draw = synth.make_weights(synth.tiny_shape(1, 64, 2, 1, 128, 37), seed=0, std=0.05, ln_random=True)
+    m16 = O.OracleModel(draw, "int4", kv_store="fp16")
+    m32 = O.OracleModel(draw, "int4")
+    prefix = synth.make_prefix(m16.shape, 1, prefix_len=6, seed=63)[0]
+
+    def trunc16(a):
+        h = np.asarray(a, np.float64).astype(np.float16)
+        back = h.astype(np.float64)
+        over = np.abs(back) > np.abs(np.asarray(a, np.float64))
+        h = h.view(np.uint16) - over.astype(np.uint16)
+        return h.view(np.float16)
+
+    c32, c16 = m32.new_cache(8), m16.new_cache(8)
+    m32.prefill(c32, prefix, [3])
+    m16.prefill(c16, prefix, [3])
+    a32 = c32.k[0][:7].ravel()
+    good = np.array([_f16_rne_bits(float(x)) for x in a32], np.uint16).view(np.float16).astype(np.float64)
+    bad = trunc16(a32).astype(np.float64)
+    assert np.array_equal(c16.k[0][:7].ravel(), good)
+    assert not np.array_equal(bad, good)

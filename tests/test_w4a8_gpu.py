@@ -1,0 +1,163 @@
+"""W4A8, the accuracy_level=4 reading ("MuScriptor Medium — optimized W4A32 ONNX Runtime",
+Model variant: activations quantised to INT8 at run time, INT32 accumulation), against the
+oracle's reading (quantize_act_int8_g32, matmul_w4a8, OracleModel(act_int8=True)).
+
+Acceptance: the INT8 codes and block scales bit-exact given the same fp32 input; the MatMul
+within the fp32 summation bound of its per-block terms.  At the model level the two sides
+quantise activations they computed in fp32 (library) and fp64 (oracle); an activation whose
+ratio to its block scale lies within ~1e-7 of a rounding boundary gets codes one apart, and
+each such flip moves its block's product by 1/127 of the block's range, which perturbs the
+next layers' activations by ~1e-3 and flips many of their codes in turn.  So the two sides'
+quantisation noise decorrelates with depth (on some streams after one early flip), and the
+model-level bar is the method's own noise, measured on the same inputs as the distance
+between the oracle with and without INT8 activations (noise = oracle W4A8 - oracle W4A32):
+  - the library's own departure from W4A32, mean |library - oracle W4A32|, is between 0.5
+    and 1.5 times the noise's mean (a library that skipped the INT8 step would sit near 0, a
+    wrong one far above 1);
+  - max |library - oracle W4A8| within twice the noise's max.
+Checked on a 2-layer model (1 to 16 streams, prefill and decode) and on the full-size small
+and medium models.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import ms_oracle as O
+
+pytestmark = pytest.mark.gpu
+ms = pytest.importorskip("decoder_only_transformer_int4_b200")
+
+U32 = 2.0 ** -24
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def test_act_int8_codes_bit_exact():
+    rng = np.random.default_rng(11)
+    M, K = 37, 1024
+    x = (rng.standard_normal((M, K)) * np.exp2(rng.integers(-20, 10, (M, 1)))).astype(np.float32)
+    x[0, 32:64] = 0.0                                                 # an all-zero block
+    x[1, :32] = np.arange(32, dtype=np.float32) - 15.5                # many ratios on .5
+    x[2, :32] = np.float32(127.0) * np.sign(np.arange(32) - 16.5)     # absmax on every element
+    q, s = ms.quantize_act_int8(_dev(x))
+    qo, so = O.quantize_act_int8_g32(x)
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 3, 64, 130])
+@pytest.mark.parametrize("N,K", [(1536, 1024), (1024, 4096), (200, 512)])
+def test_matmul_w4a8(M, N, K):
+    w = synth.make_matrix(N, K, seed=700 + K)
+    x = synth.make_activations(M, K, seed=710 + M)
+    pg, sg = ms.quantize_int4_g32(_dev(w))
+    q, s = O.quantize_int4_g32(w)
+    qa, sa = ms.quantize_act_int8(_dev(x))
+    y = ms.matmul_w4a8(qa, sa, pg, sg).cpu().numpy().astype(np.float64)
+    ref = O.matmul_w4a8(x, q, s)
+    # per-block terms isum * sa * sw are exact up to one fp32 rounding each; the K/32 of them
+    # are added in fp32: |err| <= (K/32 + 2) * 2^-24 * sum_b |term_b|
+    qao, sao = O.quantize_act_int8_g32(x)
+    KB = K // 32
+    terms = np.zeros((M, N))
+    for b in range(KB):
+        cols = slice(32 * b, 32 * b + 32)
+        isum = qao[:, cols].astype(np.float64) @ q[:, cols].astype(np.float64).T
+        terms += np.abs(isum * sao[:, b, None].astype(np.float64) * s[None, :, b].astype(np.float64))
+    assert np.all(np.abs(y - ref) <= (KB + 2) * U32 * terms + 1e-30)
+
+
+def _noise_bar(got, om8, om32, prefix, toks):
+    ref8 = om8.teacher_forced(prefix, toks)
+    ref32 = om32.teacher_forced(prefix, toks)
+    noise = np.abs(ref8 - ref32)
+    own = np.abs(got - ref32).mean() / noise.mean()
+    assert 0.5 <= own <= 1.5, own
+    assert np.abs(got - ref8).max() <= 2 * noise.max()
+
+
+def _teacher_forced(gm, batch, cap, prefix, start, forced, act_int8=True):
+    cache = ms.Cache(gm, batch, cap)
+    cache.set_act_int8(act_int8)
+    assert cache.act_int8 == act_int8
+    assert cache.decode_path == 2
+    lg, _ = cache.prefill(_dev(start.reshape(batch, 1)), _dev(prefix))
+    rows = [lg.cpu().numpy()]
+    for i in range(forced.shape[1]):
+        lg, _ = cache.decode_step(_dev(forced[:, i].astype(np.int32)))
+        rows.append(lg.cpu().numpy())
+    assert cache.device_status() == ms.MS_OK
+    return np.stack(rows), cache
+
+
+@pytest.mark.parametrize("batch", [1, 2, 3, 8, 16])
+def test_w4a8_model_teacher_forced_tiny(batch):
+    sh = synth.Shape("a8", 2, 256, 4, 2, 512, vocab=300)
+    draw = synth.make_weights(sh, seed=0, std=0.05, ln_random=True)
+    om = O.OracleModel(draw, "int4", act_int8=True)
+    om32 = O.OracleModel(draw, "int4")
+    gm = ms.Model.from_draw(draw, "int4")
+    prefix = synth.make_prefix(sh, batch, prefix_len=45, seed=151)
+    start = synth.make_start_tokens(batch, vocab=300, seed=152)
+    forced = synth.make_token_sequence(6, batch, vocab=300, seed=153)
+    got, _ = _teacher_forced(gm, batch, 64, prefix, start, forced)
+    for b in range(batch):
+        _noise_bar(got[:, b], om, om32, prefix[b], [int(start[b])] + list(forced[b]))
+
+
+def test_w4a8_switch_and_refusals():
+    sh = synth.Shape("a8s", 1, 256, 4, 4, 512, vocab=50)
+    draw = synth.make_weights(sh, seed=0)
+    gm = ms.Model.from_draw(draw, "int4")
+    c = ms.Cache(gm, 1, 32)
+    c.set_act_int8(True)
+    with pytest.raises(ms.MsError) as e:
+        c.set_decode_path(1)
+    assert e.value.status == ms.MS_ERR_UNSUPPORTED
+    c.set_act_int8(False)
+    c.set_decode_path(1)
+    with pytest.raises(ms.MsError):
+        c.set_act_int8(True)
+    gh = ms.Model.from_draw(draw, "fp16")
+    ch = ms.Cache(gh, 1, 32)
+    with pytest.raises(ms.MsError):
+        ch.set_act_int8(True)
+
+
+def test_w4a8_generate_equals_step_by_step():
+    sh = synth.Shape("a8g", 2, 256, 4, 2, 512, vocab=300)
+    draw = synth.make_weights(sh, seed=0, std=0.05, ln_random=True)
+    gm = ms.Model.from_draw(draw, "int4")
+    prefix = synth.make_prefix(sh, 2, prefix_len=30, seed=161)
+    start = synth.make_start_tokens(2, vocab=300, seed=162)
+    c1 = ms.Cache(gm, 2, 64)
+    c1.set_act_int8(True)
+    c1.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
+    toks, _ = c1.generate(10)
+    c2 = ms.Cache(gm, 2, 64)
+    c2.set_act_int8(True)
+    _, am = c2.prefill(_dev(start.reshape(2, 1)), _dev(prefix))
+    eager = []
+    for _ in range(10):
+        _, am = c2.decode_step(am.clone())
+        eager.append(am.cpu().numpy())
+    assert np.array_equal(toks.cpu().numpy(), np.stack(eager))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("key,steps", [("c2", 16), ("c3", 16)])
+def test_w4a8_full_size(key, steps):
+    wl = synth.WORKLOADS[key]
+    sh = wl.shape
+    draw = synth.make_weights(sh, seed=0)
+    om = O.OracleModel(draw, "int4", act_int8=True)
+    om32 = O.OracleModel(draw, "int4")
+    gm = ms.Model.from_draw(draw, "int4")
+    prefix = synth.make_prefix(sh, 1, seed=1)
+    start = synth.make_start_tokens(1, seed=2)
+    forced = synth.make_token_sequence(steps, 1, seed=3)
+    got, _ = _teacher_forced(gm, 1, wl.capacity, prefix, start, forced)
+    _noise_bar(got[:, 0], om, om32, prefix[0], [int(start[0])] + list(forced[0]))
