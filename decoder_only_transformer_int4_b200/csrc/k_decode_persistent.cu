@@ -515,18 +515,33 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // lo).  Lane (r = lane / 4, t = lane % 4) holds acc[0], acc[1] = rows r of columns 2t, 2t + 1
 // (stream t, hi and lo), acc[2], acc[3] = row r + 8 of the same; acc[4..7] the same for
 // streams 4 + t.  The group's INT4 scales multiply each record's sums.
+// Shared-memory loads by 32-bit shared address (the record and plane pointers reach the loop
+// as generic pointers; explicit ld.shared avoids the generic path's extra latency).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+
+// rec, blo, bhi: shared addresses of the record and of this lane's activation plane words.
 template <int M, int FMT>
-__device__ __forceinline__ void mv_record(const unsigned char* rec, const uint32_t* blo, const uint32_t* bhi, int g,
-                                          bool use, float (&acc)[8]) {
+__device__ __forceinline__ void mv_record(uint32_t rec, uint32_t blo, uint32_t bhi, int g, bool use,
+                                          float (&acc)[8]) {
   const int lane = threadIdx.x & 31, gid = lane >> 2;
-  const uint4 b = *reinterpret_cast<const uint4*>(blo + g * 16);
+  const uint4 b = lds128(blo + g * 64);
   uint4 b2 = make_uint4(0u, 0u, 0u, 0u);
-  if (M > 4) b2 = *reinterpret_cast<const uint4*>(bhi + g * 16);
+  if (M > 4) b2 = lds128(bhi + g * 64);
   uint32_t a[8];
   float s0, s1;
   if (FMT == kInt4) {
-    const uint2 w = reinterpret_cast<const uint2*>(rec)[lane];
-    const float2 s = reinterpret_cast<const float2*>(rec + 256)[gid];
+    const uint2 w = lds64(rec + lane * 8);
+    const uint2 sr = lds64(rec + 256 + gid * 8);
+    const float2 s = make_float2(__uint_as_float(sr.x), __uint_as_float(sr.y));
     s0 = use ? s.x : 0.f;
     s1 = use ? s.y : 0.f;
     const uint32_t x8 = w.x >> 8, y8 = w.y >> 8;
@@ -539,8 +554,8 @@ __device__ __forceinline__ void mv_record(const unsigned char* rec, const uint32
     a[6] = q_pair_b(x8);
     a[7] = q_pair_b(y8);
   } else {
-    const uint4 x0 = reinterpret_cast<const uint4*>(rec)[2 * lane];
-    const uint4 x1 = reinterpret_cast<const uint4*>(rec)[2 * lane + 1];
+    const uint4 x0 = lds128(rec + lane * 32);
+    const uint4 x1 = lds128(rec + lane * 32 + 16);
     s0 = s1 = use ? 1.f : 0.f;
     a[0] = x0.x;
     a[1] = x0.y;
@@ -673,8 +688,8 @@ __device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, const MvJ
   const int nu = jb.u1 - jb.u0;
   const int pw = (K >> 1) + 16;
   // this lane's B rows: plane row gid (the zero row past the streams) and, for 8 streams, gid + 8
-  const uint32_t* blo = (gid < 2 * M ? rg.planes + gid * pw : rg.zero) + tq * 4;
-  const uint32_t* bhi = rg.planes + (M > 4 ? (gid + 8) * pw : 0) + tq * 4;
+  const uint32_t blo = smem_u32((gid < 2 * M ? rg.planes + gid * pw : rg.zero) + tq * 4);
+  const uint32_t bhi = smem_u32(rg.planes + (M > 4 ? (gid + 8) * pw : 0) + tq * 4);
   for (int i = lane; i < nu * M * kTile; i += 32) {
     const int ul = i / (M * kTile);
     rg.part[(size_t)(ul * kWarps + warp) * M * kTile + (i - ul * M * kTile)] = 0.f;
@@ -683,7 +698,7 @@ __device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, const MvJ
   bool ok = true;
   for (int p = jb.rbeg; p < jb.rend; p += PER) {
     const int n = min(PER, jb.rend - p);
-    const unsigned char* buf = ring.acquire();
+    const uint32_t buf = smem_u32(ring.acquire());
     ok = ok && ring.got;
     if (ring.got) {
       const int c0 = (n * warp) >> 3, c1 = (n * (warp + 1)) >> 3;
@@ -699,7 +714,7 @@ __device__ __forceinline__ bool mv_phase(Ring& ring, const Region& rg, const MvJ
 #pragma unroll
           for (int j = 0; j < U; ++j) {
             const int ij = min(i + j, s1 - 1);  // past the segment's end: re-read its last record, not added
-            mv_record<M, FMT>(buf + (size_t)ij * RB, blo, bhi, gi + (ij - i), i + j < s1, acc);
+            mv_record<M, FMT>(buf + (uint32_t)(ij * RB), blo, bhi, gi + (ij - i), i + j < s1, acc);
           }
         }
         i = s1;   // the next segment starts exactly where this one ends
@@ -801,24 +816,37 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     mh[tid] = -INFINITY;
     lh[tid] = 0.f;
   }
-  // first run of cached keys: issue these loads before waiting on this step's q
+  // a run of up to 64 cached positions into Ks / Vs: every load of the thread (4 of K, 4 of
+  // V) is in flight before its first store, so a run costs one memory round trip.  The first
+  // run is issued before the wait on this step's q.
   auto stage = [&](int c0, int cn) {
-    for (int i = tid; i < cn * 16; i += kThreads) {
-      const int p = i >> 4, f = i & 15;
-      if (c0 + p == pos) continue;  // the new position comes from qkv
-      const size_t e = head + (size_t)(c0 + p) * 64 + 4 * f;
-      const float4 kv = h16 ? kv_load4<1>(kc, e) : kv_load4<0>(kc, e);
-      Ks[p * 65 + 4 * f + 0] = kv.x;
-      Ks[p * 65 + 4 * f + 1] = kv.y;
-      Ks[p * 65 + 4 * f + 2] = kv.z;
-      Ks[p * 65 + 4 * f + 3] = kv.w;
-      reinterpret_cast<float4*>(Vs + p * 64)[f] = h16 ? kv_load4<1>(vc, e) : kv_load4<0>(vc, e);
+    float4 kr[kAttSub * 16 / kThreads], vr[kAttSub * 16 / kThreads];
+#pragma unroll
+    for (int j = 0; j < kAttSub * 16 / kThreads; ++j) {
+      const int i = tid + j * kThreads, p = i >> 4, f = i & 15;
+      if (p < cn && c0 + p != pos) {   // the new position comes from qkv
+        const size_t e = head + (size_t)(c0 + p) * 64 + 4 * f;
+        kr[j] = h16 ? kv_load4<1>(kc, e) : kv_load4<0>(kc, e);
+        vr[j] = h16 ? kv_load4<1>(vc, e) : kv_load4<0>(vc, e);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kAttSub * 16 / kThreads; ++j) {
+      const int i = tid + j * kThreads, p = i >> 4, f = i & 15;
+      if (p < cn && c0 + p != pos) {
+        Ks[p * 65 + 4 * f + 0] = kr[j].x;
+        Ks[p * 65 + 4 * f + 1] = kr[j].y;
+        Ks[p * 65 + 4 * f + 2] = kr[j].z;
+        Ks[p * 65 + 4 * f + 3] = kr[j].w;
+        reinterpret_cast<float4*>(Vs + p * 64)[f] = vr[j];
+      }
     }
   };
   stage(t0, min(kAttSub, t1 - t0));
   // this thread's words of q (pair j, j + 32 of head tid / 32; hpg * 32 <= 256 threads)
   // and, in the split that holds pos, of the new v and k: all loaded, then settled together
   const int qh = tid >> 5, qj = tid & 31;
+  const float c_r = cs[qj], s_r = sn[qj];   // this thread's RoPE pair, read before the wait
   uint64_t w[5];
   const uint64_t* pp[5];
   bool use[5];
@@ -836,9 +864,8 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
   const bool ok = settle_words<5>(w, pp, use, a.test_stall == 1 ? (ep ^ 0x80000000u) : ep, a);
   if (use[0]) {
     const float x0 = __uint_as_float((unsigned)w[0]), x1 = __uint_as_float((unsigned)w[1]);
-    const float c = cs[qj], s = sn[qj];
-    qs[qh * 64 + qj] = (x0 * c - x1 * s) * 0.125f;
-    qs[qh * 64 + qj + 32] = (x0 * s + x1 * c) * 0.125f;
+    qs[qh * 64 + qj] = (x0 * c_r - x1 * s_r) * 0.125f;
+    qs[qh * 64 + qj + 32] = (x0 * s_r + x1 * c_r) * 0.125f;
   }
   if (use[2]) {
     // the new row: appended to the cache, and used by this step in the cache's precision
@@ -853,8 +880,7 @@ __device__ __forceinline__ bool attention_unit(const PersistArgs& a, float* scra
     vnew[tid] = v;
     if (use[3]) {
       const float x0 = __uint_as_float((unsigned)w[3]), x1 = __uint_as_float((unsigned)w[4]);
-      const float c = cs[tid], s = sn[tid];
-      float k0 = x0 * c - x1 * s, k1 = x0 * s + x1 * c;
+      float k0 = x0 * c_r - x1 * s_r, k1 = x0 * s_r + x1 * c_r;   // tid < 32: qj == tid
       if (h16) {
         k0 = __half2float(__float2half_rn(k0));
         k1 = __half2float(__float2half_rn(k1));
