@@ -481,3 +481,57 @@ class OracleCache:
         k = np.stack([kk[:t] for kk in self.k])[:, None]
         v = np.stack([vv[:t] for vv in self.v])[:, None]
         return k, v
+
+
+# ---------------------------------------------------------------------------
+# Conditioner front-end  ([ONNX-S] muscriptor-small-cond.onnx: audio f32 [1, 80000] at
+# 16 kHz, instrument ids [1, K], dataset id [1, 1] -> prefix [1, 501 + 1 + K, d], the
+# spectrogram inside the graph with the checkpoint's stored window and mel filterbank;
+# [CARD] Model description: STFT n_fft 2048, hop 160, 512 mel bins, projected to d_model)
+# ---------------------------------------------------------------------------
+
+LOG_FLOOR = 1e-6
+
+# Readings where the pages are silent: centred frames (the signal padded by n_fft / 2 on both
+# sides by reflection without repeating the edge sample, so 1 + N // hop frames: 501 for
+# 80000 samples, the pages' figure); the magnitude |X| (the pages speak of log-magnitude
+# features); the natural logarithm of the mel energies clamped below at 1e-6 (the pages' log
+# floor); the prefix rows in the order of the pages' shape 501 + 1 + K: the projected frames,
+# then the dataset row, then the K instrument rows.
+
+
+def stft_magnitude(audio: np.ndarray, window: np.ndarray, hop: int) -> np.ndarray:
+    """|STFT| of one signal ``audio`` [N]: [frames, n_fft/2 + 1], frames = 1 + N // hop.
+
+    Frame t covers padded samples [t*hop, t*hop + n_fft) of the signal padded by n_fft/2 on
+    each side by reflection (sample -i is sample i), is multiplied by ``window`` and goes
+    through the real DFT (numpy's FFT as the library primitive)."""
+    x = np.asarray(audio, np.float64)
+    w = np.asarray(window, np.float64)
+    n_fft = w.shape[0]
+    xp = np.pad(x, n_fft // 2, mode="reflect")
+    frames = 1 + x.shape[0] // hop
+    idx = np.arange(frames)[:, None] * hop + np.arange(n_fft)[None, :]
+    return np.abs(np.fft.rfft(xp[idx] * w[None, :], axis=1))
+
+
+def log_mel(mag: np.ndarray, mel_fb: np.ndarray) -> np.ndarray:
+    """ln(max(mag @ fb^T, 1e-6)): [frames, n_mels] from [frames, n_freq] and fb [n_mels, n_freq]."""
+    return np.log(np.maximum(mag @ np.asarray(mel_fb, np.float64).T, LOG_FLOOR))
+
+
+def conditioner(audio: np.ndarray, dataset: Sequence[int], instruments: np.ndarray, cond, hop: int) -> np.ndarray:
+    """The conditioner's prefix [B, frames + 1 + K, d] for audio [B, N], dataset ids [B] and
+    instrument ids [B, K]; ``cond`` holds window, mel_fb, proj_w [d, n_mels], proj_b [d],
+    inst_emb, ds_emb (synth.CondDraw)."""
+    audio = np.asarray(audio)
+    instruments = np.asarray(instruments, np.int64).reshape(audio.shape[0], -1)
+    W = np.asarray(cond.proj_w, np.float64)
+    out = []
+    for b in range(audio.shape[0]):
+        rows = log_mel(stft_magnitude(audio[b], cond.window, hop), cond.mel_fb) @ W.T + np.asarray(cond.proj_b,
+                                                                                                    np.float64)
+        ds = np.asarray(cond.ds_emb, np.float64)[[int(dataset[b])]]
+        inst = np.asarray(cond.inst_emb, np.float64)[instruments[b]]
+        out.append(np.concatenate([rows, ds, inst], axis=0))
+    return np.stack(out)

@@ -196,3 +196,65 @@ def make_kv_cache(shape: Shape, batch: int, T: int, seed: int = 4, std: float = 
         k[l] = torch.randn(*sz, generator=g, dtype=torch.float32).numpy() * std
         v[l] = torch.randn(*sz, generator=g, dtype=torch.float32).numpy() * std
     return k, v
+
+
+# ---- conditioner front-end inputs --------------------------------------------------------
+# "MuScriptor small — ONNX conversion", muscriptor-small-cond.onnx: audio f32 [1, 80000] (one
+# 5-second chunk at 16 kHz), instrument ids [1, K] (1 = unconditional), dataset id [1, 1]
+# (always 1); the checkpoint stores its STFT window and mel filterbank as half-precision
+# buffers.  "MuScriptor — small (≈100M)" model card: STFT n_fft 2048, hop 160, 512 mel bins,
+# the spectrogram projected to d_model.  The validation input of the W4A32 page is a 5-second
+# 440 Hz tone.
+
+SAMPLE_RATE = 16000
+N_SAMPLES = 80000
+N_FFT = 2048
+HOP = 160
+N_MELS = 512
+N_INSTRUMENTS = 130
+N_DATASETS = 2
+
+
+@dataclasses.dataclass
+class CondDraw:
+    window: np.ndarray      # fp32 [n_fft]: the half rounding of the periodic Hann window
+    mel_fb: np.ndarray      # fp32 [n_mels, n_fft/2 + 1]: the half rounding of the htk filterbank
+    proj_w: np.ndarray      # fp32 [d, n_mels]  (stand-in for the trained projection)
+    proj_b: np.ndarray      # fp32 [d]
+    inst_emb: np.ndarray    # fp32 [n_instruments, d]
+    ds_emb: np.ndarray      # fp32 [n_datasets, d]
+
+
+def make_tone(batch: int = 1, freq: float = 440.0, amplitude: float = 0.5, n_samples: int = N_SAMPLES,
+              sample_rate: int = SAMPLE_RATE) -> np.ndarray:
+    """A sine tone, fp32 [B, n_samples]: amplitude * sin(2 pi freq t), t = n / sample_rate."""
+    n = np.arange(n_samples, dtype=np.float64)
+    x = amplitude * np.sin(2.0 * np.pi * freq * n / sample_rate)
+    return np.repeat(x[None].astype(np.float32), batch, axis=0)
+
+
+def make_noise_audio(batch: int, seed: int = 6, n_samples: int = N_SAMPLES, std: float = 0.1) -> np.ndarray:
+    """Seeded N(0, std) audio, fp32 [B, n_samples]."""
+    return _normal(_gen(seed), (batch, n_samples), std)
+
+
+def make_cond_weights(d_model: int, seed: int = 7, n_fft: int = N_FFT, n_mels: int = N_MELS,
+                      sample_rate: int = SAMPLE_RATE) -> CondDraw:
+    """The conditioner's buffers, as the checkpoint stores them: the half rounding of
+    torch.hann_window(n_fft) (periodic, fp32) and the half rounding of the htk mel
+    filterbank (no normalisation, 0 .. sample_rate / 2; torchaudio's melscale_fbanks, fp32).
+    Projection and embeddings: seeded N(0, 0.02) stand-ins for the trained ones."""
+    import warnings
+    import torchaudio
+    window = torch.hann_window(n_fft, periodic=True, dtype=torch.float32).half().float().numpy()
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore")    # 512 htk bands over 1025 bins leave some bands empty
+        fb = torchaudio.functional.melscale_fbanks(n_fft // 2 + 1, 0.0, sample_rate / 2.0, n_mels, sample_rate,
+                                                   norm=None, mel_scale="htk")
+    fb = fb.T.contiguous().half().float().numpy()
+    g = _gen(seed)
+    proj_w = _normal(g, (d_model, n_mels), 0.02)
+    proj_b = _normal(g, (d_model,), 0.02)
+    inst_emb = _normal(g, (N_INSTRUMENTS, d_model), 0.02)
+    ds_emb = _normal(g, (N_DATASETS, d_model), 0.02)
+    return CondDraw(window, fb, proj_w, proj_b, inst_emb, ds_emb)

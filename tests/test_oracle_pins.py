@@ -897,3 +897,124 @@ def test_fp16_cache_truncation_mistake_is_caught(monkeypatch):
     bad = trunc16(a32).astype(np.float64)
     assert np.array_equal(c16.k[0][:7].ravel(), good)
     assert not np.array_equal(bad, good)
+
+
+# ---------------------------------------------------------------------------
+# Conditioner front-end ([ONNX-S] muscriptor-small-cond.onnx; [CARD] Model description)
+# ---------------------------------------------------------------------------
+
+def test_conditioner_shape_follows_the_pages():
+    cond = synth.make_cond_weights(64)
+    audio = synth.make_noise_audio(1, seed=171)
+    p = O.conditioner(audio, [1], np.array([[1]]), cond, synth.HOP)
+    figs = _gold("pages_figures.json")
+    assert p.shape == (1, 501 + 1 + 1, 64)                      # 501 frames + dataset + K = 1
+    assert p.shape[1] == figs["prefix_rows"]["value"]            # the decoder's 503 prefix rows
+
+
+def test_stft_magnitude_matches_torch_stft():
+    cond = synth.make_cond_weights(8)
+    x = synth.make_noise_audio(1, seed=172)[0]
+    ours = O.stft_magnitude(x, cond.window, synth.HOP)
+    ref = torch.stft(torch.from_numpy(x.astype(np.float64)), synth.N_FFT, synth.HOP,
+                     window=torch.from_numpy(cond.window.astype(np.float64)), center=True, pad_mode="reflect",
+                     return_complex=True).abs().numpy().T
+    assert ours.shape == ref.shape == (501, 1025)
+    assert np.allclose(ours, ref, rtol=1e-9, atol=1e-9)
+
+
+def test_stft_of_a_bin_frequency_tone_closed_form():
+    """x = A cos(2 pi k0 n / N): an interior frame's bin k0 holds A/2 sum(w) plus the
+    negative-frequency image A/2 sum(w e^{-2 pi i 2 k0 m / N}).  The exact periodic Hann window
+    has no DFT weight at bin 2 k0 = 112, so the image comes only from the stored window's
+    rounding to half: at most A/2 sum|w - w_exact|."""
+    cond = synth.make_cond_weights(8)
+    k0, A = 56, 0.5
+    n = np.arange(synth.N_SAMPLES)
+    x = A * np.cos(2 * np.pi * k0 * n / synth.N_FFT)
+    mag = O.stft_magnitude(x, cond.window, synth.HOP)
+    w = cond.window.astype(np.float64)
+    want = A / 2 * w.sum()
+    image = A / 2 * np.abs(w - (0.5 - 0.5 * np.cos(2 * np.pi * np.arange(2048) / 2048))).sum()
+    assert 0 < image < 1e-3 * want
+    assert np.all(np.abs(mag[20:480, k0] - want) <= image * (1 + 1e-9) + 1e-9)
+    assert np.all(mag[20:480].argmax(axis=1) == k0)
+
+
+def test_stft_parseval_with_a_rectangular_window():
+    x = synth.make_noise_audio(1, seed=173, n_samples=4000)[0].astype(np.float64)
+    N = 256
+    mag = O.stft_magnitude(x, np.ones(N), 64)
+    xp = np.pad(x, N // 2, mode="reflect")
+    for t in (0, 3, 40, mag.shape[0] - 1):
+        fr = xp[t * 64: t * 64 + N]
+        e = (mag[t, 0] ** 2 + 2 * (mag[t, 1:-1] ** 2).sum() + mag[t, -1] ** 2) / N
+        assert math.isclose(e, (fr ** 2).sum(), rel_tol=1e-10)
+
+
+def test_log_mel_floor_and_empty_bands():
+    cond = synth.make_cond_weights(8)
+    empty = np.where(cond.mel_fb.sum(axis=1) == 0)[0]
+    assert empty.size > 0                                           # 512 htk bands over 1025 bins
+    lm = O.log_mel(np.ones((3, 1025)), cond.mel_fb)
+    assert np.all(lm[:, empty] == np.log(1e-6))
+    full = np.where(cond.mel_fb.sum(axis=1) > 0)[0]
+    assert np.allclose(lm[:, full], np.log(cond.mel_fb[full].astype(np.float64).sum(axis=1)))
+
+
+def test_mel_filterbank_is_the_htk_triangles():
+    """The stored filterbank against the htk definition restated here in float64 (half-ulp
+    apart: the checkpoint's buffer is an fp32 computation rounded to half)."""
+    cond = synth.make_cond_weights(8)
+    freqs = np.linspace(0, 8000, 1025)
+    mel = lambda f: 2595 * np.log10(1 + f / 700)
+    pts = 700 * (10 ** (np.linspace(0, mel(8000.0), 514) / 2595) - 1)
+    fb = np.maximum(0, np.minimum((freqs[None] - pts[:-2, None]) / (pts[1:-1] - pts[:-2])[:, None],
+                                  (pts[2:, None] - freqs[None]) / (pts[2:] - pts[1:-1])[:, None]))
+    assert np.abs(cond.mel_fb - fb).max() <= 2.0 ** -11 + 1e-6
+    hann = 0.5 - 0.5 * np.cos(2 * np.pi * np.arange(2048) / 2048)
+    assert np.abs(cond.window - hann).max() <= 2.0 ** -11
+
+
+def test_conditioner_rows_by_hand_and_the_tone():
+    """Rows: projected log-mel frames, the dataset row, the instrument rows (in that order);
+    the 440 Hz tone of the W4A32 page's validation puts its energy in the mel band whose
+    centre is nearest 440 Hz."""
+    cond = synth.make_cond_weights(16)
+    tone = synth.make_tone(1)
+    p = O.conditioner(tone, [1], np.array([[5, 7]]), cond, synth.HOP)
+    assert np.array_equal(p[0, 501], cond.ds_emb[1].astype(np.float64))
+    assert np.array_equal(p[0, 502], cond.inst_emb[5].astype(np.float64))
+    assert np.array_equal(p[0, 503], cond.inst_emb[7].astype(np.float64))
+    lm = O.log_mel(O.stft_magnitude(tone[0], cond.window, synth.HOP), cond.mel_fb)
+    rows = lm @ cond.proj_w.astype(np.float64).T + cond.proj_b
+    assert np.allclose(p[0, :501], rows, rtol=0, atol=1e-12)
+    centres = (np.arange(1025) * 8000 / 1024) @ np.where(cond.mel_fb > 0, cond.mel_fb, 0).T / \
+        np.maximum(cond.mel_fb.sum(axis=1), 1e-30)
+    band = int(np.argmax(lm[250]))
+    assert abs(centres[band] - 440.0) < 20.0
+
+
+@pytest.mark.parametrize("mistake", ["power", "zero-pad", "log10"])
+def test_conditioner_planted_mistakes_are_caught(monkeypatch, mistake):
+    cond = synth.make_cond_weights(8)
+    x = synth.make_noise_audio(1, seed=174)[0]
+    ref = torch.stft(torch.from_numpy(x.astype(np.float64)), synth.N_FFT, synth.HOP,
+                     window=torch.from_numpy(cond.window.astype(np.float64)), center=True, pad_mode="reflect",
+                     return_complex=True).abs().numpy().T
+    orig_stft, orig_log = O.stft_magnitude, O.log_mel
+    if mistake == "power":
+        monkeypatch.setattr(O, "stft_magnitude", lambda a, w, h: orig_stft(a, w, h) ** 2)
+    elif mistake == "zero-pad":
+        def zp(a, w, h):
+            xp = np.pad(np.asarray(a, np.float64), len(w) // 2)
+            idx = np.arange(1 + len(a) // h)[:, None] * h + np.arange(len(w))[None, :]
+            return np.abs(np.fft.rfft(xp[idx] * np.asarray(w, np.float64)[None], axis=1))
+        monkeypatch.setattr(O, "stft_magnitude", zp)
+    else:
+        monkeypatch.setattr(O, "log_mel", lambda m, fb: np.log10(np.maximum(m @ np.asarray(fb, np.float64).T, 1e-6)))
+    caught = not np.allclose(O.stft_magnitude(x, cond.window, synth.HOP), ref, rtol=1e-9, atol=1e-9)
+    lm = O.log_mel(np.ones((2, 1025)), cond.mel_fb)
+    empty = np.where(cond.mel_fb.sum(axis=1) == 0)[0]
+    caught = caught or not np.all(lm[:, empty] == np.log(1e-6))
+    assert caught, mistake
