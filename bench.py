@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -54,6 +55,7 @@ def _args():
                     help="skip the batched-decode block (the 64-stream medium workload)")
     ap.add_argument("--no-prefill-tensor", action="store_true",
                     help="skip the prefill GEMM tensor-pipe block")
+    ap.add_argument("--no-cond", action="store_true", help="skip the conditioner block")
     ap.add_argument("--no-pages", action="store_true",
                     help="skip the page-faithful block (kv heads = heads, fp32 and fp16 caches)")
     ap.add_argument("--decode-path", type=int, default=0, choices=[0, 1, 2],
@@ -403,6 +405,64 @@ def _pages_block(ms, torch, dev, flush, steps=2, warmup=1):
     return res
 
 
+# fp64 FMA lanes per SM on B200 (the published 37 TFLOP/s fp64 over 148 SMs at 1.965 GHz)
+_FP64_LANES_PER_SM = 64
+
+
+def _cond_block(ms, torch, dev, flush, d_model, batches, reps=5, warmup=2):
+    """The conditioner front-end (5 s of 16 kHz audio -> 501 log-mel frames projected to
+    d_model, then the dataset and instrument rows), device-timed per call with CUDA events, L2
+    flushed before each.  The log-mel kernel alone is timed through ms_cond_log_mel (the same
+    kernel writing fp32 rows instead of the GEMM's planes).  Its roofline is fp64 arithmetic:
+    algorithmic flops per frame = 2.5 n log2 n for the real FFT of n = n_fft points, plus the
+    window (n), the magnitudes (3 per bin) and the mel sums (2 per filterbank weight), against
+    148 SMs x 64 fp64 FMA lanes x 2 flops x the SM clock (nominal, derived from unit counts)."""
+    cond = synth.make_cond_weights(d_model)
+    nnz = int((cond.mel_fb != 0).sum())
+    n = synth.N_FFT
+    flops_frame = 2.5 * n * math.log2(n) + n + 3 * (n // 2 + 1) + 2 * nnz
+    props = torch.cuda.get_device_properties(dev)
+    sm_ghz = 1.965
+    peak64 = props.multi_processor_count * _FP64_LANES_PER_SM * 2 * sm_ghz * 1e9 / 1e12
+    stream = torch.cuda.current_stream(dev)
+    out = {"workload": f"conditioner: 5 s at 16 kHz (80000 samples), n_fft 2048, hop 160, 512 mel bands, "
+                       f"d_model {d_model}, one instrument row", "cases": []}
+    for B in batches:
+        c = ms.Conditioner.from_draw(cond, synth.N_SAMPLES, synth.HOP, max_batch=B, device=dev.index or 0)
+        audio = torch.from_numpy(synth.make_noise_audio(B, seed=6)).to(dev)
+        dataset = torch.zeros(B, dtype=torch.int32, device=dev)
+        inst = torch.zeros((B, 1), dtype=torch.int32, device=dev)
+        prefix = torch.empty((B, c.rows(1), d_model), dtype=torch.float32, device=dev)
+        lm = torch.empty((B, c.frames, synth.N_MELS), dtype=torch.float32, device=dev)
+        t_all, t_lm = [], []
+        for i in range(warmup + reps):
+            for fn, acc in ((lambda: c(audio, dataset, inst, out=prefix), t_all), (lambda: c.log_mel(audio, out=lm), t_lm)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                e1.synchronize()
+                if i >= warmup:
+                    acc.append(e0.elapsed_time(e1))
+        assert c.device_status() == ms.MS_OK
+        frames = B * c.frames
+        ms_all, ms_lm = statistics.median(t_all), statistics.median(t_lm)
+        ach = flops_frame * frames / (ms_lm / 1e3) / 1e12
+        proj_tflop = 2.0 * frames * d_model * synth.N_MELS / 1e12
+        out["cases"].append({
+            "streams": B, "frames": frames, "ms_per_call": ms_all, "frames_per_s": frames / (ms_all / 1e3),
+            "log_mel_ms": ms_lm, "projection_and_rows_ms": max(ms_all - ms_lm, 0.0),
+            "projection_model_tflops": proj_tflop / (max(ms_all - ms_lm, 1e-6) / 1e3),
+            "roofline": {"bound": "alu", "kernel": "log_mel_kernel (fp64 FFT, magnitudes, mel sums, log)",
+                         "achieved": ach, "peak": peak64, "unit": "TFLOP/s", "frac": ach / peak64,
+                         "peak_kind": f"derived: {props.multi_processor_count} SMs x {_FP64_LANES_PER_SM} fp64 "
+                                      f"FMA lanes x 2 x {sm_ghz} GHz",
+                         "algorithmic_flops_per_frame": flops_frame}})
+        c.close()
+    return out
+
+
 def _prefill_tensor_block(ms, torch, model, shape, rows_list, dev, flush, reps=5, warmup=2):
     """Prefill GEMMs on the tensor cores: each backbone MatMul of layer 0 of the benchmark's
     model at M = prefill rows, through ms_model_matmul (the tcgen05 GEMM prefill runs, on the
@@ -576,7 +636,7 @@ def run_ours(a):
         roof["traffic"] = tr["bytes"]
         roof["traffic_per"] = f"one launch of {tr['tokens']} decode steps, cache lengths {t_lo}..{t_hi} (ncu)"
         roof["traffic_over_algorithmic"] = tr["bytes"] / alg
-    batched = prefill_tc = pages = None
+    batched = prefill_tc = pages = cond = None
     if world == 1 and not a.no_batched and a.workload in _BATCHED:
         batched = _batched_block(ms, torch, model, _BATCHED[a.workload], dev, flush)
     if world == 1 and not a.no_pages and a.workload == "c3":
@@ -586,6 +646,9 @@ def run_ours(a):
         if a.workload in _BATCHED:
             rows.append(synth.WORKLOADS[_BATCHED[a.workload]].batch * (wl.prefix_len + 1))
         prefill_tc = _prefill_tensor_block(ms, torch, model, sh, rows, dev, flush)
+    if world == 1 and not a.no_cond:
+        nb = [1] + ([synth.WORKLOADS[_BATCHED[a.workload]].batch] if a.workload in _BATCHED else [])
+        cond = _cond_block(ms, torch, dev, flush, sh.d_model, nb)
     if world > 1:
         dist.barrier()
     if rank == 0:
@@ -611,6 +674,8 @@ def run_ours(a):
             line["prefill_tensor"] = prefill_tc
         if pages is not None:
             line["pages"] = pages
+        if cond is not None:
+            line["conditioner"] = cond
         print(json.dumps(line), flush=True)
     cache.close()
     model.close()

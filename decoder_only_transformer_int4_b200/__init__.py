@@ -58,6 +58,17 @@ class Weights(ctypes.Structure):
                 ("ln_f_b", ctypes.c_void_p), ("layers", ctypes.POINTER(LayerWeights))]
 
 
+class CondConfig(ctypes.Structure):
+    _fields_ = [("n_samples", ctypes.c_int), ("n_fft", ctypes.c_int), ("hop", ctypes.c_int),
+                ("n_mels", ctypes.c_int), ("d_model", ctypes.c_int), ("n_instruments", ctypes.c_int),
+                ("n_datasets", ctypes.c_int), ("max_batch", ctypes.c_int)]
+
+
+class CondWeights(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_void_p), ("mel_fb", ctypes.c_void_p), ("proj_w", ctypes.c_void_p),
+                ("proj_b", ctypes.c_void_p), ("inst_emb", ctypes.c_void_p), ("ds_emb", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
@@ -100,6 +111,12 @@ _PROTOS = {
     "ms_model_matmul": (_I, [_P, _I, _I, _P, _P, _I, _I, _P, _I, _P]),
     "ms_op_lm_head_argmax": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
     "ms_op_lm_head_argmax_static": (_I, [_P, _I, _I, _I, _P, _P, _F, _P, _I, _P, _P, _P]),
+    "ms_cond_create": (_I, [ctypes.POINTER(CondConfig), ctypes.POINTER(CondWeights), _I, ctypes.POINTER(_P)]),
+    "ms_cond_destroy": (_I, [_P]),
+    "ms_cond_frames": (_I, [_P]),
+    "ms_condition": (_I, [_P, _P, _I, _P, _P, _I, _P, _P]),
+    "ms_cond_log_mel": (_I, [_P, _P, _I, _P, _P]),
+    "ms_cond_device_status": (_I, [_P, _P]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _fn = getattr(_lib, _name)
@@ -431,6 +448,77 @@ class Cache:
     def close(self):
         if getattr(self, "_h", None):
             _lib.ms_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Conditioner:
+    """The conditioner front-end (ms_cond_create): audio [B, n_samples] -> the decoder's prefix
+    [B, frames + 1 + K, d_model] (log-mel frames projected, then the dataset row and the K
+    instrument rows)."""
+
+    def __init__(self, window, mel_fb, proj_w, proj_b, inst_emb, ds_emb, n_samples: int, hop: int,
+                 max_batch: int = 1, device: int = 0):
+        mel_fb = np.ascontiguousarray(mel_fb, dtype=np.float32)
+        proj_w = np.ascontiguousarray(proj_w, dtype=np.float32)
+        inst_emb = np.ascontiguousarray(inst_emb, dtype=np.float32)
+        ds_emb = np.ascontiguousarray(ds_emb, dtype=np.float32)
+        window = np.ascontiguousarray(window, dtype=np.float32)
+        proj_b = np.ascontiguousarray(proj_b, dtype=np.float32)
+        self.cfg = CondConfig(int(n_samples), int(window.shape[0]), int(hop), int(mel_fb.shape[0]),
+                              int(proj_w.shape[0]), int(inst_emb.shape[0]), int(ds_emb.shape[0]), int(max_batch))
+        self.device = device
+        W = CondWeights(*(a.ctypes.data for a in (window, mel_fb, proj_w, proj_b, inst_emb, ds_emb)))
+        h = ctypes.c_void_p()
+        _check(_lib.ms_cond_create(ctypes.byref(self.cfg), ctypes.byref(W), device, ctypes.byref(h)),
+               "ms_cond_create")
+        self._h = h
+
+    @classmethod
+    def from_draw(cls, draw, n_samples: int, hop: int, max_batch: int = 1, device: int = 0) -> "Conditioner":
+        """From host arrays (synth.CondDraw)."""
+        return cls(draw.window, draw.mel_fb, draw.proj_w, draw.proj_b, draw.inst_emb, draw.ds_emb, n_samples, hop,
+                   max_batch, device)
+
+    @property
+    def frames(self) -> int:
+        return int(_lib.ms_cond_frames(self._h))
+
+    def rows(self, K: int) -> int:
+        return self.frames + 1 + K
+
+    def __call__(self, audio: torch.Tensor, dataset: torch.Tensor, instruments: Optional[torch.Tensor],
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """audio fp32 [B, n_samples], dataset int32 [B], instruments int32 [B, K] (or None for
+        K = 0) -> prefix fp32 [B, frames + 1 + K, d_model] (ms_condition)."""
+        B = audio.shape[0]
+        K = 0 if instruments is None else instruments.shape[1]
+        y = out if out is not None else torch.empty((B, self.rows(K), self.cfg.d_model), dtype=torch.float32,
+                                                   device=audio.device)
+        _check(_lib.ms_condition(self._h, _ptr(audio), B, _ptr(dataset), _ptr(instruments), K, _ptr(y), _stream()),
+               "ms_condition")
+        return y
+
+    def log_mel(self, audio: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """audio fp32 [B, n_samples] -> fp32 [B, frames, n_mels] (ms_cond_log_mel)."""
+        B = audio.shape[0]
+        y = out if out is not None else torch.empty((B, self.frames, self.cfg.n_mels), dtype=torch.float32,
+                                                   device=audio.device)
+        _check(_lib.ms_cond_log_mel(self._h, _ptr(audio), B, _ptr(y), _stream()), "ms_cond_log_mel")
+        return y
+
+    def device_status(self) -> int:
+        """ms_cond_device_status: synchronises and returns (and clears) the status."""
+        return int(_lib.ms_cond_device_status(self._h, _stream()))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.ms_cond_destroy(self._h)
             self._h = None
 
     def __del__(self):

@@ -115,6 +115,30 @@ cudaError_t launch_matmul_w4a8(const Launch& L, const WView& w, const int8_t* qa
                                int M, float* y, int ldy, int epi, int sms);
 cudaError_t init_attrs_w4a8();
 
+// Conditioner front-end: the log-mel spectrogram of centred, reflection-padded frames (one
+// CTA per frame and stream, double-precision FFT), and the prefix rows after the projection.
+constexpr int kCondMaxFft = 4096;
+struct CondDev {
+  const float* window;     // [n_fft]
+  const double2* twiddle;  // [n_fft / 2]: e^{-2 pi i k / n_fft}
+  const int* band_lo;      // [n_mels]: first bin of band m's non-zero range
+  const int* band_off;     // [n_mels + 1]: band m's weights are band_w[band_off[m] .. band_off[m+1])
+  const float* band_w;
+  int n_fft, hop, n_mels;
+  int kp;                  // columns of the fp16 planes: n_mels rounded up to 64, zero-filled
+};
+size_t log_mel_smem_bytes(int n_fft);
+cudaError_t init_attrs_cond();
+// out (fp32 [B * frames][n_mels]) and / or the planes xh, xl ([B * frames][kp]); either may be null.
+cudaError_t launch_log_mel(const Launch& L, const float* audio, int n_samples, int B, const CondDev& c, int frames,
+                           float* out, __half* xh, __half* xl);
+// prefix [B][frames + 1 + K][d]: y rows * yscale + bias, then ds_emb[dataset[b]], then
+// inst_emb[instruments[b][k]] (ids out of range are clamped and flag kErrTokenBit).
+cudaError_t launch_cond_assemble(const Launch& L, const float* y, float yscale, const float* bias,
+                                 const float* ds_emb, int n_ds, const float* inst_emb, int n_inst,
+                                 const int32_t* dataset, const int32_t* instruments, int K, int frames, int d, int B,
+                                 float* prefix);
+
 // Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
 // the combine done by the last CTA of each (stream, kv head).
 struct AttnDecodeWork {

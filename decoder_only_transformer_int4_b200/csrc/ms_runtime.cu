@@ -145,6 +145,7 @@ cudaError_t ensure_kernel_attributes() {
   if (e == cudaSuccess) e = ms::init_attrs_persistent();
   if (e == cudaSuccess) e = ms::init_attrs_gemm_f16();
   if (e == cudaSuccess) e = ms::init_attrs_w4a8();
+  if (e == cudaSuccess) e = ms::init_attrs_cond();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -1231,6 +1232,237 @@ ms_status ms_op_lm_head_argmax(const float* x, int ldx, int M, int d, const floa
   return check_launch(ms::launch_lm_head(L, x, ldx, M, d, gamma, beta, eps, W, V, logits, argmax, nullptr, M, 0, nullptr,
                                          0, w),
                       "lm_head");
+}
+
+}  // extern "C"
+
+// ---- conditioner front-end --------------------------------------------------------------
+
+struct ms_cond {
+  ms_cond_config cfg;
+  int device = 0;
+  int frames = 0, kp = 0;
+  float yscale = 1.f;        // 2^-s: the projection weights are stored times 2^s
+  char* base = nullptr;
+  ms::CondDev dev{};
+  uint16_t *wh = nullptr, *wl = nullptr;
+  float *bias = nullptr, *inst = nullptr, *ds = nullptr, *y = nullptr;
+  __half *xh = nullptr, *xl = nullptr;
+  unsigned* status = nullptr;
+  ~ms_cond() {
+    if (base) cudaFree(base);
+  }
+};
+
+namespace {
+
+bool cond_config_ok(const ms_cond_config& c) {
+  const bool pow2 = c.n_fft >= 16 && c.n_fft <= ms::kCondMaxFft && (c.n_fft & (c.n_fft - 1)) == 0;
+  return pow2 && c.hop >= 1 && c.n_samples > c.n_fft / 2 && c.n_mels >= 1 && c.n_mels <= 4096 && c.d_model >= 4 &&
+         c.d_model % 4 == 0 && c.n_instruments >= 1 && c.n_datasets >= 1 && c.max_batch >= 1 &&
+         c.max_batch <= 65535 && 1 + c.n_samples / c.hop <= (1 << 24);
+}
+
+ms::WView cond_view(const ms_cond* c, const uint16_t* h) {
+  ms::WView w{};
+  w.h = h;
+  w.N = c->cfg.d_model;
+  w.K = c->kp;
+  w.fmt = ms::kFp16;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* wt, int device, ms_cond** out) {
+  if (!cfg || !wt || !out) return fail(MS_ERR_INVALID_ARG, "ms_cond_create: null argument");
+  *out = nullptr;
+  if (!wt->window || !wt->mel_fb || !wt->proj_w || !wt->proj_b || !wt->inst_emb || !wt->ds_emb)
+    return fail(MS_ERR_INVALID_ARG, "ms_cond_create: null weight pointer");
+  const ms_cond_config c = *cfg;
+  if (!cond_config_ok(c))
+    return fail(MS_ERR_INVALID_ARG,
+                "ms_cond_create: need n_fft a power of two in 16..%d, hop >= 1, n_samples > n_fft / 2, "
+                "n_mels 1..4096, d_model a positive multiple of 4, tables and max_batch >= 1",
+                ms::kCondMaxFft);
+  DeviceGuard dg(device);
+  if (!dg.ok) return fail(MS_ERR_CUDA, "ms_cond_create: cannot select device %d", device);
+  {
+    cudaError_t ea = ensure_kernel_attributes();
+    if (ea != cudaSuccess) return fail(MS_ERR_CUDA, "ms_cond_create: kernel attributes: %s", cudaGetErrorString(ea));
+  }
+  const int d = c.d_model, nf = c.n_fft / 2 + 1, half = c.n_fft / 2;
+  const int frames = 1 + c.n_samples / c.hop, kp = (c.n_mels + 63) / 64 * 64;
+  // host copies of what the preprocessing reads (the pointers may be host or device)
+  std::vector<float> fb((size_t)c.n_mels * nf), pw((size_t)d * c.n_mels);
+  CUDA_TRY(cudaMemcpy(fb.data(), wt->mel_fb, fb.size() * 4, cudaMemcpyDefault));
+  CUDA_TRY(cudaMemcpy(pw.data(), wt->proj_w, pw.size() * 4, cudaMemcpyDefault));
+  // each filterbank row compressed to its non-zero range
+  std::vector<int> lo(c.n_mels), off(c.n_mels + 1, 0);
+  std::vector<float> bw;
+  for (int m = 0; m < c.n_mels; ++m) {
+    const float* row = fb.data() + (size_t)m * nf;
+    int first = -1, last = -1;
+    for (int k = 0; k < nf; ++k)
+      if (row[k] != 0.f) {
+        if (first < 0) first = k;
+        last = k;
+      }
+    lo[m] = first < 0 ? 0 : first;
+    if (first >= 0) bw.insert(bw.end(), row + first, row + last + 1);
+    off[m + 1] = (int)bw.size();
+  }
+  if (bw.empty()) bw.push_back(0.f);
+  // twiddles e^{-2 pi i k / n_fft}, k < n_fft / 2, in double on the host
+  std::vector<double2> tw(half);
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int k = 0; k < half; ++k) {
+    const double a = two_pi * (double)k / (double)c.n_fft;
+    tw[k] = make_double2(std::cos(a), -std::sin(a));
+  }
+  // projection weights times 2^s (largest magnitude below 2^15), split into fp16 hi and lo
+  float amax = 0.f;
+  for (float v : pw) amax = std::max(amax, std::fabs(v));
+  int e2 = 0;
+  if (amax > 0.f) std::frexp(amax, &e2);     // amax < 2^e2
+  const int sh = std::max(-60, std::min(60, 15 - e2));
+  std::vector<uint16_t> wh((size_t)d * kp, 0), wl((size_t)d * kp, 0);
+  for (int n = 0; n < d; ++n)
+    for (int k = 0; k < c.n_mels; ++k) {
+      const float v = std::ldexp(pw[(size_t)n * c.n_mels + k], sh);
+      const __half hi = __float2half_rn(v);
+      const __half lo16 = __float2half_rn(v - __half2float(hi));
+      wh[(size_t)n * kp + k] = __half_as_ushort(hi);
+      wl[(size_t)n * kp + k] = __half_as_ushort(lo16);
+    }
+
+  ms_cond* q = new (std::nothrow) ms_cond;
+  if (!q) return fail(MS_ERR_OOM, "ms_cond_create: host allocation failed");
+  q->cfg = c;
+  q->device = device;
+  q->frames = frames;
+  q->kp = kp;
+  q->yscale = std::ldexp(1.f, -sh);
+  const size_t rows = (size_t)c.max_batch * frames;
+  Arena a;
+  for (int pass = 0; pass < 2; ++pass) {
+    a.used = 0;
+    q->dev.window = a.take<float>(c.n_fft);
+    q->dev.twiddle = a.take<double2>(half);
+    q->dev.band_lo = a.take<int>(c.n_mels);
+    q->dev.band_off = a.take<int>(c.n_mels + 1);
+    q->dev.band_w = a.take<float>(bw.size());
+    q->wh = a.take<uint16_t>((size_t)d * kp);
+    q->wl = a.take<uint16_t>((size_t)d * kp);
+    q->bias = a.take<float>(d);
+    q->inst = a.take<float>((size_t)c.n_instruments * d);
+    q->ds = a.take<float>((size_t)c.n_datasets * d);
+    q->xh = a.take<__half>(rows * kp);
+    q->xl = a.take<__half>(rows * kp);
+    q->y = a.take<float>(rows * d);
+    q->status = a.take<unsigned>(1);
+    if (pass == 0) {
+      a.size = round_up(a.used, 256);
+      cudaError_t e = cudaMalloc(&a.base, a.size);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete q;
+        return fail(e == cudaErrorMemoryAllocation ? MS_ERR_OOM : MS_ERR_CUDA, "ms_cond_create: cudaMalloc(%zu): %s",
+                    a.size, cudaGetErrorString(e));
+      }
+      q->base = a.base;
+    }
+  }
+  q->dev.n_fft = c.n_fft;
+  q->dev.hop = c.hop;
+  q->dev.n_mels = c.n_mels;
+  q->dev.kp = kp;
+  auto cp = [&](const void* dst, const void* src, size_t bytes) -> cudaError_t {
+    return cudaMemcpy(const_cast<void*>(dst), src, bytes, cudaMemcpyDefault);
+  };
+  cudaError_t e = cp(q->dev.window, wt->window, (size_t)c.n_fft * 4);
+  if (e == cudaSuccess) e = cp(q->dev.twiddle, tw.data(), tw.size() * sizeof(double2));
+  if (e == cudaSuccess) e = cp(q->dev.band_lo, lo.data(), lo.size() * 4);
+  if (e == cudaSuccess) e = cp(q->dev.band_off, off.data(), off.size() * 4);
+  if (e == cudaSuccess) e = cp(q->dev.band_w, bw.data(), bw.size() * 4);
+  if (e == cudaSuccess) e = cp(q->wh, wh.data(), wh.size() * 2);
+  if (e == cudaSuccess) e = cp(q->wl, wl.data(), wl.size() * 2);
+  if (e == cudaSuccess) e = cp(q->bias, wt->proj_b, (size_t)d * 4);
+  if (e == cudaSuccess) e = cp(q->inst, wt->inst_emb, (size_t)c.n_instruments * d * 4);
+  if (e == cudaSuccess) e = cp(q->ds, wt->ds_emb, (size_t)c.n_datasets * d * 4);
+  if (e == cudaSuccess) e = cudaMemset(q->status, 0, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    delete q;
+    return fail(MS_ERR_CUDA, "ms_cond_create: copy: %s", cudaGetErrorString(e));
+  }
+  *out = q;
+  return MS_OK;
+}
+
+ms_status ms_cond_destroy(ms_cond* cond) {
+  if (!cond) return MS_OK;
+  DeviceGuard dg(cond->device);
+  delete cond;
+  return MS_OK;
+}
+
+int ms_cond_frames(const ms_cond* cond) { return cond ? cond->frames : 0; }
+
+ms_status ms_cond_log_mel(ms_cond* cond, const float* audio, int B, float* out, void* stream) {
+  if (!cond || !audio || !out) return fail(MS_ERR_INVALID_ARG, "ms_cond_log_mel: null argument");
+  if (B < 1 || B > cond->cfg.max_batch)
+    return fail(MS_ERR_SHAPE, "ms_cond_log_mel: B = %d outside 1..%d", B, cond->cfg.max_batch);
+  DeviceGuard dg(cond->device);
+  ms::Launch L{(cudaStream_t)stream, false, cond->status};
+  return check_launch(ms::launch_log_mel(L, audio, cond->cfg.n_samples, B, cond->dev, cond->frames, out, nullptr,
+                                         nullptr),
+                      "log_mel");
+}
+
+ms_status ms_condition(ms_cond* cond, const float* audio, int B, const int32_t* dataset, const int32_t* instruments,
+                       int K, float* prefix, void* stream) {
+  if (!cond || !audio || !dataset || !prefix || (K > 0 && !instruments))
+    return fail(MS_ERR_INVALID_ARG, "ms_condition: null argument");
+  if (B < 1 || B > cond->cfg.max_batch || K < 0 || K > 65536)
+    return fail(MS_ERR_SHAPE, "ms_condition: B = %d outside 1..%d or K = %d outside 0..65536", B,
+                cond->cfg.max_batch, K);
+  if (reinterpret_cast<uintptr_t>(prefix) & 15) return fail(MS_ERR_INVALID_ARG, "ms_condition: prefix must be 16-byte aligned");
+  DeviceGuard dg(cond->device);
+  int nsm = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, cond->device));
+  const ms::GemmWork gw{nsm > 0 ? nsm : 1};
+  const ms::GemmWeights none{nullptr, nullptr};
+  ms::Launch L{(cudaStream_t)stream, false, cond->status};
+  const int M = B * cond->frames, d = cond->cfg.d_model;
+  cudaError_t e = ms::launch_log_mel(L, audio, cond->cfg.n_samples, B, cond->dev, cond->frames, nullptr, cond->xh,
+                                     cond->xl);
+  if (e == cudaSuccess)
+    e = ms::launch_gemm_f16(L, cond_view(cond, cond->wh), none, cond->xh, cond->xl, cond->kp, M, cond->y, d, nullptr,
+                            nullptr, 0, ms::kStore, &gw);
+  if (e == cudaSuccess)
+    e = ms::launch_gemm_f16(L, cond_view(cond, cond->wl), none, cond->xh, cond->xl, cond->kp, M, cond->y, d, nullptr,
+                            nullptr, 0, ms::kAdd, &gw);
+  if (e == cudaSuccess)
+    e = ms::launch_cond_assemble(L, cond->y, cond->yscale, cond->bias, cond->ds, cond->cfg.n_datasets, cond->inst,
+                                 cond->cfg.n_instruments, dataset, instruments, K, cond->frames, d, B, prefix);
+  return check_launch(e, "ms_condition");
+}
+
+ms_status ms_cond_device_status(ms_cond* cond, void* stream) {
+  if (!cond) return fail(MS_ERR_INVALID_ARG, "ms_cond_device_status: null cond");
+  DeviceGuard dg(cond->device);
+  CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned w = 0;
+  CUDA_TRY(cudaMemcpy(&w, cond->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  const unsigned zero = 0;
+  CUDA_TRY(cudaMemcpy(cond->status, &zero, sizeof(unsigned), cudaMemcpyHostToDevice));
+  if (w & ms::kErrTokenBit)
+    return fail(MS_ERR_TOKEN_RANGE, "a dataset or instrument id was outside its table (status 0x%x)", w);
+  if (w & ms::kErrShapeBit) return fail(MS_ERR_SHAPE, "a device-side size check failed (status 0x%x)", w);
+  return MS_OK;
 }
 
 }  // extern "C"

@@ -336,6 +336,69 @@ ms_status ms_op_lm_head_argmax_static(const float* x, int ldx, int M, int d, con
                                       const float* beta, float eps, const float* W, int V,
                                       float* logits, int32_t* argmax, void* stream);
 
+/* ---- conditioner front-end ------------------------------------------------------------
+ * "MuScriptor small — ONNX conversion", the conditioner graph muscriptor-small-cond.onnx:
+ * audio fp32 [1, N] at 16 kHz, instrument ids [1, K] and a dataset id -> the decoder's prefix
+ * [1, frames + 1 + K, d]; the spectrogram is computed inside that graph from a window and a mel
+ * filterbank stored with the checkpoint.  MuScriptor model card, Model description: STFT with
+ * n_fft 2048 and hop 160, 512 mel bands, log features, a projection to d_model.
+ * The conditioner computes, per stream b:
+ *   frame t (t = 0 .. frames-1, frames = 1 + n_samples / hop) = samples t*hop - n_fft/2 ..
+ *     t*hop + n_fft/2 - 1 of the signal extended by reflection at both ends (sample -i is
+ *     sample i, sample N-1+i is sample N-1-i; the edge sample is not repeated), times window;
+ *   mag[t][k] = |DFT(frame t)[k]|, k = 0 .. n_fft/2;
+ *   logmel[t][m] = ln(max(sum_k mel_fb[m][k] * mag[t][k], 1e-6));
+ *   prefix[b][t] = logmel[t] . proj_w^T + proj_b (t < frames);
+ *   prefix[b][frames] = ds_emb[dataset[b]];  prefix[b][frames + 1 + k] = inst_emb[instruments[b][k]].
+ * Which of these steps the pages leave open and how they are read here: centred frames with
+ * reflection, the magnitude (not the power), the natural log, and the row order (frames,
+ * dataset, instruments), which gives the decoder's 503 prefix rows for 501 frames and one
+ * instrument.
+ * Arithmetic: window, DFT, magnitudes, mel sums and log in double precision, rounded to fp32;
+ * the projection on the tensor cores with the features and the weights each as an fp16 hi + lo
+ * pair (the weights scaled by a power of two first) and fp32 accumulation; bias in fp32. */
+typedef struct ms_cond ms_cond;
+
+typedef struct {
+  int n_samples;      /* audio samples per stream (80000: 5 s at 16 kHz); > n_fft / 2 */
+  int n_fft;          /* a power of two, 16 .. 4096 (2048) */
+  int hop;            /* frame step in samples, >= 1 (160) */
+  int n_mels;         /* mel bands, 1 .. 4096 (512) */
+  int d_model;        /* width of the prefix rows (the decoder's d_model), a multiple of 4 */
+  int n_instruments;  /* rows of the instrument table, >= 1 (130) */
+  int n_datasets;     /* rows of the dataset table, >= 1 (2) */
+  int max_batch;      /* most streams one call may take, >= 1 (work buffers are sized for it) */
+} ms_cond_config;
+
+typedef struct {              /* host or device pointers; copied at create; caller keeps ownership */
+  const float* window;        /* [n_fft] */
+  const float* mel_fb;        /* [n_mels][n_fft/2 + 1], row m = band m's weight of each bin */
+  const float* proj_w;        /* [d_model][n_mels] */
+  const float* proj_b;        /* [d_model] */
+  const float* inst_emb;      /* [n_instruments][d_model] */
+  const float* ds_emb;        /* [n_datasets][d_model] */
+} ms_cond_weights;
+
+/* Copies the weights to `device` and allocates the work buffers for max_batch streams
+ * (about max_batch * frames * (4 * n_mels + 4 * d_model) bytes).  MS_ERR_INVALID_ARG for NULL
+ * pointers or a config outside the ranges above, MS_ERR_OOM, MS_ERR_CUDA. */
+ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* w, int device, ms_cond** out);
+ms_status ms_cond_destroy(ms_cond* cond);
+/* frames = 1 + n_samples / hop (501 for 5 s at 16 kHz and hop 160); 0 on NULL. */
+int ms_cond_frames(const ms_cond* cond);
+/* The prefix of B streams (1 <= B <= max_batch): audio fp32 [B][n_samples], dataset int32 [B],
+ * instruments int32 [B][K] (K >= 0; may be NULL when K = 0) -> prefix fp32
+ * [B][frames + 1 + K][d_model], 16-byte aligned.  Device pointers of the cond's device;
+ * asynchronous on `stream`.  An id outside its table is clamped on the device and flagged:
+ * ms_cond_device_status then returns MS_ERR_TOKEN_RANGE.  Calls on one cond share its work
+ * buffers: order them on one stream. */
+ms_status ms_condition(ms_cond* cond, const float* audio, int B, const int32_t* dataset,
+                       const int32_t* instruments, int K, float* prefix, void* stream);
+/* The log-mel features alone: audio fp32 [B][n_samples] -> out fp32 [B][frames][n_mels]. */
+ms_status ms_cond_log_mel(ms_cond* cond, const float* audio, int B, float* out, void* stream);
+/* Synchronises `stream`, reads and clears the cond's device status word. */
+ms_status ms_cond_device_status(ms_cond* cond, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -110,3 +110,33 @@ def test_guidance_rejects_null_cache():
     import ctypes
     assert ms._lib.ms_cache_set_guidance(None, ctypes.c_float(2.0)) == ms.MS_ERR_INVALID_ARG
     assert ms._lib.ms_cache_guidance(None) == 0.0
+
+
+def _cond_cfg(**change):
+    c = ms.CondConfig(80000, 2048, 160, 512, 1024, 130, 2, 1)
+    for k, v in change.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_cond_create_rejects_bad_configs_on_the_host():
+    buf = (ctypes.c_float * 16)()
+    p = ctypes.cast(buf, ctypes.c_void_p).value
+    W = ms.CondWeights(p, p, p, p, p, p)
+    out = ctypes.c_void_p()
+    bad = [dict(n_fft=2000), dict(n_fft=8), dict(n_fft=8192), dict(hop=0), dict(n_samples=1024),
+           dict(n_mels=0), dict(n_mels=5000), dict(d_model=1022), dict(n_instruments=0), dict(n_datasets=0),
+           dict(max_batch=0)]
+    for change in bad:
+        st = ms._lib.ms_cond_create(ctypes.byref(_cond_cfg(**change)), ctypes.byref(W), 0, ctypes.byref(out))
+        assert st == ms.MS_ERR_INVALID_ARG, (change, ms.last_error())
+        assert out.value is None
+    W0 = ms.CondWeights(p, None, p, p, p, p)
+    assert ms._lib.ms_cond_create(ctypes.byref(_cond_cfg()), ctypes.byref(W0), 0, ctypes.byref(out)) == \
+        ms.MS_ERR_INVALID_ARG
+    assert ms._lib.ms_cond_create(None, ctypes.byref(W), 0, ctypes.byref(out)) == ms.MS_ERR_INVALID_ARG
+    assert ms._lib.ms_cond_frames(None) == 0
+    assert ms._lib.ms_cond_destroy(None) == ms.MS_OK
+    assert ms._lib.ms_condition(None, None, 1, None, None, 0, None, None) == ms.MS_ERR_INVALID_ARG
+    assert ms._lib.ms_cond_log_mel(None, None, 1, None, None) == ms.MS_ERR_INVALID_ARG
+    assert ms._lib.ms_cond_device_status(None, None) == ms.MS_ERR_INVALID_ARG
