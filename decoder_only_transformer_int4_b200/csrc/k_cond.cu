@@ -5,9 +5,10 @@
 //
 // log_mel_kernel: one CTA per (frame, stream).  The frame is the reflection-padded, centred
 // slice of the signal times the stored window; its real DFT is taken as a complex DFT of half
-// the length (even samples in the real part, odd ones in the imaginary part; radix-2,
-// decimation in time, in shared memory) followed by the split into the even and odd halves'
-// spectra.  All of it in double precision: the magnitudes feed a logarithm, which turns an
+// the length (even samples in the real part, odd ones in the imaginary part; radix-4
+// decimation-in-frequency stages in shared memory, the first taken on the values as they are
+// read, outputs left in digit-reversed order) followed by the split into the even and odd
+// halves' spectra.  All of it in double precision: the magnitudes feed a logarithm, which turns an
 // fp32 FFT's absolute error into a large relative error in low-energy bands.  Each mel band is
 // the weighted sum of its own range of bins (the filterbank rows are stored compressed to
 // their non-zero range), floored at 1e-6 and logged.  The result leaves as fp32 rows and / or
@@ -27,18 +28,56 @@ namespace ms {
 
 namespace {
 
+// Position, after the decimation-in-frequency stages below, of frequency k of the half-length
+// transform: the stages take radix 4 from the full length down (radix 2 last when log2(half) is
+// odd), and each stage's output digit selects a quarter (half) of the current span.
+__device__ __forceinline__ int dif_pos(int k, int half) {
+  int p = 0, span = half;
+  while (span > 1) {
+    const int r = span >= 4 ? 4 : 2;
+    span /= r;
+    p += (k % r) * span;
+    k /= r;
+  }
+  return p;
+}
+
+__device__ __forceinline__ double2 cmul(double2 a, double2 w) {
+  return make_double2(a.x * w.x - a.y * w.y, a.x * w.y + a.y * w.x);
+}
+
+// One radix-4 decimation-in-frequency butterfly on a0..a3 = x[t1 + q * L/4] of a span of length
+// L: the 4-point DFT over q, output digit m times W_L^{t1 m} (the twiddle table holds
+// W_{n_fft}^i, so W_L^j = table[j * n_fft / L]).
+__device__ __forceinline__ void dif4(double2& a0, double2& a1, double2& a2, double2& a3, int t1, int tstep,
+                                     const double2* __restrict__ tw) {
+  const double2 s02 = make_double2(a0.x + a2.x, a0.y + a2.y), d02 = make_double2(a0.x - a2.x, a0.y - a2.y);
+  const double2 s13 = make_double2(a1.x + a3.x, a1.y + a3.y), d13 = make_double2(a1.x - a3.x, a1.y - a3.y);
+  a0 = make_double2(s02.x + s13.x, s02.y + s13.y);
+  const double2 c2 = make_double2(s02.x - s13.x, s02.y - s13.y);
+  const double2 c1 = make_double2(d02.x + d13.y, d02.y - d13.x);   // d02 - i d13
+  const double2 c3 = make_double2(d02.x - d13.y, d02.y + d13.x);   // d02 + i d13
+  if (t1 == 0) {
+    a1 = c1, a2 = c2, a3 = c3;
+  } else {
+    a1 = cmul(c1, __ldg(tw + t1 * tstep));
+    a2 = cmul(c2, __ldg(tw + 2 * t1 * tstep));
+    a3 = cmul(c3, __ldg(tw + 3 * t1 * tstep));
+  }
+}
+
 __global__ void __launch_bounds__(256) log_mel_kernel(const float* __restrict__ audio, int n_samples, CondDev c,
                                                       int frames, float* __restrict__ out, __half* __restrict__ xh,
                                                       __half* __restrict__ xl) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int half = c.n_fft >> 1;
+  const int half = c.n_fft >> 1, q4 = half >> 2;
   double2* z = reinterpret_cast<double2*>(smem_raw);            // [half]
   double* mag = reinterpret_cast<double*>(z + half);            // [half + 1]
   const int t = blockIdx.x, b = blockIdx.y;
   const float* x = audio + (size_t)b * n_samples;
-  const int lg = 31 - __clz(half);
-  // frame samples 2n and 2n+1, windowed, into the bit-reversed slot of n
-  for (int n = threadIdx.x; n < half; n += blockDim.x) {
+  // z[n] = (f[2n], f[2n+1]), f = window x the frame; the first radix-4 stage (span = half) is
+  // taken on the values as they arrive
+  auto frame_pair = [&](int n) {
     double f[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -46,24 +85,37 @@ __global__ void __launch_bounds__(256) log_mel_kernel(const float* __restrict__ 
       int j = t * c.hop + m - half;                               // index into the unpadded signal
       if (j < 0) j = -j;                                          // reflection without the edge sample
       if (j >= n_samples) j = 2 * (n_samples - 1) - j;
-      f[e] = (double)__ldg(c.window + m) * (double)__ldg(x + j);
+      f[e] = __ldg(c.window + m) * (double)__ldg(x + j);
     }
-    const int r = lg ? (int)(__brev((unsigned)n) >> (32 - lg)) : 0;
-    z[r] = make_double2(f[0], f[1]);
+    return make_double2(f[0], f[1]);
+  };
+  int span = half;
+  if (half >= 4) {
+    for (int t1 = threadIdx.x; t1 < q4; t1 += blockDim.x) {
+      double2 a0 = frame_pair(t1), a1 = frame_pair(t1 + q4), a2 = frame_pair(t1 + 2 * q4), a3 = frame_pair(t1 + 3 * q4);
+      dif4(a0, a1, a2, a3, t1, c.n_fft / half, c.twiddle);
+      z[t1] = a0, z[t1 + q4] = a1, z[t1 + 2 * q4] = a2, z[t1 + 3 * q4] = a3;
+    }
+    span = q4;
+  } else {
+    for (int n = threadIdx.x; n < half; n += blockDim.x) z[n] = frame_pair(n);
   }
   __syncthreads();
-  // radix-2 stages of the half-length complex DFT; the twiddles of the full length serve it
-  // at every second index
-  for (int h = 1; h < half; h <<= 1) {
-    const int step = c.n_fft / (2 * h);
+  for (; span >= 4; span >>= 2) {
+    const int L4 = span >> 2, tstep = c.n_fft / span;
+    for (int i = threadIdx.x; i < q4; i += blockDim.x) {
+      const int t1 = i % L4, base = (i / L4) * span + t1;
+      double2 a0 = z[base], a1 = z[base + L4], a2 = z[base + 2 * L4], a3 = z[base + 3 * L4];
+      dif4(a0, a1, a2, a3, t1, tstep, c.twiddle);
+      z[base] = a0, z[base + L4] = a1, z[base + 2 * L4] = a2, z[base + 3 * L4] = a3;
+    }
+    __syncthreads();
+  }
+  if (span == 2) {                                              // a last radix-2 stage
     for (int i = threadIdx.x; i < (half >> 1); i += blockDim.x) {
-      const int j = i & (h - 1);
-      const int p = ((i - j) << 1) + j, q = p + h;
-      const double2 w = __ldg(c.twiddle + j * step);
-      const double2 u = z[p], v = z[q];
-      const double vr = v.x * w.x - v.y * w.y, vi = v.x * w.y + v.y * w.x;
-      z[p] = make_double2(u.x + vr, u.y + vi);
-      z[q] = make_double2(u.x - vr, u.y - vi);
+      const double2 a0 = z[2 * i], a1 = z[2 * i + 1];
+      z[2 * i] = make_double2(a0.x + a1.x, a0.y + a1.y);
+      z[2 * i + 1] = make_double2(a0.x - a1.x, a0.y - a1.y);
     }
     __syncthreads();
   }
@@ -73,7 +125,7 @@ __global__ void __launch_bounds__(256) log_mel_kernel(const float* __restrict__ 
       const double2 z0 = z[0];
       mag[k] = fabs(k == 0 ? z0.x + z0.y : z0.x - z0.y);
     } else {
-      const double2 a = z[k], cz = z[half - k];
+      const double2 a = z[dif_pos(k, half)], cz = z[dif_pos(half - k, half)];
       const double er = 0.5 * (a.x + cz.x), ei = 0.5 * (a.y - cz.y);     // (a + conj(cz)) / 2
       const double orr = 0.5 * (a.y + cz.y), oi = -0.5 * (a.x - cz.x);  // (a - conj(cz)) / 2i
       const double2 w = __ldg(c.twiddle + k);

@@ -119,8 +119,8 @@ cudaError_t init_attrs_w4a8();
 // CTA per frame and stream, double-precision FFT), and the prefix rows after the projection.
 constexpr int kCondMaxFft = 4096;
 struct CondDev {
-  const float* window;     // [n_fft]
-  const double2* twiddle;  // [n_fft / 2]: e^{-2 pi i k / n_fft}
+  const double* window;    // [n_fft]
+  const double2* twiddle;  // [n_fft]: e^{-2 pi i k / n_fft}
   const int* band_lo;      // [n_mels]: first bin of band m's non-zero range
   const int* band_off;     // [n_mels + 1]: band m's weights are band_w[band_off[m] .. band_off[m+1])
   const float* band_w;

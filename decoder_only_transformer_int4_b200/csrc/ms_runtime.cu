@@ -1299,6 +1299,9 @@ ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* wt, i
   std::vector<float> fb((size_t)c.n_mels * nf), pw((size_t)d * c.n_mels);
   CUDA_TRY(cudaMemcpy(fb.data(), wt->mel_fb, fb.size() * 4, cudaMemcpyDefault));
   CUDA_TRY(cudaMemcpy(pw.data(), wt->proj_w, pw.size() * 4, cudaMemcpyDefault));
+  std::vector<float> win32(c.n_fft);
+  CUDA_TRY(cudaMemcpy(win32.data(), wt->window, win32.size() * 4, cudaMemcpyDefault));
+  const std::vector<double> win(win32.begin(), win32.end());
   // each filterbank row compressed to its non-zero range
   std::vector<int> lo(c.n_mels), off(c.n_mels + 1, 0);
   std::vector<float> bw;
@@ -1315,10 +1318,10 @@ ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* wt, i
     off[m + 1] = (int)bw.size();
   }
   if (bw.empty()) bw.push_back(0.f);
-  // twiddles e^{-2 pi i k / n_fft}, k < n_fft / 2, in double on the host
-  std::vector<double2> tw(half);
+  // twiddles e^{-2 pi i k / n_fft}, k < n_fft, in double on the host; the window in double
+  std::vector<double2> tw(c.n_fft);
   const double two_pi = 6.283185307179586476925286766559;
-  for (int k = 0; k < half; ++k) {
+  for (int k = 0; k < c.n_fft; ++k) {
     const double a = two_pi * (double)k / (double)c.n_fft;
     tw[k] = make_double2(std::cos(a), -std::sin(a));
   }
@@ -1349,8 +1352,8 @@ ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* wt, i
   Arena a;
   for (int pass = 0; pass < 2; ++pass) {
     a.used = 0;
-    q->dev.window = a.take<float>(c.n_fft);
-    q->dev.twiddle = a.take<double2>(half);
+    q->dev.window = a.take<double>(c.n_fft);
+    q->dev.twiddle = a.take<double2>(c.n_fft);
     q->dev.band_lo = a.take<int>(c.n_mels);
     q->dev.band_off = a.take<int>(c.n_mels + 1);
     q->dev.band_w = a.take<float>(bw.size());
@@ -1382,7 +1385,7 @@ ms_status ms_cond_create(const ms_cond_config* cfg, const ms_cond_weights* wt, i
   auto cp = [&](const void* dst, const void* src, size_t bytes) -> cudaError_t {
     return cudaMemcpy(const_cast<void*>(dst), src, bytes, cudaMemcpyDefault);
   };
-  cudaError_t e = cp(q->dev.window, wt->window, (size_t)c.n_fft * 4);
+  cudaError_t e = cp(q->dev.window, win.data(), win.size() * sizeof(double));
   if (e == cudaSuccess) e = cp(q->dev.twiddle, tw.data(), tw.size() * sizeof(double2));
   if (e == cudaSuccess) e = cp(q->dev.band_lo, lo.data(), lo.size() * 4);
   if (e == cudaSuccess) e = cp(q->dev.band_off, off.data(), off.size() * 4);
