@@ -245,175 +245,4 @@ cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, 
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Prefill: causal flash attention on CUDA cores.  Grid (ceil(n / 64), H, B): one CTA per
-// 64 new query rows of one head.  Key tiles of 64 from position 0 up to the tile's last
-// query; running max and sum per row; scores never leave shared memory.  Query rows are
-// at positions len + i, the keys are the cache rows rope_append has just written.
-// ---------------------------------------------------------------------------------
-namespace {
-constexpr int kPreT = 64;
-constexpr int kPrePad = kPreT + 4;
-
-struct AttnPreArgs {
-  const float* q;
-  const void* kc;   // fp32 or IEEE half elements (the kernel's KV parameter)
-  const void* vc;
-  int B, n, H, Hk, cap;
-  const int* dlen;
-  float* o;
-};
-
-constexpr size_t kPreSmem = sizeof(float) * (3 * 64 * kPrePad + 64 * 64);
-}  // namespace
-
-template <int KV>
-__global__ void __launch_bounds__(256) attn_prefill_kernel(AttnPreArgs a) {
-  extern __shared__ __align__(16) float sm[];
-  float(*Qs)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm);                   // [d][row]
-  float(*Ks)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm + 64 * kPrePad);    // [d][key]
-  float(*Ps)[kPrePad] = reinterpret_cast<float(*)[kPrePad]>(sm + 2 * 64 * kPrePad);  // [key][row]
-  float(*Vs)[64] = reinterpret_cast<float(*)[64]>(sm + 3 * 64 * kPrePad);          // [key][d]
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int g = h / (a.H / a.Hk);
-  pdl_wait();
-  pdl_trigger();
-  const int pos0 = *a.dlen;
-  const int i0 = qt * kPreT;
-  const int ivalid = min(kPreT, a.n - i0);
-  const int kend = pos0 + i0 + ivalid;  // keys [0, kend) are needed
-
-  for (int idx = tid; idx < kPreT * 16; idx += 256) {
-    const int r = idx >> 4, f = idx & 15;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < ivalid) v = reinterpret_cast<const float4*>(a.q + ((size_t)b * a.n + i0 + r) * a.H * 64 + h * 64)[f];
-    Qs[4 * f + 0][r] = v.x * 0.125f;
-    Qs[4 * f + 1][r] = v.y * 0.125f;
-    Qs[4 * f + 2][r] = v.z * 0.125f;
-    Qs[4 * f + 3][r] = v.w * 0.125f;
-  }
-  float m_i[4], l_i[4], O[4][4];
-  int qpos[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m_i[i] = -INFINITY;
-    l_i[i] = 0.f;
-    qpos[i] = pos0 + i0 + ty * 4 + i;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) O[i][j] = 0.f;
-  }
-  const size_t head = ((size_t)b * a.Hk + g) * a.cap * 64;   // first element of the head's rows
-
-  for (int c0 = 0; c0 < kend; c0 += kPreT) {
-    __syncthreads();
-    for (int idx = tid; idx < kPreT * 16; idx += 256) {
-      const int r = idx >> 4, f = idx & 15;
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-      if (c0 + r < kend) {
-        kv = kv_load4<KV>(a.kc, head + (size_t)(c0 + r) * 64 + 4 * f);
-        vv = kv_load4<KV>(a.vc, head + (size_t)(c0 + r) * 64 + 4 * f);
-      }
-      Ks[4 * f + 0][r] = kv.x;
-      Ks[4 * f + 1][r] = kv.y;
-      Ks[4 * f + 2][r] = kv.z;
-      Ks[4 * f + 3][r] = kv.w;
-      reinterpret_cast<float4*>(&Vs[r][0])[f] = vv;
-    }
-    __syncthreads();
-    float s[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
-#pragma unroll 8
-    for (int dd = 0; dd < 64; ++dd) {
-      const float4 qa = *reinterpret_cast<const float4*>(&Qs[dd][ty * 4]);
-      const float4 kk = *reinterpret_cast<const float4*>(&Ks[dd][tx * 4]);
-      const float qr[4] = {qa.x, qa.y, qa.z, qa.w};
-      const float kr[4] = {kk.x, kk.y, kk.z, kk.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) s[i][j] = fmaf(qr[i], kr[j], s[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int key = c0 + tx * 4 + j;
-        if (key > qpos[i] || key >= kend) s[i][j] = -INFINITY;
-        mx = fmaxf(mx, s[i][j]);
-      }
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float mnew = fmaxf(m_i[i], mx);
-      const float cf = mnew == -INFINITY ? 1.f : expf(m_i[i] - mnew);
-      float rs = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float p = s[i][j] == -INFINITY ? 0.f : expf(s[i][j] - mnew);
-        s[i][j] = p;
-        rs += p;
-      }
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
-      l_i[i] = l_i[i] * cf + rs;
-      m_i[i] = mnew;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) O[i][j] *= cf;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) Ps[tx * 4 + j][ty * 4 + i] = s[i][j];
-    __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < kPreT; ++c) {
-      const float4 pa = *reinterpret_cast<const float4*>(&Ps[c][ty * 4]);
-      const float4 vv = *reinterpret_cast<const float4*>(&Vs[c][tx * 4]);
-      const float pr[4] = {pa.x, pa.y, pa.z, pa.w};
-      const float vr[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) O[i][j] = fmaf(pr[i], vr[j], O[i][j]);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty * 4 + i;
-    if (r >= ivalid) continue;
-    const float inv = 1.0f / l_i[i];
-    float4 v = make_float4(O[i][0] * inv, O[i][1] * inv, O[i][2] * inv, O[i][3] * inv);
-    reinterpret_cast<float4*>(a.o + ((size_t)b * a.n + i0 + r) * a.H * 64 + h * 64)[tx] = v;
-  }
-}
-
-cudaError_t init_attrs_attn() {
-  cudaError_t e = allow_smem(attn_prefill_kernel<0>, kMaxDynSmem);
-  if (e == cudaSuccess) e = allow_smem(attn_prefill_kernel<1>, kMaxDynSmem);
-  return e;
-}
-
-cudaError_t launch_attn_prefill(const Launch& L, const float* q, const void* kc, const void* vc, int B, int n,
-                                int H, int Hk, int cap, const int* dlen, float* o, int kv16) {
-  if (n <= 0) return cudaSuccess;
-  AttnPreArgs a;
-  a.q = q;
-  a.kc = kc;
-  a.vc = vc;
-  a.B = B;
-  a.n = n;
-  a.H = H;
-  a.Hk = Hk;
-  a.cap = cap;
-  a.dlen = dlen;
-  a.o = o;
-  const dim3 grid((n + kPreT - 1) / kPreT, H, B);
-  if (kv16) return launch_k(L, attn_prefill_kernel<1>, grid, dim3(256), kPreSmem, a);
-  return launch_k(L, attn_prefill_kernel<0>, grid, dim3(256), kPreSmem, a);
-}
-
 }  // namespace ms

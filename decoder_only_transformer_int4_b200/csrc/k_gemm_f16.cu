@@ -39,6 +39,7 @@
 
 #include "ms_device.cuh"
 #include "ms_launch.cuh"
+#include "ms_tc.cuh"
 
 namespace ms {
 
@@ -92,54 +93,8 @@ __device__ __forceinline__ float ld_peer(uint32_t local_saddr, uint32_t rank) {
   return v;
 }
 
-// K-major operand tile with 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes
-// apart (stride byte offset), descriptor version 1, layout type 2 (SWIZZLE_128B).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 // Instruction descriptor, kind::f16: D fp32, A and B fp16, both K-major, M = 128, N = bn.
-__device__ __forceinline__ uint32_t idesc_f16(int bn) {
-  return (1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(GM >> 4) << 24);
-}
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
-          tmem_d),
-      "l"(da), "l"(db), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// 2-D TMA tile load (x = inner coordinate in elements, y = row), completing on bar.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ uint32_t sw128(int r, int chunk) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4));
-}
-__device__ __forceinline__ uint32_t pack_h2(float lo_elem, float hi_elem) {  // element order: lo first
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_elem), "f"(lo_elem));
-  return r;
-}
-__device__ __forceinline__ float2 unpack_h2(uint32_t h) {
-  const __half2 v = *reinterpret_cast<const __half2*>(&h);
-  return __half22float2(v);
-}
+__device__ __forceinline__ uint32_t idesc_f16(int bn) { return idesc_f16_mn(GM, bn, false); }
 
 }  // namespace
 

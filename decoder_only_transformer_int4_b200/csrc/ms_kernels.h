@@ -45,7 +45,6 @@ void set_last_error(const char* msg);
 
 // Opt every kernel that needs it into large dynamic shared memory on the current device.
 cudaError_t init_attrs_gemv();
-cudaError_t init_attrs_attn();
 
 cudaError_t launch_quantize_int4(const float* w, int N, int K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
@@ -115,6 +114,16 @@ cudaError_t launch_matmul_w4a8(const Launch& L, const WView& w, const int8_t* qa
                                int M, float* y, int ldy, int epi, int sms);
 cudaError_t init_attrs_w4a8();
 
+// Causal prefill attention on the tensor cores (tcgen05, fp16 hi / lo operands, three products):
+// q [B * n][H * 64] post-RoPE, the layer's cache slices, positions len .. len + n - 1 with len
+// read from dlen; the result as fp32 rows o [B * n][H * 64] and / or fp16 hi / lo planes
+// oh, ol [B * n][ldo] (ldo a multiple of 8).  H / Hk query heads per kv head, at most 128.
+bool attn_prefill_tc_fits(int H, int Hk);
+cudaError_t init_attrs_attn_tc();
+cudaError_t launch_attn_prefill_tc(const Launch& L, const float* q, const void* kc, const void* vc, int B, int n,
+                                   int H, int Hk, int cap, const int* dlen, float* o, __half* oh, __half* ol, int ldo,
+                                   int kv16);
+
 // Conditioner front-end: the log-mel spectrogram of centred, reflection-padded frames (one
 // CTA per frame and stream, double-precision FFT), and the prefix rows after the projection.
 constexpr int kCondMaxFft = 4096;
@@ -150,10 +159,6 @@ cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, 
                                int B, int H, int Hk, int cap, const int* dlen, int add,
                                const AttnDecodeWork& w, float* o, int kv16);
 int attn_decode_splits(int B, int Hk, int cap);
-
-// Causal prefill attention for n new rows per stream at positions len .. len + n - 1.
-cudaError_t launch_attn_prefill(const Launch& L, const float* q, const void* kc, const void* vc,
-                                int B, int n, int H, int Hk, int cap, const int* dlen, float* o, int kv16);
 
 // LM head + argmax over rows x[m * ldx], m < M.  Writes logits (may be null), argmax
 // (may be null), hist[(len + hist_off) * B + m] (may be null) and, in its last CTA,

@@ -141,11 +141,11 @@ cudaError_t ensure_kernel_attributes() {
   if ((int)g_attr_done.size() <= dev) g_attr_done.resize(dev + 1, 0);
   if (g_attr_done[dev]) return cudaSuccess;
   e = ms::init_attrs_gemv();
-  if (e == cudaSuccess) e = ms::init_attrs_attn();
   if (e == cudaSuccess) e = ms::init_attrs_persistent();
   if (e == cudaSuccess) e = ms::init_attrs_gemm_f16();
   if (e == cudaSuccess) e = ms::init_attrs_w4a8();
   if (e == cudaSuccess) e = ms::init_attrs_cond();
+  if (e == cudaSuccess) e = ms::init_attrs_attn_tc();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -256,7 +256,8 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
     if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
     if (e == cudaSuccess)
       e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
-    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, c->kv16);
+    if (e == cudaSuccess)
+      e = ms::launch_attn_prefill_tc(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, nullptr, nullptr, 0, c->kv16);
     if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
     if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], c->h, d, R, c->u, F, ms::kGelu);
@@ -275,8 +276,8 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
       e = ms::launch_gemm_f16(L, ly.w[0], ly.gw[0], c->hh, c->hl, kh, R, c->qkv, nq, nullptr, nullptr, 0, ms::kStore, &gw);
     if (e == cudaSuccess)
       e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
-    if (e == cudaSuccess) e = ms::launch_attn_prefill(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, c->kv16);
-    if (e == cudaSuccess) e = ms::launch_split_f16(L, c->o, H * 64, R, H * 64, c->hh, c->hl, kh);
+    if (e == cudaSuccess)
+      e = ms::launch_attn_prefill_tc(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, nullptr, c->hh, c->hl, kh, c->kv16);
     if (e == cudaSuccess)
       e = ms::launch_gemm_f16(L, ly.w[1], ly.gw[1], c->hh, c->hl, kh, R, c->y, d, nullptr, nullptr, 0, ms::kStore, &gw);
     if (e == cudaSuccess)
