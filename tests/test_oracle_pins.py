@@ -1018,3 +1018,31 @@ def test_conditioner_planted_mistakes_are_caught(monkeypatch, mistake):
     empty = np.where(cond.mel_fb.sum(axis=1) == 0)[0]
     caught = caught or not np.all(lm[:, empty] == np.log(1e-6))
     assert caught, mistake
+
+
+def test_stored_buffers_match_the_pages_figures():
+    """The page puts the stored window and filterbank about 2.4e-4 from the textbook ones (the
+    half rounding of values in [0.5, 1) moves them by up to 2^-12 = 2.44e-4), and says that with
+    them the bins the textbook buffers leave at the log(1e-6) floor sit near -4.  For the
+    440 Hz tone (amplitude 0.5; the page's amplitude is not given) those bands land between -7
+    and -3, and they are at the floor with the textbook buffers."""
+    figs = _gold("pages_figures.json")
+    cond = synth.make_cond_weights(8)
+    hann = 0.5 - 0.5 * np.cos(2 * np.pi * np.arange(2048) / 2048)
+    freqs = np.linspace(0, 8000, 1025)
+    mel = lambda f: 2595 * np.log10(1 + f / 700)
+    pts = 700 * (10 ** (np.linspace(0, mel(8000.0), 514) / 2595) - 1)
+    fb = np.maximum(0, np.minimum((freqs[None] - pts[:-2, None]) / (pts[1:-1] - pts[:-2])[:, None],
+                                  (pts[2:, None] - freqs[None]) / (pts[2:] - pts[1:-1])[:, None]))
+    dev = figs["cond_buffer_deviation"]["value"]
+    assert abs(np.abs(cond.window - hann).max() - dev) < 0.05e-4
+    # the filterbank's fresh computation is fp32 arithmetic (up to ~3e-5 from these fp64 triangles)
+    assert abs(np.abs(cond.mel_fb - fb).max() - dev) < 0.4e-4
+    tone = synth.make_tone(1)[0].astype(np.float64)
+    lm_text = O.log_mel(O.stft_magnitude(tone, hann, synth.HOP), fb)[250]
+    lm_stored = O.log_mel(O.stft_magnitude(tone, cond.window, synth.HOP), cond.mel_fb)[250]
+    floor = np.log(figs["cond_floor_bins_stored"]["floor"])
+    at_floor = (lm_text <= floor + 1e-9) & (fb.sum(axis=1) > 0)
+    assert at_floor.sum() >= 20
+    near = figs["cond_floor_bins_stored"]["value"]
+    assert np.all(np.abs(lm_stored[at_floor] - near) <= 3.0)
