@@ -9,11 +9,11 @@
 // One CTA per (128-row tile, kv group, stream).  A tile stacks the hpg = H / Hk query heads of
 // the group: row r = hh * prows + p is head g * hpg + hh at new row i0 + p (prows = 128 / hpg
 // rounded down), so every key tile staged in shared memory serves all of the group's heads.
-// Per key tile of 64 positions:
+// Per key tile of 64 positions (the next tile's K and V loads in flight meanwhile):
 //   S = Q K^T on the tensor cores (M = 128 rows, N = 64 keys, K = 64) into TMEM;
 //   online softmax on the CUDA cores: the two threads of a row (warps w and w + 4 read the same
-//   TMEM lane quarter) both take the row maximum over the 64 scores, each exponentiates its 32
-//   and writes them as the A operand of the next product;
+//   TMEM lane quarter) each read their 32 scores, exchange their maxima through shared memory,
+//   exponentiate their 32 and write them as the A operand of the next product;
 //   O_tile = P V (M = 128, N = 64 head dims, K = 64 keys) into TMEM, with V read as an MN-major
 //   operand straight from its row-per-key tile; each thread adds its 32 columns into registers
 //   after scaling them by the softmax correction.
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kAtThreads, 2) attn_prefill_tc_kernel(const At
   extern __shared__ __align__(1024) unsigned char dsm[];
   __shared__ uint64_t bar_s, bar_o, bar_end;
   __shared__ uint32_t tmem_base_s;
-  __shared__ float red[2][kAtRows];
+  __shared__ float red[2][kAtRows], red_m[2][kAtRows];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -139,19 +139,34 @@ __global__ void __launch_bounds__(kAtThreads, 2) attn_prefill_tc_kernel(const At
   const int nkt = (kend + kAtKeys - 1) / kAtKeys;
   bool ok = true;
 
+  // K and V of a key tile travel in registers: each thread holds 4 float4 of K and of V
+  // (key = (tid + 256 i) / 16, elements 4 f .. 4 f + 3 with f = (tid + 256 i) % 16); the next
+  // tile's loads are issued right after the current one is staged, so they are in flight
+  // during the current tile's products and softmax.
+  float4 pk[4], pv[4];
+  auto load_kv = [&](int c0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + kAtThreads * i, key = idx >> 4, f = idx & 15;
+      pk[i] = pv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + key < kend) {
+        pk[i] = kv_load4<KV>(a.kc, head + (size_t)(c0 + key) * 64 + 4 * f);
+        pv[i] = kv_load4<KV>(a.vc, head + (size_t)(c0 + key) * 64 + 4 * f);
+      }
+    }
+  };
+  load_kv(0);
+
   for (int kt = 0; kt < nkt; ++kt) {
     const int c0 = kt * kAtKeys;
     if (__syncthreads_or(!ok)) break;   // also: the previous tile's P V has been read by every thread
-    for (int idx = tid; idx < kAtKeys * 16; idx += kAtThreads) {
-      const int key = idx >> 4, f = idx & 15;
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-      if (c0 + key < kend) {
-        kv = kv_load4<KV>(a.kc, head + (size_t)(c0 + key) * 64 + 4 * f);
-        vv = kv_load4<KV>(a.vc, head + (size_t)(c0 + key) * 64 + 4 * f);
-      }
-      big |= put4(base + kAtKh, base + kAtKl, key, f, kv, kAtIn);
-      big |= put4(base + kAtVh, base + kAtVl, key, f, vv, kAtIn);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + kAtThreads * i, key = idx >> 4, f = idx & 15;
+      big |= put4(base + kAtKh, base + kAtKl, key, f, pk[i], kAtIn);
+      big |= put4(base + kAtVh, base + kAtVl, key, f, pv[i], kAtIn);
     }
+    if (kt + 1 < nkt) load_kv(c0 + kAtKeys);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -172,20 +187,19 @@ __global__ void __launch_bounds__(kAtThreads, 2) attn_prefill_tc_kernel(const At
     // a wait that runs out clears ok; the thread still takes every barrier of the iteration
     ok = mbar_wait(&bar_s, (uint32_t)(kt & 1), a.status) && ok;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    // scores of the row: both halves for the maximum, this thread's half for P
-    uint32_t s_own[32], s_oth[32];
+    // this thread's half of the row's scores; the row maximum through the partner thread
+    uint32_t s_own[32];
     tmem_ld32(tS + lane_base + (uint32_t)(half * 32), s_own);
-    tmem_ld32(tS + lane_base + (uint32_t)((1 - half) * 32), s_oth);
     tmem_ld_wait();
     const float sc = 1.f / 512.f;   // (8 q) . (8 k) / 64 / 8
-    const int cb = c0 + half * 32, co = c0 + (1 - half) * 32;
+    const int cb = c0 + half * 32;
     float mx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 32; ++j)
       if (cb + j <= qpos) mx = fmaxf(mx, __uint_as_float(s_own[j]) * sc);
-      if (co + j <= qpos) mx = fmaxf(mx, __uint_as_float(s_oth[j]) * sc);
-    }
-    const float m_new = fmaxf(m_i, mx);
+    red_m[half][r] = mx;
+    __syncthreads();
+    const float m_new = fmaxf(m_i, fmaxf(red_m[0][r], red_m[1][r]));
     const float alpha = m_new == -INFINITY ? 1.f : expf(m_i - m_new);
     m_i = m_new;
     float psum = 0.f;

@@ -427,6 +427,7 @@ cudaError_t gf_go(const Launch& L, GArgs a, int epi, const GemmWork* gw, const C
     const int nk = a.K / GK;
     if (s > nk / 2) s = nk / 2;
     if (s > 8) s = 8;
+    while (s & (s - 1)) s &= s - 1;   // a power of two: 3- and 6-CTA clusters measured slower
     if (s > 1) a.splits = s;
   }
   const dim3 grid(ntile, (a.M + BN - 1) / BN, a.splits);
@@ -525,13 +526,17 @@ cudaError_t launch_gemm_f16(const Launch& L, const WView& w, const GemmWeights& 
     cudaError_t e = map_f16(&tA, w.h, w.N, w.K, w.K, GM);
     if (e != cudaSuccess) return e;
   }
-  // tile width: the widest that still gives every SM a tile, else the narrowest
+  // tile width by rows; 256 only when even those tiles fill every SM twice
   const int ntile = (w.N + GM - 1) / GM;
   auto tiles = [&](int bn) { return ntile * ((M + bn - 1) / bn); };
   const int sms = gw ? gw->sms : 148;
+  // 128 rather than 64 unless it pads more rows: 128-row activation tiles halve the weight
+  // tiles each CTA dequantises (measured faster at 504 rows even with SMs left idle; slower at
+  // 130, where the second 128-row tile is nearly empty)
+  auto padded = [&](int b) { return (M + b - 1) / b * b; };
   int bn = 32;
   if (M > 32) bn = 64;
-  if (M > 64 && tiles(128) >= sms) bn = 128;
+  if (M > 64 && padded(128) <= padded(64)) bn = 128;
   if (M > 128 && tiles(256) >= 2 * sms) bn = 256;
   switch (bn) {
     case 32: return h ? gf_go<32, kFp16>(L, a, epi, gw, tA, xh, xl, ldx) : gf_go<32, kInt4>(L, a, epi, gw, tA, xh, xl, ldx);
