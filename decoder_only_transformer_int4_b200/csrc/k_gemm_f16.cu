@@ -144,24 +144,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const int nk = kb1 - kb0;
   bool ok = true;
 
+  pdl_trigger();
   if (warp == 0) {
     // ---- producer ----
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < nk && ok; ++kb) {
+      auto load_weights = [&](int kb) {
+        unsigned char* st = base + (size_t)(kb % NS) * LY::kStage;
+        if (FMT == kInt4)
+          bulk_g2s(st + LY::kA + 2 * LY::kBTile, a.wt + ((size_t)tile * nkb_all + kb0 + kb) * kRawA, kRawA,
+                   &full[kb % NS]);
+        else
+          tma_load_2d(st, &tmA, (kb0 + kb) * GK, n0, &full[kb % NS]);
+      };
+      auto load_acts = [&](int kb) {
+        unsigned char* st = base + (size_t)(kb % NS) * LY::kStage;
+        tma_load_2d(st + LY::kA, &tmBh, (kb0 + kb) * GK, m0, &full[kb % NS]);
+        tma_load_2d(st + LY::kA + LY::kBTile, &tmBl, (kb0 + kb) * GK, m0, &full[kb % NS]);
+      };
+      // the weights are constants: the first stages' weight copies go out before the wait for
+      // the kernel that produces the activations (programmatic dependent launch)
+      const int pre = nk < NS ? nk : NS;
+      for (int kb = 0; kb < pre; ++kb) {
+        mbar_expect_tx(&full[kb], LY::kTx);
+        load_weights(kb);
+      }
+      pdl_wait();
+      for (int kb = 0; kb < pre; ++kb) load_acts(kb);
+      int issued = pre;
+      for (int kb = pre; kb < nk && ok; ++kb) {
         const int s = kb % NS;
-        if (kb >= NS && !mbar_wait(&empty[s], (uint32_t)(((kb / NS) - 1) & 1), a.status)) {
+        if (!mbar_wait(&empty[s], (uint32_t)(((kb / NS) - 1) & 1), a.status)) {
           ok = false;
           break;
         }
-        unsigned char* st = base + (size_t)s * LY::kStage;
         mbar_expect_tx(&full[s], LY::kTx);
-        if (FMT == kInt4)
-          bulk_g2s(st + LY::kA + 2 * LY::kBTile, a.wt + ((size_t)tile * nkb_all + kb0 + kb) * kRawA, kRawA, &full[s]);
-        else
-          tma_load_2d(st, &tmA, (kb0 + kb) * GK, n0, &full[s]);
-        tma_load_2d(st + LY::kA, &tmBh, (kb0 + kb) * GK, m0, &full[s]);
-        tma_load_2d(st + LY::kA + LY::kBTile, &tmBl, (kb0 + kb) * GK, m0, &full[s]);
+        load_weights(kb);
+        load_acts(kb);
         ++issued;
       }
       // before leaving: the last copy issued into each stage has landed
@@ -232,6 +250,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
 
   // ---- epilogue (warps 2-9) ----
+  pdl_wait();   // before any global read or write of activations (returns at once by now)
   if (__syncthreads_or(!ok)) {
     if (tid == 0) flag_error(a.status, kErrTimeout);
   }
@@ -439,13 +458,22 @@ cudaError_t gf_go(const Launch& L, GArgs a, int epi, const GemmWork* gw, const C
   cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = GLayout<BN, FMT>::kBytes;
   cfg.stream = L.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = (unsigned)a.splits;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (a.splits > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = (unsigned)a.splits;
+    ++na;
+  }
+  if (L.pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = a.splits > 1 ? 1 : 0;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, k, a, tA, tBh, tBl);
   if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
   return e;
