@@ -56,6 +56,7 @@ def _args():
     ap.add_argument("--no-prefill-tensor", action="store_true",
                     help="skip the prefill GEMM tensor-pipe block")
     ap.add_argument("--no-cond", action="store_true", help="skip the conditioner block")
+    ap.add_argument("--no-w4a8", action="store_true", help="skip the W4A8 block")
     ap.add_argument("--no-pages", action="store_true",
                     help="skip the page-faithful block (kv heads = heads, fp32 and fp16 caches)")
     ap.add_argument("--decode-path", type=int, default=0, choices=[0, 1, 2],
@@ -360,6 +361,44 @@ def _batched_block(ms, torch, model, key, dev, flush, steps=2, warmup=1):
     }
 
 
+def _w4a8_block(ms, torch, model, wl, dev, flush, steps=2, warmup=1, decode_steps=256):
+    """The W4A8 option (INT8 dynamic activation codes per 32-element block, dp4a integer dot
+    products) on the benchmark's model and batch: prefill and a run of greedy decode steps on
+    the per-operation path (the persistent kernel keeps fp32-level activations), device-timed
+    with CUDA events, L2 flushed before each step.  Decode is timed alongside the fp32-activation
+    run of the same path for comparison."""
+    B, sh = wl.batch, wl.shape
+    prefix = torch.from_numpy(synth.make_prefix(sh, B, wl.prefix_len, seed=1)).to(dev)
+    start = torch.from_numpy(synth.make_start_tokens(B, seed=2).reshape(B, 1)).to(dev)
+    out = torch.empty((decode_steps, B), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {"workload": f"{_config_json(wl, 1)['workload']}; {decode_steps} decode steps per timing",
+           "decode_path": "one kernel per operation, CUDA graph per step"}
+    for name, a8 in (("w4a8", True), ("w4a32", False)):
+        cache = ms.Cache(model, B, wl.capacity)
+        cache.set_decode_path(2)
+        cache.set_act_int8(a8)
+        pre, dec = [], []
+        for i in range(warmup + steps):
+            cache.reset()
+            flush.zero_()
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            cache.prefill(start, prefix)
+            e1.record(stream)
+            cache.generate(decode_steps, out_tokens=out, logits=False)
+            e2.record(stream)
+            e2.synchronize()
+            if i >= warmup:
+                pre.append(e0.elapsed_time(e1))
+                dec.append(e1.elapsed_time(e2))
+        assert cache.device_status() == ms.MS_OK
+        res[name] = {"prefill_ms": statistics.mean(pre), "decode_ms_per_step": statistics.mean(dec) / decode_steps,
+                     "decode_tokens_per_s": B * decode_steps / (statistics.mean(dec) / 1e3)}
+        cache.close()
+    return res
+
+
 def _pages_block(ms, torch, dev, flush, steps=2, warmup=1):
     """The page-faithful medium shape (kv heads = heads = 16: the W4A32 page's 469.5 MiB
     cache at 2504 positions) at batch 1, the whole prefill + 2000-step greedy run, once with
@@ -636,7 +675,7 @@ def run_ours(a):
         roof["traffic"] = tr["bytes"]
         roof["traffic_per"] = f"one launch of {tr['tokens']} decode steps, cache lengths {t_lo}..{t_hi} (ncu)"
         roof["traffic_over_algorithmic"] = tr["bytes"] / alg
-    batched = prefill_tc = pages = cond = None
+    batched = prefill_tc = pages = cond = w4a8 = None
     if world == 1 and not a.no_batched and a.workload in _BATCHED:
         batched = _batched_block(ms, torch, model, _BATCHED[a.workload], dev, flush)
     if world == 1 and not a.no_pages and a.workload == "c3":
@@ -646,6 +685,8 @@ def run_ours(a):
         if a.workload in _BATCHED:
             rows.append(synth.WORKLOADS[_BATCHED[a.workload]].batch * (wl.prefix_len + 1))
         prefill_tc = _prefill_tensor_block(ms, torch, model, sh, rows, dev, flush)
+    if world == 1 and not a.no_w4a8 and sh.n_layers > 0 and wl.weight_format == "int4":
+        w4a8 = _w4a8_block(ms, torch, model, wl, dev, flush)
     if world == 1 and not a.no_cond:
         nb = [1] + ([synth.WORKLOADS[_BATCHED[a.workload]].batch] if a.workload in _BATCHED else [])
         cond = _cond_block(ms, torch, dev, flush, sh.d_model, nb)
@@ -676,6 +717,8 @@ def run_ours(a):
             line["pages"] = pages
         if cond is not None:
             line["conditioner"] = cond
+        if w4a8 is not None:
+            line["w4a8"] = w4a8
         print(json.dumps(line), flush=True)
     cache.close()
     model.close()

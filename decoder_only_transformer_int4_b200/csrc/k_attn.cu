@@ -4,6 +4,7 @@
 //
 // Cache layout: K and V each [B][Hk][cap][64] per layer, so the keys of one (stream,
 // kv head) are one contiguous run of 256-byte rows.
+#include <cuda_fp16.h>
 #include <math.h>
 #include "ms_device.cuh"
 #include "ms_launch.cuh"
@@ -22,6 +23,7 @@ namespace ms {
 namespace {
 constexpr int kDecThreads = 128;
 constexpr int kDecSub = 64;        // positions staged in shared memory at a time
+static_assert(kDecThreads == 2 * kDecSub && kDecSub == 64, "the score and PV loops map two thread halves onto 64 rows");
 constexpr int kMinPerSplit = 16;   // smallest run of positions worth a CTA
 constexpr int kDecTargetCtas = 6 * 148;   // several resident CTAs per SM overlap their K/V loads
 constexpr int kMaxSplits = 128;    // partials one (stream, kv head) may have
@@ -36,6 +38,9 @@ struct AttnDecArgs {
   int splits;
   float* part;
   unsigned* counters;
+  __half* oh;       // if set, the result as fp16 hi / lo planes [B][ldo] instead of fp32 o
+  __half* ol;
+  int ldo;
   float* o;
 };
 }  // namespace
@@ -51,10 +56,10 @@ int attn_decode_splits(int B, int Hk, int cap) {
 
 template <int HPG, int KV>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a) {
-  __shared__ float qs[HPG][64];
+  __shared__ __align__(16) float qs[HPG][64];
   __shared__ float Ks[kDecSub][65];
   __shared__ __align__(16) float Vs[kDecSub][64];
-  __shared__ float sc[HPG][kDecSub];
+  __shared__ __align__(16) float sc[HPG][kDecSub];
   __shared__ float mh[HPG], lh[HPG], corr[HPG];
   __shared__ float mwbuf[HPG * kMaxSplits], lbuf[HPG * kMaxSplits];
   __shared__ unsigned last;
@@ -113,19 +118,36 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
         Ks[p][4 * f + 2] = pk[j].z;
         Ks[p][4 * f + 3] = pk[j].w;
         reinterpret_cast<float4*>(&Vs[p][0])[f] = pv[j];
+      } else {
+        reinterpret_cast<float4*>(&Vs[p][0])[f] = make_float4(0.f, 0.f, 0.f, 0.f);   // read as 0 x p = 0
       }
     }
     if (c0 + kDecSub < t1) fetch(c0 + kDecSub, min(kDecSub, t1 - c0 - kDecSub));
     __syncthreads();
-    for (int i = tid; i < HPG * kDecSub; i += kDecThreads) {
-      const int h = i / kDecSub, p = i - h * kDecSub;
-      float s = -INFINITY;
-      if (p < cn) {
-        s = 0.f;
-#pragma unroll 16
-        for (int dd = 0; dd < 64; ++dd) s = fmaf(qs[h][dd], Ks[p][dd], s);
+    {
+      // thread: position p = tid % 64, heads hg, hg + 2, ... (hg = tid / 64); each K element is
+      // loaded once for all of them, q by broadcast float4 reads
+      const int p = tid & (kDecSub - 1), hg = tid / kDecSub;
+      float sacc[kSlots];
+#pragma unroll
+      for (int k = 0; k < kSlots; ++k) sacc[k] = 0.f;
+#pragma unroll 4
+      for (int dd = 0; dd < 64; dd += 4) {
+        const float k0 = Ks[p][dd], k1 = Ks[p][dd + 1], k2 = Ks[p][dd + 2], k3 = Ks[p][dd + 3];
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) {
+          const int h = hg + 2 * k;
+          if (h < HPG) {
+            const float4 q4 = *reinterpret_cast<const float4*>(&qs[h][dd]);
+            sacc[k] = fmaf(q4.x, k0, fmaf(q4.y, k1, fmaf(q4.z, k2, fmaf(q4.w, k3, sacc[k]))));
+          }
+        }
       }
-      sc[h][p] = s;
+#pragma unroll
+      for (int k = 0; k < kSlots; ++k) {
+        const int h = hg + 2 * k;
+        if (h < HPG) sc[h][p] = p < cn ? sacc[k] : -INFINITY;
+      }
     }
     __syncthreads();
     for (int h = warp; h < HPG; h += kDecThreads / 32) {
@@ -147,14 +169,24 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
       }
     }
     __syncthreads();
+    {
+      // thread: dimension dd = tid % 64 of heads hg, hg + 2, ...; each V element loaded once for
+      // all of them, the probabilities by broadcast float4 reads (rows past cn hold 0 x 0)
+      const int dd = tid & 63, hg = tid >> 6;
+      const int cn4 = (cn + 3) & ~3;
 #pragma unroll
-    for (int k = 0; k < kSlots; ++k) {
-      const int idx = tid + k * kDecThreads;
-      if (idx < HPG * 64) {
-        const int h = idx >> 6, dd = idx & 63;
-        float acc = oacc[k] * corr[h];
-        for (int p = 0; p < cn; ++p) acc = fmaf(sc[h][p], Vs[p][dd], acc);
-        oacc[k] = acc;
+      for (int k = 0; k < kSlots; ++k)
+        if (hg + 2 * k < HPG) oacc[k] *= corr[hg + 2 * k];
+      for (int p = 0; p < cn4; p += 4) {
+        const float v0 = Vs[p][dd], v1 = Vs[p + 1][dd], v2 = Vs[p + 2][dd], v3 = Vs[p + 3][dd];
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) {
+          const int h = hg + 2 * k;
+          if (h < HPG) {
+            const float4 p4 = *reinterpret_cast<const float4*>(&sc[h][p]);
+            oacc[k] = fmaf(p4.x, v0, fmaf(p4.y, v1, fmaf(p4.z, v2, fmaf(p4.w, v3, oacc[k]))));
+          }
+        }
       }
     }
   }
@@ -206,7 +238,14 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecArgs a)
     float O = 0.f;
 #pragma unroll 8
     for (int s = 0; s < s_act; ++s) O = fmaf(mwbuf[h * kMaxSplits + s], __ldcg(p0 + ((size_t)s * HPG + h) * 66 + 2 + dd), O);
-    a.o[((size_t)b * a.H + g * HPG + h) * 64 + dd] = O * Linv[h];
+    const float r = O * Linv[h];
+    if (a.oh) {
+      const __half hi = __float2half_rn(r);
+      a.oh[(size_t)b * a.ldo + (g * HPG + h) * 64 + dd] = hi;
+      a.ol[(size_t)b * a.ldo + (g * HPG + h) * 64 + dd] = __float2half_rn(r - __half2float(hi));
+    } else {
+      a.o[((size_t)b * a.H + g * HPG + h) * 64 + dd] = r;
+    }
   }
   if (tid == 0) *ctr = 0u;
 }
@@ -219,8 +258,12 @@ static cudaError_t attn_dec_go(const Launch& L, const AttnDecArgs& a, int kv16) 
 
 cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, const void* vc, int B, int H,
                                int Hk, int cap, const int* dlen, int add, const AttnDecodeWork& w, float* o,
-                               int kv16) {
+                               int kv16, __half* oh, __half* ol, int ldo) {
+  if (oh && (!ol || ldo < H * 64)) return cudaErrorInvalidValue;
   AttnDecArgs a;
+  a.oh = oh;
+  a.ol = ol;
+  a.ldo = ldo;
   a.q = q;
   a.kc = kc;
   a.vc = vc;

@@ -149,7 +149,8 @@ cudaError_t launch_cond_assemble(const Launch& L, const float* y, float yscale, 
                                  float* prefix);
 
 // Split-K decode attention over positions [0, len + add) of each (stream, kv head), with
-// the combine done by the last CTA of each (stream, kv head).
+// the combine done by the last CTA of each (stream, kv head); the result as fp32 rows o, or
+// (oh set) as fp16 hi / lo planes [B][ldo] for the O GEMM.
 struct AttnDecodeWork {
   float* part;        // [B][Hk][splits][hpg][66]
   unsigned* counters; // [B][Hk], zero between launches
@@ -157,7 +158,8 @@ struct AttnDecodeWork {
 };
 cudaError_t launch_attn_decode(const Launch& L, const float* q, const void* kc, const void* vc,
                                int B, int H, int Hk, int cap, const int* dlen, int add,
-                               const AttnDecodeWork& w, float* o, int kv16);
+                               const AttnDecodeWork& w, float* o, int kv16, __half* oh = nullptr,
+                               __half* ol = nullptr, int ldo = 0);
 int attn_decode_splits(int B, int Hk, int cap);
 
 // LM head + argmax over rows x[m * ldx], m < M.  Writes logits (may be null), argmax

@@ -338,13 +338,14 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
     }
     if (e == cudaSuccess)
       e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
-    if (e == cudaSuccess) e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o, c->kv16);
+    if (e == cudaSuccess)
+      e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o, c->kv16, gv ? nullptr : c->hh,
+                                 gv ? nullptr : c->hl, c->kh);
     if (gv) {
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[1], c->o, H * 64, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[2], c->x, d, B, ly.ln2_g, ly.ln2_b, g.ln_eps, c->u, F, ms::kGelu);
       if (e == cudaSuccess) e = ms::launch_gemv(L, ly.w[3], c->u, F, B, nullptr, nullptr, 0.f, c->x, d, ms::kAdd);
     } else {
-      if (e == cudaSuccess) e = ms::launch_split_f16(L, c->o, H * 64, B, H * 64, c->hh, c->hl, c->kh);
       if (e == cudaSuccess)
         e = ms::launch_gemm_f16(L, ly.w[1], ly.gw[1], c->hh, c->hl, c->kh, B, c->x, d, nullptr, nullptr, 0, ms::kAdd, &gw);
       if (e == cudaSuccess)
