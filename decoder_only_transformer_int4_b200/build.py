@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libms_b200.so")
-SOURCES = ["k_elementwise.cu", "k_gemv.cu", "k_gemm_f16.cu", "k_w4a8.cu", "k_attn.cu", "k_attn_tc.cu", "k_decode_persistent.cu", "k_cond.cu", "ms_runtime.cu",
+SOURCES = ["k_elementwise.cu", "k_gemv.cu", "k_gemm_f16.cu", "k_w4a8.cu", "k_gemm_i8.cu", "k_attn.cu", "k_attn_tc.cu", "k_decode_persistent.cu", "k_cond.cu", "ms_runtime.cu",
            "ms_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -415,6 +415,24 @@ EncodeTiled encoder() {
   return fn;
 }
 
+}  // namespace
+
+cudaError_t encode_map_2d(CUtensorMap* m, CUtensorMapDataType type, const void* ptr, uint64_t cols, uint64_t rows,
+                          uint64_t stride_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiled enc = encoder();
+  if (!enc) return cudaErrorNotSupported;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || stride_bytes % 16 != 0) return cudaErrorInvalidValue;
+  const cuuint64_t dim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t stride[1] = {(cuuint64_t)stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, type, 2, const_cast<void*>(ptr), dim, stride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+
 // 2-D fp16 tensor [rows][cols] (row stride ld halves) in boxes of 64 columns x box_rows rows,
 // 128-byte swizzle; out-of-range rows read as zero.
 cudaError_t map_f16(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_rows) {

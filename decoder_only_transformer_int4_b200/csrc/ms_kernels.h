@@ -113,6 +113,13 @@ cudaError_t launch_quantize_act_int8(const Launch& L, const float* x, int ldx, i
 cudaError_t launch_matmul_w4a8(const Launch& L, const WView& w, const int8_t* qa, int ldqa, const float* sa, int ldsa,
                                int M, float* y, int ldy, int epi, int sms);
 cudaError_t init_attrs_w4a8();
+// The same MatMul on tcgen05 (kind::i8, one int32 TMEM result per 32-wide block, scaled while
+// the next stage's MMAs run) for M >= 128, reading the weights from the tcgen05 f16 GEMM's
+// tile-packed copy (g); qa and sa 16-byte aligned, ldqa a multiple of 16, ldsa of 4.
+bool w4a8_tc_fits(const WView& w, int M, int ldqa, int ldsa);
+cudaError_t launch_matmul_w4a8_tc(const Launch& L, const WView& w, const GemmWeights& g, const int8_t* qa, int ldqa,
+                                  const float* sa, int ldsa, int M, float* y, int ldy, int epi);
+cudaError_t init_attrs_w4a8_tc();
 
 // Causal prefill attention on the tensor cores (tcgen05, fp16 hi / lo operands, three products):
 // q [B * n][H * 64] post-RoPE, the layer's cache slices, positions len .. len + n - 1 with len

@@ -146,6 +146,7 @@ cudaError_t ensure_kernel_attributes() {
   if (e == cudaSuccess) e = ms::init_attrs_w4a8();
   if (e == cudaSuccess) e = ms::init_attrs_cond();
   if (e == cudaSuccess) e = ms::init_attrs_attn_tc();
+  if (e == cudaSuccess) e = ms::init_attrs_w4a8_tc();
   if (e == cudaSuccess) g_attr_done[dev] = 1;
   return e;
 }
@@ -229,11 +230,13 @@ void* kv_layer(const ms_cache* c, void* base, int l) {
 }
 
 // W4A8: quantise fp32 rows x [R][ldx] (K columns) to the cache's INT8 codes, then MatMul i.
-cudaError_t w4a8(const ms::Launch& L, ms_cache* c, const ms::WView& w, const float* x, int ldx, int R, float* y,
-                 int ldy, int epi) {
+cudaError_t w4a8(const ms::Launch& L, ms_cache* c, const ms::WView& w, const ms::GemmWeights& g, const float* x, int ldx,
+                 int R, float* y, int ldy, int epi) {
   cudaError_t e = ms::launch_quantize_act_int8(L, x, ldx, R, w.K, c->qa, c->ka, c->sa, c->ka / 32);
-  if (e == cudaSuccess) e = ms::launch_matmul_w4a8(L, w, c->qa, c->ka, c->sa, c->ka / 32, R, y, ldy, epi, c->nsm);
-  return e;
+  if (e != cudaSuccess) return e;
+  if (g.wt && ms::w4a8_tc_fits(w, R, c->ka, c->ka / 32))
+    return ms::launch_matmul_w4a8_tc(L, w, g, c->qa, c->ka, c->sa, c->ka / 32, R, y, ldy, epi);
+  return ms::launch_matmul_w4a8(L, w, c->qa, c->ka, c->sa, c->ka / 32, R, y, ldy, epi, c->nsm);
 }
 
 // ---- one decoder call, kernel by kernel ----------------------------------------------
@@ -253,15 +256,15 @@ cudaError_t run_prefill(ms_model* m, ms_cache* c, const int64_t* tokens, int S, 
     void* kc = kv_layer(c, c->k, l);
     void* vc = kv_layer(c, c->v, l);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, l == 0 ? nullptr : c->y, ly.ln1_g, ly.ln1_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], c->h, d, R, c->qkv, nq, ms::kStore);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], ly.gw[0], c->h, d, R, c->qkv, nq, ms::kStore);
     if (e == cudaSuccess)
       e = ms::launch_rope_append(L, c->qkv, B, n, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
     if (e == cudaSuccess)
       e = ms::launch_attn_prefill_tc(L, c->q, kc, vc, B, n, H, Hk, c->cap, c->dlen, c->o, nullptr, nullptr, 0, c->kv16);
-    if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], c->o, H * 64, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], ly.gw[1], c->o, H * 64, R, c->y, d, ms::kStore);
     if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, c->y, ly.ln2_g, ly.ln2_b, g.ln_eps, R, d, c->h);
-    if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], c->h, d, R, c->u, F, ms::kGelu);
-    if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], c->u, F, R, c->y, d, ms::kStore);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], ly.gw[2], c->h, d, R, c->u, F, ms::kGelu);
+    if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], ly.gw[3], c->u, F, R, c->y, d, ms::kStore);
   }
   for (int l = 0; l < g.n_layers && e == cudaSuccess && !c->act_int8; ++l) {
     const DevLayer& ly = m->layers[l];
@@ -317,15 +320,15 @@ cudaError_t run_decode(ms_model* m, ms_cache* c, const int32_t* tokens, float* l
     if (c->act_int8) {
       // W4A8: each backbone MatMul on the INT8 codes of its fp32 input
       e = ms::launch_skipln(L, c->x, nullptr, ly.ln1_g, ly.ln1_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], c->h, d, B, c->qkv, nq, ms::kStore);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[0], ly.gw[0], c->h, d, B, c->qkv, nq, ms::kStore);
       if (e == cudaSuccess)
         e = ms::launch_rope_append(L, c->qkv, B, 1, H, Hk, c->cosv, c->sinv, c->dlen, c->q, kc, vc, c->cap, c->kv16);
       if (e == cudaSuccess)
         e = ms::launch_attn_decode(L, c->q, kc, vc, B, H, Hk, c->cap, c->dlen, 1, aw, c->o, c->kv16);
-      if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], c->o, H * 64, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[1], ly.gw[1], c->o, H * 64, B, c->x, d, ms::kAdd);
       if (e == cudaSuccess) e = ms::launch_skipln(L, c->x, nullptr, ly.ln2_g, ly.ln2_b, g.ln_eps, B, d, c->h);
-      if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], c->h, d, B, c->u, F, ms::kGelu);
-      if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], c->u, F, B, c->x, d, ms::kAdd);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[2], ly.gw[2], c->h, d, B, c->u, F, ms::kGelu);
+      if (e == cudaSuccess) e = w4a8(L, c, ly.w[3], ly.gw[3], c->u, F, B, c->x, d, ms::kAdd);
       continue;
     }
     if (gv) {
@@ -1157,6 +1160,21 @@ ms_status ms_op_matmul_w4a8(const int8_t* qa, const float* sa, int M, int K, con
   CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
   ms::WView w{packed, scales, nullptr, N, K, ms::kInt4, K / 2, K / 32};
   ms::Launch L{(cudaStream_t)stream, false, nullptr};
+  if (ms::w4a8_tc_fits(w, M, K, K / 32) && !(reinterpret_cast<uintptr_t>(sa) & 15)) {
+    // the tcgen05 kernel reads the tile-packed copy, made in stream-ordered temporaries
+    const size_t tiles = ms::gemm_tiles_bytes(w), rows = ms::gemm_rows_padded(w);
+    char* tmp = nullptr;
+    CUDA_TRY(cudaMallocAsync(reinterpret_cast<void**>(&tmp), round_up(tiles, 256) + 2 * round_up(rows * 4, 256),
+                             (cudaStream_t)stream));
+    ms::GemmWeights g{reinterpret_cast<unsigned char*>(tmp), reinterpret_cast<float*>(tmp + round_up(tiles, 256))};
+    float* rexp = reinterpret_cast<float*>(tmp + round_up(tiles, 256) + round_up(rows * 4, 256));
+    cudaError_t e = ms::launch_gemm_repack(w, g, rexp, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = ms::launch_matmul_w4a8_tc(L, w, g, qa, K, sa, K / 32, M, y, N, ms::kStore);
+    const cudaError_t ef = cudaFreeAsync(tmp, (cudaStream_t)stream);
+    if (e != cudaSuccess) return check_launch(e, "matmul_w4a8 (tcgen05)");
+    CUDA_TRY(ef);
+    return MS_OK;
+  }
   return check_launch(ms::launch_matmul_w4a8(L, w, qa, K, sa, K / 32, M, y, N, ms::kStore, nsm > 0 ? nsm : 1),
                       "matmul_w4a8");
 }

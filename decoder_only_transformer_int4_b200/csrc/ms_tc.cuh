@@ -3,6 +3,7 @@
 // fp16 hi / lo packing of fp32 operands.
 #pragma once
 #include <cuda.h>
+#include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -81,6 +82,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+// Host: a 2-D tiled TMA map of [rows][cols] elements of `type` (row stride in bytes, a multiple
+// of 16; base 16-byte aligned); out-of-range elements read as zero.
+cudaError_t encode_map_2d(CUtensorMap* m, CUtensorMapDataType type, const void* ptr, uint64_t cols, uint64_t rows,
+                          uint64_t stride_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 }  // namespace ms

@@ -48,7 +48,7 @@ def test_act_int8_codes_bit_exact():
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 8, 3, 64, 130])
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 3, 64, 129, 130, 504])
 @pytest.mark.parametrize("N,K", [(1536, 1024), (1024, 4096), (200, 512)])
 def test_matmul_w4a8(M, N, K):
     w = synth.make_matrix(N, K, seed=700 + K)
