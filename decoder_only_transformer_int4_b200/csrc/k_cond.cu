@@ -42,6 +42,10 @@ __device__ __forceinline__ int dif_pos(int k, int half) {
   return p;
 }
 
+// Shared-memory slot of complex element p: one 16-byte pad after every 8 elements, so that the
+// strided and digit-reversed accesses of the stages and the split spread over the banks.
+__device__ __forceinline__ int zi(int p) { return p + (p >> 3); }
+
 __device__ __forceinline__ double2 cmul(double2 a, double2 w) {
   return make_double2(a.x * w.x - a.y * w.y, a.x * w.y + a.y * w.x);
 }
@@ -71,8 +75,8 @@ __global__ void __launch_bounds__(256) log_mel_kernel(const float* __restrict__ 
                                                       __half* __restrict__ xl) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int half = c.n_fft >> 1, q4 = half >> 2;
-  double2* z = reinterpret_cast<double2*>(smem_raw);            // [half]
-  double* mag = reinterpret_cast<double*>(z + half);            // [half + 1]
+  double2* z = reinterpret_cast<double2*>(smem_raw);            // [half + half / 8], element p at zi(p)
+  double* mag = reinterpret_cast<double*>(z + half + half / 8); // [half + 1]
   const int t = blockIdx.x, b = blockIdx.y;
   const float* x = audio + (size_t)b * n_samples;
   // z[n] = (f[2n], f[2n+1]), f = window x the frame; the first radix-4 stage (span = half) is
@@ -94,38 +98,38 @@ __global__ void __launch_bounds__(256) log_mel_kernel(const float* __restrict__ 
     for (int t1 = threadIdx.x; t1 < q4; t1 += blockDim.x) {
       double2 a0 = frame_pair(t1), a1 = frame_pair(t1 + q4), a2 = frame_pair(t1 + 2 * q4), a3 = frame_pair(t1 + 3 * q4);
       dif4(a0, a1, a2, a3, t1, c.n_fft / half, c.twiddle);
-      z[t1] = a0, z[t1 + q4] = a1, z[t1 + 2 * q4] = a2, z[t1 + 3 * q4] = a3;
+      z[zi(t1)] = a0, z[zi(t1 + q4)] = a1, z[zi(t1 + 2 * q4)] = a2, z[zi(t1 + 3 * q4)] = a3;
     }
     span = q4;
   } else {
-    for (int n = threadIdx.x; n < half; n += blockDim.x) z[n] = frame_pair(n);
+    for (int n = threadIdx.x; n < half; n += blockDim.x) z[zi(n)] = frame_pair(n);
   }
   __syncthreads();
   for (; span >= 4; span >>= 2) {
     const int L4 = span >> 2, tstep = c.n_fft / span;
     for (int i = threadIdx.x; i < q4; i += blockDim.x) {
       const int t1 = i % L4, base = (i / L4) * span + t1;
-      double2 a0 = z[base], a1 = z[base + L4], a2 = z[base + 2 * L4], a3 = z[base + 3 * L4];
+      double2 a0 = z[zi(base)], a1 = z[zi(base + L4)], a2 = z[zi(base + 2 * L4)], a3 = z[zi(base + 3 * L4)];
       dif4(a0, a1, a2, a3, t1, tstep, c.twiddle);
-      z[base] = a0, z[base + L4] = a1, z[base + 2 * L4] = a2, z[base + 3 * L4] = a3;
+      z[zi(base)] = a0, z[zi(base + L4)] = a1, z[zi(base + 2 * L4)] = a2, z[zi(base + 3 * L4)] = a3;
     }
     __syncthreads();
   }
   if (span == 2) {                                              // a last radix-2 stage
     for (int i = threadIdx.x; i < (half >> 1); i += blockDim.x) {
-      const double2 a0 = z[2 * i], a1 = z[2 * i + 1];
-      z[2 * i] = make_double2(a0.x + a1.x, a0.y + a1.y);
-      z[2 * i + 1] = make_double2(a0.x - a1.x, a0.y - a1.y);
+      const double2 a0 = z[zi(2 * i)], a1 = z[zi(2 * i + 1)];
+      z[zi(2 * i)] = make_double2(a0.x + a1.x, a0.y + a1.y);
+      z[zi(2 * i + 1)] = make_double2(a0.x - a1.x, a0.y - a1.y);
     }
     __syncthreads();
   }
   // X[k] = E[k] + e^{-2 pi i k / n_fft} O[k], E and O the spectra of the even and odd samples
   for (int k = threadIdx.x; k <= half; k += blockDim.x) {
     if (k == 0 || k == half) {
-      const double2 z0 = z[0];
+      const double2 z0 = z[zi(0)];
       mag[k] = fabs(k == 0 ? z0.x + z0.y : z0.x - z0.y);
     } else {
-      const double2 a = z[dif_pos(k, half)], cz = z[dif_pos(half - k, half)];
+      const double2 a = z[zi(dif_pos(k, half))], cz = z[zi(dif_pos(half - k, half))];
       const double er = 0.5 * (a.x + cz.x), ei = 0.5 * (a.y - cz.y);     // (a + conj(cz)) / 2
       const double orr = 0.5 * (a.y + cz.y), oi = -0.5 * (a.x - cz.x);  // (a - conj(cz)) / 2i
       const double2 w = __ldg(c.twiddle + k);
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(256) cond_assemble_kernel(const float* __restr
 }  // namespace
 
 size_t log_mel_smem_bytes(int n_fft) {
-  return (size_t)(n_fft / 2) * sizeof(double2) + (size_t)(n_fft / 2 + 1) * sizeof(double);
+  return (size_t)(n_fft / 2 + n_fft / 16) * sizeof(double2) + (size_t)(n_fft / 2 + 1) * sizeof(double);
 }
 
 cudaError_t init_attrs_cond() { return allow_smem(log_mel_kernel, log_mel_smem_bytes(kCondMaxFft)); }
