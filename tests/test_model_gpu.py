@@ -61,6 +61,7 @@ TINY = [
     (2, 256, 4, 1, 512, 1393),
     (1, 768, 12, 4, 1024, 500),     # 3 query heads per kv head
     (1, 512, 8, 1, 512, 257),       # 8 query heads per kv head
+    (1, 768, 12, 2, 1024, 500),     # 6 query heads per kv head: 6 x 21 of a 128-row prefill tile used
 ]
 
 
