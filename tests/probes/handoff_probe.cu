@@ -82,7 +82,7 @@ __global__ void probe_kernel(int mode, int rounds, int width, uint64_t* words, d
   }
   uint64_t t0 = 0;
   for (int r = 1; r <= rounds; ++r) {
-    if (r == 2) t0 = gtime();   // round 1 lines the CTAs up
+    if (r == 2) t0 = gtime();   // the first pass lines the CTAs up
     const uint32_t ep = mode == 2 ? 1u : (uint32_t)r;
     if (mode == 1)
       for (int i = tid; i < width; i += blockDim.x) st_word(words + (size_t)c * width + i, (uint32_t)c, ep);
