@@ -175,3 +175,60 @@ def test_late_c5_large_16_streams():
 def test_late_c4_medium_64_streams():
     wl = synth.WORKLOADS["c4"]
     _late_window(wl.shape, "int4", wl.batch, wl.capacity, wl.capacity - 32, 32, [0, 21, 42, 63], 2)
+
+
+@pytest.mark.parametrize("dims,kv_format", [
+    ((2, 512, 8, 2, 1024), ms.MS_KV_F32),   # 4 query heads per kv head: 32 new rows per tile
+    ((2, 768, 12, 4, 1024), ms.MS_KV_F16),  # 3 per kv head (42 rows per tile), half-precision cache
+    ((1, 256, 4, 4, 512), ms.MS_KV_F32),    # 1 per kv head: 128 rows per tile
+])
+def test_prefill_onto_a_long_cache(dims, kv_format):
+    """Prefill of 200 token rows onto an imported cache of 2000 positions (two streams): each
+    new row attends over 2000+ keys, i.e. 32 and more key tiles of the tensor-core prefill
+    attention, with the causal offset of its position and a ragged last tile.  Last-position
+    logits within 2e-3 of the oracle given the same cache; the rows the prefill appended
+    (post-RoPE k, v) against the oracle's.  With the half cache the imported state is rounded
+    to halves on both sides first, and the oracle stores each new key and value as its half."""
+    L, d, H, Hk, F = dims
+    sh = synth.Shape("late-prefill", L, d, H, Hk, F, vocab=300)
+    half = kv_format == ms.MS_KV_F16
+    draw = synth.make_weights(sh, seed=0, std=0.05, ln_random=True)
+    om = O.OracleModel(draw, "int4", kv_store="fp16" if half else "fp32")
+    gm = ms.Model.from_draw(draw, "int4")
+    T, S, cap, B = 2000, 200, 2304, 2
+    k, v = synth.make_kv_cache(sh, B, T, seed=4)
+    if half:
+        k, v = k.astype(np.float16).astype(np.float32), v.astype(np.float16).astype(np.float32)
+    g = torch.Generator().manual_seed(3)
+    toks = torch.randint(0, sh.vocab, (B, S), generator=g, dtype=torch.int64).numpy()
+    cache = ms.Cache(gm, B, cap, kv_format=kv_format)
+    cache.import_(k, v)
+    lg, _ = cache.prefill(_dev(toks), None)
+    assert cache.device_status() == ms.MS_OK
+    assert cache.length == T + S
+    ke, ve = cache.export()
+    got = lg.cpu().numpy()
+    for b in range(B):
+        oc = om.new_cache(cap)
+        oc.load(k[:, b], v[:, b])
+        ref = om.prefill(oc, None, [int(t) for t in toks[b]])
+        assert np.abs(got[b] - ref).max() <= TOL, (dims, b, float(np.abs(got[b] - ref).max()))
+        ok_, ov_ = oc.export()
+        # appended rows.  fp32: the two sides' rounding.  Halves: layer 0's keys and values agree
+        # before rounding up to the prefill GEMM's absolute error (22-bit operands: about
+        # 2^-22 sum |x w|, a few 1e-6 here, which matters where cancellation leaves a key near
+        # zero), so the two roundings to half differ by one half ulp plus that; deeper layers'
+        # inputs already carry the previous layers' half-cache rounding differences (attention
+        # over 2000 + 200 rounded keys: a few 1e-4 on a layer-1 key), bounded by half the
+        # decoder's 2e-3 logits bar.  A wrong position, head or rotation moves values by O(1).
+        for name, got_kv, ref_kv in (("k", ke[:, b, T:], ok_[:, 0, T:]), ("v", ve[:, b, T:], ov_[:, 0, T:])):
+            mag = np.maximum(np.abs(got_kv), np.abs(ref_kv))
+            for l in range(L):
+                if half:
+                    bound = 2.0 ** -10 * mag[l] + 1e-5 if l == 0 else 2.0 ** -8 * mag[l] + 1e-3
+                else:
+                    bound = 1e-5 * mag[l] + 1e-4
+                err = np.abs(got_kv[l] - ref_kv[l])
+                w = np.unravel_index(np.argmax(err - bound), err.shape)
+                assert np.all(err <= bound), (dims, b, name, l, w, float(got_kv[l][w]), float(ref_kv[l][w]),
+                                              float(bound[w]), int((err > bound).sum()))
