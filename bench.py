@@ -399,6 +399,55 @@ def _w4a8_block(ms, torch, model, wl, dev, flush, steps=2, warmup=1, decode_step
     return res
 
 
+def _e2e_audio_block(ms, torch, cache, wl, dev, flush, start_h, out_tok, steps=2, warmup=1):
+    """The pages' pipeline end to end through the public API: a 5-s 440 Hz clip (fp32 at 16 kHz)
+    copied in from pinned host memory with its dataset and instrument ids, the conditioner (the
+    stand-in buffers of synth.make_cond_weights) making the decoder's 501 + 1 + 1 prefix rows,
+    prefill with the start token, the greedy decode, the tokens copied back; CUDA events around
+    all of it, L2 flushed before each step."""
+    B, sh = wl.batch, wl.shape
+    if wl.prefix_len != 503:
+        return None
+    cond = ms.Conditioner.from_draw(synth.make_cond_weights(sh.d_model), synth.N_SAMPLES, synth.HOP, max_batch=B,
+                                    device=dev.index or 0)
+    audio_h = torch.from_numpy(synth.make_tone(B)).pin_memory()
+    ds_h = torch.ones(B, dtype=torch.int32).pin_memory()
+    inst_h = torch.zeros((B, 1), dtype=torch.int32).pin_memory()
+    audio, ds, inst = audio_h.to(dev), ds_h.to(dev), inst_h.to(dev)
+    start = start_h.to(dev)
+    prefix = torch.empty((B, cond.rows(1), sh.d_model), dtype=torch.float32, device=dev)
+    out_h = torch.empty((wl.decode_steps, B), dtype=torch.int32).pin_memory()
+    am_h = torch.empty((B,), dtype=torch.int32).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for i in range(warmup + steps):
+        cache.reset()
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        audio.copy_(audio_h, non_blocking=True)
+        ds.copy_(ds_h, non_blocking=True)
+        inst.copy_(inst_h, non_blocking=True)
+        start.copy_(start_h, non_blocking=True)
+        cond(audio, ds, inst, out=prefix)
+        _, am = cache.prefill(start, prefix)
+        cache.generate(wl.decode_steps, out_tokens=out_tok, logits=False)
+        am_h.copy_(am, non_blocking=True)
+        out_h.copy_(out_tok, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    assert cond.device_status() == ms.MS_OK and cache.device_status() == ms.MS_OK
+    cond.close()
+    ms_step = statistics.mean(times)
+    return {"value": B * (wl.decode_steps + 1) / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step,
+            "steps": steps, "warmup": warmup,
+            "h2d_bytes_per_step": audio_h.numel() * 4 + ds_h.numel() * 4 + inst_h.numel() * 4 + start_h.numel() * 8,
+            "d2h_bytes_per_step": out_h.numel() * 4 + am_h.numel() * 4,
+            "pipeline": "audio 5 s at 16 kHz -> conditioner -> prefill 503+1 -> greedy decode -> tokens"}
+
+
 def _pages_block(ms, torch, dev, flush, steps=2, warmup=1):
     """The page-faithful medium shape (kv heads = heads = 16: the W4A32 page's 469.5 MiB
     cache at 2504 positions) at batch 1, the whole prefill + 2000-step greedy run, once with
@@ -654,6 +703,10 @@ def run_ours(a):
     e2e_job_ms = max_over_ranks(statistics.mean(e2e_ms), dev) if e2e_ms else None
     e2e_val = world * tokens_per_step / (e2e_job_ms / 1e3) if e2e_job_ms else None
 
+    e2e_audio = None
+    if world == 1 and not a.no_e2e:
+        e2e_audio = _e2e_audio_block(ms, torch, cache, wl, dev, flush, start_h, out_tok)
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         v, dt, threads, sample, _, _ = _oracle_sample(wl, a.cpu_decode_steps)
@@ -719,6 +772,8 @@ def run_ours(a):
             line["conditioner"] = cond
         if w4a8 is not None:
             line["w4a8"] = w4a8
+        if e2e_audio is not None:
+            line["e2e_audio"] = e2e_audio
         print(json.dumps(line), flush=True)
     cache.close()
     model.close()
